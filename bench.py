@@ -1,0 +1,431 @@
+"""Benchmark of the HGA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--batch B]
+    python bench.py --impl reference ...      # the float64 CPU oracle, timed on host cores
+
+One step = one decode step of one attention layer for the whole batch: append
+the new token's summary rows, route chunks, route groups, attend (steps 1-5 of
+the HGA hot path), on inputs already resident in HBM.  L2 is flushed (a 256 MB
+write) before every timed step, outside the timed events.  Prints one JSON line.
+
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch of
+independent sequences (weak scaling, no collective on the data path); the
+step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import hga_synth as S  # noqa: E402
+
+METRIC = "HGA decode tokens/s + attn µs/layer at 32K–128K ctx; % HBM roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
+    ap.add_argument("--workload", default="llama3_8b_decode_32k")
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- byte counts
+
+def step_bytes(wl: S.Workload) -> dict:
+    """Algorithmic HBM bytes of one decode step per kernel (whole batch).
+
+    route_chunks: the candidate chunk-summary rows (fp32) + the G query rows;
+    route_groups: the groups of the kc selected chunks + query rows + chunk ids;
+    attend: K and V rows of the T routed tokens + query rows + output (fp32);
+    summaries: the closing chunk's and group's key rows + the rows written.
+    """
+    e = 2 if wl.dtype == "bf16" else 4
+    d, g = wl.head_dim, wl.gqa
+    p = wl.context - 1
+    cur = p // wl.chunk
+    n_cand = max(0, cur - wl.local - wl.sink)
+    kc = min(wl.topk_chunks, n_cand)
+    ng = wl.chunk // wl.group
+    kg = min(wl.topk_groups, kc * ng)
+    forced = (min(wl.sink, max(0, cur - wl.local)) * wl.chunk + (p - max(0, cur - wl.local) * wl.chunk + 1))
+    t = forced + kg * wl.group
+    units = wl.batch * wl.heads_kv
+    qrow = g * d * e
+    closes_chunk = (p + 1) % wl.chunk == 0
+    closes_group = (p + 1) % wl.group == 0
+    summ = 0
+    if closes_chunk:
+        summ = wl.chunk * d * e + (d + ng * d) * 4
+    elif closes_group:
+        summ = wl.group * d * e + d * 4
+    return dict(
+        summaries=units * summ,
+        route_chunks=units * (n_cand * d * 4 + qrow),
+        route_groups=units * (kc * ng * d * 4 + qrow + wl.topk_chunks * 4),
+        attend=units * (t * d * e * 2 + qrow + g * d * 4 + wl.topk_groups * 4),
+        tokens=t,
+    )
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv:
+            self._t.join()
+
+    def report(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CUDA arm
+
+def run_hga(args, rank: int, world: int):
+    import torch
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    from hierarchical_sparse_attention_hga_b200.build import build
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    build()
+    B.load_library()
+    wl = S.workload(args.workload)
+    if args.batch:
+        wl = wl.with_(batch=args.batch)
+    if wl.prefill:
+        raise SystemExit("the decode bench takes a decode workload")
+    dev = torch.device("cuda")
+    seed = S.seed_for(list(S.WORKLOADS).index(args.workload)) + 7919 * rank
+    x = S.make_inputs(wl, seed)
+    n = wl.context
+    p = n - 1
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16 if wl.dtype == "bf16" else np.float32))
+        return (t.view(torch.bfloat16) if wl.dtype == "bf16" else t).to(dev)
+
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    pos = torch.as_tensor(x["pos"], device=dev)
+    layer = B.Layer(batch=wl.batch, heads_q=wl.heads_q, heads_kv=wl.heads_kv, head_dim=wl.head_dim,
+                    chunk=wl.chunk, group=wl.group, sink_chunks=wl.sink, local_chunks=wl.local,
+                    topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
+                    n_high_pairs=wl.n_high_pairs, rope_theta=wl.rope_theta,
+                    dtype=B.HGA_BF16 if wl.dtype == "bf16" else B.HGA_F32, out_dtype=B.HGA_F32)
+    bh = wl.batch * wl.heads_kv
+    nc, ng = n // wl.chunk, wl.chunk // wl.group
+    cs = torch.empty(bh, nc, wl.head_dim, device=dev)
+    gs = torch.empty(bh, nc, ng, wl.head_dim, device=dev)
+    ci = torch.empty(bh, wl.topk_chunks, dtype=torch.int32, device=dev)
+    gi = torch.empty(bh, wl.topk_groups, dtype=torch.int32, device=dev)
+    out = torch.empty(wl.batch, wl.heads_q, 1, wl.head_dim, device=dev)
+    lse = torch.empty(wl.batch, wl.heads_q, 1, device=dev)
+    wsb = B.hga_workspace_size(layer, n, 1)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    # prefix summaries (setup, untimed): every row closed before the new token
+    B.hga_build_summaries(layer, k, n, 0, p, cs, gs, stream=sh)
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+
+    def step(record: bool):
+        if record:
+            ev[0].record(stream)
+        B.hga_build_summaries(layer, k, n, p, p + 1, cs, gs, stream=sh)
+        if record:
+            ev[1].record(stream)
+        B.hga_route_chunks(layer, q, 1, pos, cs, n, ci, stream=sh)
+        if record:
+            ev[2].record(stream)
+        B.hga_route_groups(layer, q, 1, pos, gs, n, ci, gi, stream=sh)
+        if record:
+            ev[3].record(stream)
+        B.hga_attend(layer, q, 1, pos, k, v, n, gi, out, lse, ws, wsb, stream=sh)
+        if record:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(False)
+    torch.cuda.synchronize()
+    assert B.hga_device_status(sh) == 0
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    per = {"step": [], "summaries": [], "route_chunks": [], "route_groups": [], "attend": []}
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            step(True)
+            ev[4].synchronize()
+            per["step"].append(ev[0].elapsed_time(ev[4]))
+            per["summaries"].append(ev[0].elapsed_time(ev[1]))
+            per["route_chunks"].append(ev[1].elapsed_time(ev[2]))
+            per["route_groups"].append(ev[2].elapsed_time(ev[3]))
+            per["attend"].append(ev[3].elapsed_time(ev[4]))
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = {kk: sum(vv) / len(vv) for kk, vv in per.items()}
+    ms_step = ms["step"]
+    if dist:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    # ---- e2e: host (pinned) q and new K/V rows in, output back, every step
+    q_host = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).pin_memory() \
+        if wl.dtype == "bf16" else torch.from_numpy(x["q"]).pin_memory()
+    kv_new = torch.empty(2, wl.batch, wl.heads_kv, wl.head_dim, dtype=k.dtype).pin_memory()
+    kv_new[0].copy_(k[:, :, p].cpu())
+    kv_new[1].copy_(v[:, :, p].cpu())
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    qv = q.view(torch.int16) if wl.dtype == "bf16" else q
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e = []
+    for i in range(args.warmup + min(args.steps, 200)):
+        flush.zero_()
+        e0.record(stream)
+        qv.copy_(q_host, non_blocking=True)
+        k[:, :, p].copy_(kv_new[0], non_blocking=True)
+        v[:, :, p].copy_(kv_new[1], non_blocking=True)
+        step(False)
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= args.warmup:
+            e2e.append(e0.elapsed_time(e1))
+    ms_e2e = sum(e2e) / len(e2e)
+    if dist:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    h2d = q_host.numel() * q_host.element_size() + kv_new.numel() * kv_new.element_size()
+    d2h = out_host.numel() * out_host.element_size()
+
+    nb = step_bytes(wl)
+    kern = max(("route_chunks", "route_groups", "attend", "summaries"), key=lambda kk: ms[kk])
+    hbm, peak_kind = peaks()
+    achieved = nb[kern] / (ms[kern] * 1e-3) / 1e9
+    total_bytes = nb["summaries"] + nb["route_chunks"] + nb["route_groups"] + nb["attend"]
+    nsplit_combine = 1 if wsb > 0 else 0
+    launches_per_step = 1 + 1 + 1 + 1 + nsplit_combine
+    tokens = wl.batch * world
+    line = {
+        "metric": METRIC,
+        "value": tokens / (ms_step * 1e-3),
+        "unit": "decode tokens/s (one attention layer)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "attn_us_per_layer": ms_step * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 K/V, fp32 accumulation" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) q/k/v; 2 needle chunks per KV head)",
+        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": n,
+                   "heads_q": wl.heads_q, "heads_kv": wl.heads_kv, "head_dim": wl.head_dim,
+                   "chunk": wl.chunk, "group": wl.group, "sink": wl.sink, "local": wl.local,
+                   "topk_chunks": wl.topk_chunks, "topk_groups": wl.topk_groups,
+                   "tokens_attended_per_kv_head": nb["tokens"],
+                   "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": f"replicas x{world} (independent sequences per GPU)"},
+        "per_kernel_us": {kk: ms[kk] * 1e3 for kk in ("summaries", "route_chunks", "route_groups", "attend")},
+        "step_hbm_bytes": total_bytes,
+        "step_hbm_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
+        "roofline": {"kernel": kern, "bound": "hbm", "achieved": achieved, "peak": hbm,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "algorithmic_bytes": nb[kern]},
+        "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "decode tokens/s (one attention layer)",
+                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.report(),
+    }
+    return line, wl, seed, x
+
+
+# ------------------------------------------------------------ oracle (CPU) arm
+
+def oracle_decode_rate(wl: S.Workload, seed: int, budget_s: float, x=None):
+    """Oracle decode step, timed per (sequence, KV head) unit on a bounded sample.
+
+    Per unit: summaries of the rows the new token closes, level-1 and level-2
+    routing, token set and exact attention of the G query heads.  The prefix
+    summaries are built before timing (they are state, not step work).
+    Returns (tokens/s for the whole batch, sample description, threads used).
+    """
+    from threadpoolctl import threadpool_limits
+
+    from oracle import hga_oracle as O
+    prm = O.HGAParams(head_dim=wl.head_dim, heads_q=wl.heads_q, heads_kv=wl.heads_kv,
+                      chunk=wl.chunk, group=wl.group, sink=wl.sink, local=wl.local,
+                      topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
+                      n_high_pairs=wl.n_high_pairs, rope_theta=wl.rope_theta)
+    p = wl.context - 1
+    cur = p // wl.chunk
+    g = wl.gqa
+    times = []
+    spent = 0.0
+    units = [(b, h) for b in range(wl.batch) for h in range(wl.heads_kv)]
+    with threadpool_limits(limits=1):
+        for b, h in units:
+            if spent >= budget_s:
+                break
+            if x is not None:
+                qb, kb, vb = x["q"][b, h * g:(h + 1) * g], x["k"][b, h], x["v"][b, h]
+            else:
+                q1 = S.query_slice(wl, seed, b, 1)
+                qb = q1[h * g:(h + 1) * g]
+                kb, vb = S.key_slice(wl, seed, b, h, q1), S.value_slice(wl, seed, b, h)
+            q64, k64, v64 = S.widen(qb, wl.dtype), S.widen(kb, wl.dtype), S.widen(vb, wl.dtype)
+            cs, gs = O.build_summaries(k64[:cur * wl.chunk], prm)
+            cs = np.concatenate([cs, np.full((1, wl.head_dim), np.nan)])
+            gs = np.concatenate([gs, np.full((1, gs.shape[1], wl.head_dim), np.nan)])
+            t0 = time.perf_counter()
+            c0 = cur * wl.chunk
+            cs[cur] = O.span_summary(k64[c0:c0 + wl.chunk], c0, prm.n_high_pairs, prm.rope_theta)
+            g0 = p + 1 - wl.group
+            gs[cur, -1] = O.span_summary(k64[g0:p + 1], g0, prm.n_high_pairs, prm.rope_theta)
+            qbar = O.routing_query(q64[:, 0])
+            cidx, _, _ = O.route_chunks(qbar, cs, cur, prm)
+            gidx, _, _ = O.route_groups(qbar, gs, cidx, prm)
+            toks = O.visible_tokens(p, cur, gidx, prm)
+            for hh in range(g):
+                O.attend(q64[hh, 0], k64, v64, toks)
+            dt = time.perf_counter() - t0
+            times.append(dt)
+            spent += dt
+    per_unit = sum(times) / len(times)
+    step_s = per_unit * len(units)
+    sample = (f"{len(times)} of {len(units)} (sequence, KV head) units of one decode step at "
+              f"position {p}, extrapolated to the batch ({sum(times):.1f} s of oracle time)")
+    return wl.batch / step_s, sample, 1
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return None
+    wl = S.workload(args.workload)
+    if args.batch:
+        wl = wl.with_(batch=args.batch)
+    seed = S.seed_for(list(S.WORKLOADS).index(args.workload))
+    rates = []
+    # each step is a bounded sample sized so that the whole run stays within ~3 minutes
+    budget = max(0.02, min(args.cpu_seconds / 10, 150.0 / (args.warmup + args.steps)))
+    for i in range(args.warmup + args.steps):
+        r, sample, cores = oracle_decode_rate(wl, seed, budget_s=budget)
+        if i >= args.warmup:
+            rates.append(r)
+    value = statistics.median(rates)
+    unit = "decode tokens/s (one attention layer)"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+            "n_gpus": args.gpus, "steps": len(rates), "warmup": args.warmup,
+            "ms_per_step": wl.batch / value * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, same generator)",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": wl.context},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+        if line:
+            print(json.dumps(line))
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    line, wl, seed, x = run_hga(args, rank, world)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            val, sample, cores = oracle_decode_rate(wl, seed, args.cpu_seconds, x)
+            line["cpu_baseline"] = {"value": val, "unit": line["unit"], "cores": cores,
+                                    "kind": "oracle", "sample": sample}
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,182 @@
+"""Thin Python binding of libhga.so (the C ABI in include/hga.h).
+
+Argument marshalling only: every step of the HGA path runs in the library's
+CUDA kernels.  Tensors are passed as raw pointers; the caller allocates them
+(PyTorch is used for device memory and streams).  If the library is missing,
+every call raises - there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhga.so")
+
+HGA_F32, HGA_BF16 = 0, 1
+HGA_KV_DEVICE, HGA_KV_HOST_PINNED = 0, 1
+
+STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_SHAPE", 3: "HGA_ERR_UNSUPPORTED",
+                4: "HGA_ERR_CUDA", 5: "HGA_ERR_TIMEOUT", 6: "HGA_ERR_DEVICE_CHECK",
+                7: "HGA_ERR_WORKSPACE"}
+
+# Exported symbols of the C ABI, in header order.
+SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device_status",
+           "hga_workspace_size", "hga_build_summaries", "hga_route_chunks", "hga_route_groups",
+           "hga_attend")
+
+
+class HGAConfig(ctypes.Structure):
+    """Mirror of struct hga_config."""
+
+    _fields_ = [("batch", ctypes.c_int32), ("heads_q", ctypes.c_int32),
+                ("heads_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("chunk", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("sink_chunks", ctypes.c_int32), ("local_chunks", ctypes.c_int32),
+                ("topk_chunks", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
+                ("n_high_pairs", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("out_dtype", ctypes.c_int32), ("kv_loc", ctypes.c_int32),
+                ("rope_theta", ctypes.c_double)]
+
+
+class HGAError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libhga.so once.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libhga.so not found at {path}; build it with "
+                           "`python -m hierarchical_sparse_attention_hga_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    C = ctypes.POINTER(HGAConfig)
+    sig = {
+        "hga_abi_version": (I32, []),
+        "hga_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "hga_last_error": (ctypes.c_char_p, []),
+        "hga_device_status": (ctypes.c_int, [P]),
+        "hga_workspace_size": (ctypes.c_int, [C, I64, I32, ctypes.POINTER(SZ)]),
+        "hga_build_summaries": (ctypes.c_int, [C, P, I64, I64, I64, P, P, P]),
+        "hga_route_chunks": (ctypes.c_int, [C, P, I32, P, P, I64, P, P, P]),
+        "hga_route_groups": (ctypes.c_int, [C, P, I32, P, P, I64, P, P, P, P]),
+        "hga_attend": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise HGAError(status, where, load_library().hga_last_error().decode())
+
+
+def _ptr(x):
+    """Raw address of a tensor (or an int address, or None)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+@dataclass
+class Layer:
+    """Shape and method parameters of one layer; ``config()`` gives the C struct."""
+
+    batch: int
+    heads_q: int
+    heads_kv: int
+    head_dim: int
+    chunk: int = 64
+    group: int = 16
+    sink_chunks: int = 1
+    local_chunks: int = 4
+    topk_chunks: int = 16
+    topk_groups: int = 32
+    n_high_pairs: int = 32
+    rope_theta: float = 500000.0
+    dtype: int = HGA_BF16
+    out_dtype: int = HGA_F32
+    kv_loc: int = HGA_KV_DEVICE
+
+    def config(self) -> HGAConfig:
+        return HGAConfig(self.batch, self.heads_q, self.heads_kv, self.head_dim, self.chunk,
+                         self.group, self.sink_chunks, self.local_chunks, self.topk_chunks,
+                         self.topk_groups, self.n_high_pairs, self.dtype, self.out_dtype,
+                         self.kv_loc, float(self.rope_theta))
+
+
+def _cfg(cfg) -> HGAConfig:
+    return cfg.config() if isinstance(cfg, Layer) else cfg
+
+
+def hga_abi_version() -> int:
+    return load_library().hga_abi_version()
+
+
+def hga_status_string(status: int) -> str:
+    return load_library().hga_status_string(status).decode()
+
+
+def hga_device_status(stream=None) -> int:
+    """Status of the device-side argument checks since the last call (clears them)."""
+    return load_library().hga_device_status(_stream(stream))
+
+
+def hga_workspace_size(cfg, n_alloc: int, q_len: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().hga_workspace_size(ctypes.byref(_cfg(cfg)), n_alloc, q_len,
+                                             ctypes.byref(out)), "hga_workspace_size")
+    return out.value
+
+
+def hga_build_summaries(cfg, k, n_alloc: int, t_begin: int, t_end: int, chunk_sum, group_sum,
+                        stream=None) -> None:
+    _check(load_library().hga_build_summaries(ctypes.byref(_cfg(cfg)), _ptr(k), n_alloc, t_begin,
+                                              t_end, _ptr(chunk_sum), _ptr(group_sum),
+                                              _stream(stream)), "hga_build_summaries")
+
+
+def hga_route_chunks(cfg, q, q_len: int, pos, chunk_sum, n_alloc: int, chunk_idx,
+                     chunk_score=None, stream=None) -> None:
+    _check(load_library().hga_route_chunks(ctypes.byref(_cfg(cfg)), _ptr(q), q_len, _ptr(pos),
+                                           _ptr(chunk_sum), n_alloc, _ptr(chunk_idx),
+                                           _ptr(chunk_score), _stream(stream)), "hga_route_chunks")
+
+
+def hga_route_groups(cfg, q, q_len: int, pos, group_sum, n_alloc: int, chunk_idx, group_idx,
+                     group_score=None, stream=None) -> None:
+    _check(load_library().hga_route_groups(ctypes.byref(_cfg(cfg)), _ptr(q), q_len, _ptr(pos),
+                                           _ptr(group_sum), n_alloc, _ptr(chunk_idx),
+                                           _ptr(group_idx), _ptr(group_score), _stream(stream)),
+           "hga_route_groups")
+
+
+def hga_attend(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=None,
+               workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    _check(load_library().hga_attend(ctypes.byref(_cfg(cfg)), _ptr(q), q_len, _ptr(pos), _ptr(k),
+                                     _ptr(v), n_alloc, _ptr(group_idx), _ptr(out), _ptr(lse),
+                                     _ptr(workspace), workspace_bytes, _stream(stream)),
+           "hga_attend")

@@ -1,0 +1,204 @@
+// C ABI of the HGA hot path: argument validation, the per-device error word
+// and dispatch to the kernels.  Every entry point returns a status and never
+// aborts; see include/hga.h for the contract of each call.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/hga.h"
+#include "kernels.h"
+
+namespace hga {
+namespace {
+
+thread_local char g_msg[512] = "";
+
+hga_status fail(hga_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+hga_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(HGA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// Sticky device error word: one per device that loads the library.
+__device__ unsigned g_device_error;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_err_mu;
+unsigned* g_err_ptr[kMaxDevices] = {};
+
+// Device address of g_device_error on the current device (looked up once per device).
+hga_status device_error_ptr(unsigned** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(HGA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  if (!g_err_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(device error word)");
+    g_err_ptr[dev] = static_cast<unsigned*>(ptr);
+  }
+  *out = g_err_ptr[dev];
+  return HGA_OK;
+}
+
+// Host-side checks of cfg and the derived kernel parameters.
+hga_status make_params(const hga_config* cfg, int64_t n_alloc, int32_t q_len, LayerParams* p) {
+  if (!cfg) return fail(HGA_ERR_INVALID_ARG, "cfg is NULL");
+  const hga_config& c = *cfg;
+  if (c.batch <= 0 || c.heads_q <= 0 || c.heads_kv <= 0 || c.head_dim <= 0 || c.chunk <= 0 ||
+      c.group <= 0 || c.sink_chunks < 0 || c.local_chunks < 0 || c.topk_chunks <= 0 ||
+      c.topk_groups <= 0 || c.n_high_pairs < 0)
+    return fail(HGA_ERR_INVALID_ARG, "config sizes must be positive (sink/local/n_high >= 0)");
+  if (!(c.rope_theta > 1.0)) return fail(HGA_ERR_INVALID_ARG, "rope_theta must be > 1");
+  if (c.dtype != HGA_F32 && c.dtype != HGA_BF16) return fail(HGA_ERR_INVALID_ARG, "dtype %d", c.dtype);
+  if (c.out_dtype != HGA_F32 && c.out_dtype != HGA_BF16)
+    return fail(HGA_ERR_INVALID_ARG, "out_dtype %d", c.out_dtype);
+  if (c.kv_loc != HGA_KV_DEVICE) return fail(HGA_ERR_UNSUPPORTED, "kv_loc %d", c.kv_loc);
+  if (c.heads_q % c.heads_kv) return fail(HGA_ERR_SHAPE, "heads_q %% heads_kv != 0");
+  if (c.heads_q / c.heads_kv > 16) return fail(HGA_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
+  if (c.head_dim != 64 && c.head_dim != 128) return fail(HGA_ERR_UNSUPPORTED, "head_dim %d", c.head_dim);
+  if (c.chunk != 64 && c.chunk != 128) return fail(HGA_ERR_UNSUPPORTED, "chunk %d", c.chunk);
+  if (c.group != 16) return fail(HGA_ERR_UNSUPPORTED, "group %d (16 is built)", c.group);
+  if (c.n_high_pairs > c.head_dim / 2) return fail(HGA_ERR_SHAPE, "n_high_pairs > head_dim/2");
+  if (c.topk_chunks > 256) return fail(HGA_ERR_UNSUPPORTED, "topk_chunks > 256");
+  if (c.topk_groups > 1024) return fail(HGA_ERR_UNSUPPORTED, "topk_groups > 1024");
+  if (n_alloc <= 0 || n_alloc % c.chunk) return fail(HGA_ERR_SHAPE, "n_alloc must be a positive multiple of chunk");
+  if (n_alloc / c.chunk > 32768) return fail(HGA_ERR_UNSUPPORTED, "n_alloc / chunk > 32768");
+  if (q_len <= 0) return fail(HGA_ERR_INVALID_ARG, "q_len must be positive");
+  if (q_len > 1 && q_len % c.chunk) return fail(HGA_ERR_UNSUPPORTED, "prefill q_len must be a multiple of chunk");
+  if (q_len > n_alloc) return fail(HGA_ERR_SHAPE, "q_len > n_alloc");
+  const int64_t rows = static_cast<int64_t>(c.batch) * c.heads_kv * q_len;
+  if (rows > 0x7fffffffLL) return fail(HGA_ERR_UNSUPPORTED, "batch * heads_kv * q_len too large");
+  if (static_cast<int64_t>(c.topk_chunks) * (c.chunk / c.group) > 8192)
+    return fail(HGA_ERR_UNSUPPORTED, "topk_chunks * chunk/group > 8192");
+  p->B = c.batch; p->Hq = c.heads_q; p->Hkv = c.heads_kv; p->G = c.heads_q / c.heads_kv;
+  p->D = c.head_dim; p->C = c.chunk; p->g = c.group; p->Ng = c.chunk / c.group;
+  p->sink = c.sink_chunks; p->local = c.local_chunks;
+  p->kc = c.topk_chunks; p->kg = c.topk_groups; p->n_high = c.n_high_pairs;
+  p->q_len = q_len; p->nblk = q_len == 1 ? 1 : q_len / c.chunk;
+  p->n_alloc = n_alloc; p->n_chunks = static_cast<int>(n_alloc / c.chunk);
+  p->theta = c.rope_theta;
+  return HGA_OK;
+}
+
+}  // namespace
+}  // namespace hga
+
+using namespace hga;
+
+extern "C" {
+
+int32_t hga_abi_version(void) { return HGA_ABI_VERSION; }
+
+const char* hga_status_string(hga_status s) {
+  switch (s) {
+    case HGA_OK: return "HGA_OK";
+    case HGA_ERR_INVALID_ARG: return "HGA_ERR_INVALID_ARG";
+    case HGA_ERR_SHAPE: return "HGA_ERR_SHAPE";
+    case HGA_ERR_UNSUPPORTED: return "HGA_ERR_UNSUPPORTED";
+    case HGA_ERR_CUDA: return "HGA_ERR_CUDA";
+    case HGA_ERR_TIMEOUT: return "HGA_ERR_TIMEOUT";
+    case HGA_ERR_DEVICE_CHECK: return "HGA_ERR_DEVICE_CHECK";
+    case HGA_ERR_WORKSPACE: return "HGA_ERR_WORKSPACE";
+  }
+  return "HGA_ERR_UNKNOWN";
+}
+
+const char* hga_last_error(void) { return g_msg; }
+
+hga_status hga_device_status(void* stream) {
+  unsigned* err = nullptr;
+  hga_status st = device_error_ptr(&err);
+  if (st != HGA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, err, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(err, 0, sizeof(unsigned), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "hga_device_status");
+  if (host) return fail(HGA_ERR_DEVICE_CHECK, "device check failed, bits 0x%x", host);
+  return HGA_OK;
+}
+
+hga_status hga_workspace_size(const hga_config* cfg, int64_t n_alloc, int32_t q_len, size_t* bytes) {
+  if (!bytes) return fail(HGA_ERR_INVALID_ARG, "bytes is NULL");
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, q_len, &p);
+  if (st != HGA_OK) return st;
+  *bytes = attend_workspace_bytes(p);
+  return HGA_OK;
+}
+
+hga_status hga_build_summaries(const hga_config* cfg, const void* k, int64_t n_alloc,
+                               int64_t t_begin, int64_t t_end, float* chunk_sum,
+                               float* group_sum, void* stream) {
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if (!k || !chunk_sum || !group_sum) return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (t_begin < 0 || t_end < t_begin || t_end > n_alloc)
+    return fail(HGA_ERR_INVALID_ARG, "need 0 <= t_begin <= t_end <= n_alloc");
+  cudaError_t e = launch_summaries(p, cfg->dtype, k, t_begin, t_end, chunk_sum, group_sum,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_build_summaries");
+}
+
+hga_status hga_route_chunks(const hga_config* cfg, const void* q, int32_t q_len,
+                            const int64_t* pos, const float* chunk_sum, int64_t n_alloc,
+                            int32_t* chunk_idx, float* chunk_score, void* stream) {
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, q_len, &p);
+  if (st != HGA_OK) return st;
+  if (!q || !pos || !chunk_sum || !chunk_idx) return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_route_chunks(p, cfg->dtype, q, pos, chunk_sum, chunk_idx, chunk_score,
+                                      err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_chunks");
+}
+
+hga_status hga_route_groups(const hga_config* cfg, const void* q, int32_t q_len,
+                            const int64_t* pos, const float* group_sum, int64_t n_alloc,
+                            const int32_t* chunk_idx, int32_t* group_idx, float* group_score,
+                            void* stream) {
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, q_len, &p);
+  if (st != HGA_OK) return st;
+  if (!q || !pos || !group_sum || !chunk_idx || !group_idx)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_route_groups(p, cfg->dtype, q, pos, group_sum, chunk_idx, group_idx,
+                                      group_score, err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_groups");
+}
+
+hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const int64_t* pos,
+                      const void* k, const void* v, int64_t n_alloc, const int32_t* group_idx,
+                      void* out, float* lse, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, q_len, &p);
+  if (st != HGA_OK) return st;
+  if (!q || !pos || !k || !v || !group_idx || !out) return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  const size_t need = attend_workspace_bytes(p);
+  if (need && (!workspace || workspace_bytes < need))
+    return fail(HGA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_attend(p, cfg->dtype, cfg->out_dtype, q, pos, k, v, group_idx, out, lse,
+                                workspace, err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attend");
+}
+
+}  // extern "C"

@@ -1,0 +1,264 @@
+// Steps 2 and 3: two-level routing.
+//
+// HGA technical summary ("Hierarchical Global Attention (HGA)", gist.science
+// 2606.30709), "Metodologia -> Meccanismo Core", item 2: level 1 scores the
+// current block against the compact table of chunk key summaries of earlier
+// chunks; level 2 scores the group summaries inside the selected chunks.  The
+// sink, local and current chunks are always visible, so they are not
+// candidates: content routing covers the intermediate context only.
+//
+// One CTA per (sequence, KV head, query block).  The routing query is the mean
+// of the block's post-RoPE query rows over the G heads sharing the KV head,
+// summed in a fixed order (deterministic).  Summary rows are streamed with
+// 16-byte loads, one row per D/4 lanes, four rows in flight per lane; scores
+// land in shared memory and a block radix select keeps the top-k.
+#include "common.cuh"
+#include "kernels.h"
+#include "topk.cuh"
+
+namespace hga {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// qbar[0..D) = mean of the q rows (G heads x nr rows) of (b, KV head h).
+template <typename T, int D>
+__device__ void routing_query(const T* __restrict__ q, const LayerParams& p, int b, int h, int r0,
+                              int nr, float* qbar, float (*part)[D]) {
+  constexpr int DPL = D / 32;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  float acc[DPL];
+#pragma unroll
+  for (int u = 0; u < DPL; ++u) acc[u] = 0.f;
+  const int rows = p.G * nr;
+  for (int r = wid; r < rows; r += kWarps) {
+    const int hh = r / nr, rr = r % nr;
+    const T* src = q + ((static_cast<size_t>(b) * p.Hq + h * p.G + hh) * p.q_len + r0 + rr) * D +
+                   lane * DPL;
+    float x[DPL];
+    if constexpr (DPL == 4) load4(src, x); else load2(src, x);
+#pragma unroll
+    for (int u = 0; u < DPL; ++u) acc[u] += x[u];
+  }
+#pragma unroll
+  for (int u = 0; u < DPL; ++u) part[wid][lane * DPL + u] = acc[u];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s += part[w][threadIdx.x];
+    qbar[threadIdx.x] = s / static_cast<float>(rows);
+  }
+  __syncthreads();
+}
+
+// sc[i] = qbar . row(i) for i < n; row(i) returns a pointer to D floats (16 B aligned).
+template <int D, typename RowFn>
+__device__ void score_rows(int n, const float* qbar, float* sc, RowFn row) {
+  constexpr int LPR = D / 4;          // lanes per row
+  constexpr int RPW = 32 / LPR;       // rows per warp step
+  constexpr int UNR = 4;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int sub = lane / LPR, l = lane % LPR;
+  const float4 qv = reinterpret_cast<const float4*>(qbar)[l];
+  const int step = kWarps * RPW;
+  // The loop bound is uniform across the warp (all lanes join the shuffles);
+  // rows past n are masked per lane.
+  for (int wbase = wid * RPW; wbase < n; wbase += step * UNR) {
+    const int base = wbase + sub;
+    float4 v[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int i = base + u * step;
+      v[u] = i < n ? __ldg(reinterpret_cast<const float4*>(row(i)) + l) : make_float4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      float d = v[u].x * qv.x + v[u].y * qv.y + v[u].z * qv.z + v[u].w * qv.w;
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      const int i = base + u * step;
+      if (l == 0 && i < n) sc[i] = d;
+    }
+  }
+}
+
+// Decode (q_len == 1): one block, the query's chunk.  Prefill: block blk holds
+// queries blk*C .. blk*C+C-1 and its current chunk is their chunk.
+__device__ __forceinline__ void block_rows(const LayerParams& p, int64_t pos, int blk, int* r0,
+                                           int* nr, int* cur) {
+  const int64_t first = pos - p.q_len + 1;
+  *r0 = p.q_len == 1 ? 0 : blk * p.C;
+  *nr = p.q_len == 1 ? 1 : p.C;
+  *cur = static_cast<int>((first + *r0 + *nr - 1) / p.C);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+route_chunks_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
+                    const float* __restrict__ chunk_sum, LayerParams p,
+                    int32_t* __restrict__ chunk_idx, float* __restrict__ chunk_score,
+                    unsigned* err) {
+  __shared__ __align__(16) float qbar[D];
+  __shared__ float part[kWarps][D];
+  __shared__ TopkSmem tsm;
+  extern __shared__ __align__(16) float dyn[];
+  const int item = blockIdx.x;
+  const int blk = item % p.nblk;
+  const int bh = item / p.nblk;
+  const int h = bh % p.Hkv, b = bh / p.Hkv;
+  int32_t* out = chunk_idx + static_cast<size_t>(item) * p.kc;
+  float* out_sc = chunk_score ? chunk_score + static_cast<size_t>(item) * p.kc : nullptr;
+  const int64_t pb = pos[b];
+  if (!valid_position(pb, p, threadIdx.x == 0 ? err : nullptr)) {
+    for (int i = threadIdx.x; i < p.kc; i += kThreads) {
+      out[i] = -1;
+      if (out_sc) out_sc[i] = CUDART_NAN_F;
+    }
+    return;
+  }
+  int r0, nr, cur;
+  block_rows(p, pb, blk, &r0, &nr, &cur);
+  routing_query<T, D>(q, p, b, h, r0, nr, qbar, part);
+
+  const int n_cand = max(0, cur - p.local - p.sink);
+  float* sc = dyn;                                   // [n_chunks]
+  int* sel = reinterpret_cast<int*>(dyn + p.n_chunks);  // [kc]
+  const float* rows = chunk_sum + (static_cast<size_t>(bh) * p.n_chunks + p.sink) * D;
+  score_rows<D>(n_cand, qbar, sc, [&](int i) { return rows + static_cast<size_t>(i) * D; });
+  __syncthreads();
+  const int ns = block_topk<kThreads>(sc, n_cand, p.kc, sel, tsm);
+  for (int i = threadIdx.x; i < p.kc; i += kThreads) {
+    out[i] = i < ns ? sel[i] + p.sink : -1;
+    if (out_sc) out_sc[i] = i < ns ? sc[sel[i]] : CUDART_NAN_F;
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
+                    const float* __restrict__ group_sum, const int32_t* __restrict__ chunk_idx,
+                    LayerParams p, int32_t* __restrict__ group_idx,
+                    float* __restrict__ group_score, unsigned* err) {
+  __shared__ __align__(16) float qbar[D];
+  __shared__ float part[kWarps][D];
+  __shared__ TopkSmem tsm;
+  __shared__ int n_sel;
+  extern __shared__ __align__(16) float dyn[];
+  const int item = blockIdx.x;
+  const int blk = item % p.nblk;
+  const int bh = item / p.nblk;
+  const int h = bh % p.Hkv, b = bh / p.Hkv;
+  int32_t* out = group_idx + static_cast<size_t>(item) * p.kg;
+  float* out_sc = group_score ? group_score + static_cast<size_t>(item) * p.kg : nullptr;
+  const int64_t pb = pos[b];
+  if (!valid_position(pb, p, threadIdx.x == 0 ? err : nullptr)) {
+    for (int i = threadIdx.x; i < p.kg; i += kThreads) {
+      out[i] = -1;
+      if (out_sc) out_sc[i] = CUDART_NAN_F;
+    }
+    return;
+  }
+  int r0, nr, cur;
+  block_rows(p, pb, blk, &r0, &nr, &cur);
+
+  const int n_cand_max = p.kc * p.Ng;
+  float* sc = dyn;                                        // [kc * Ng]
+  int* sel = reinterpret_cast<int*>(dyn + n_cand_max);    // [kg]
+  int* chunks = sel + p.kg;                               // [kc]
+  const int32_t* cidx = chunk_idx + static_cast<size_t>(item) * p.kc;
+  for (int i = threadIdx.x; i < p.kc; i += kThreads) chunks[i] = cidx[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Keep the ascending complete candidate chunks; flag anything else.
+    int n = 0, prev = -1;
+    bool bad = false;
+    for (int i = 0; i < p.kc; ++i) {
+      const int c = chunks[i];
+      if (c < 0) continue;
+      if (c < p.sink || c >= cur - p.local || c <= prev) { bad = true; continue; }
+      chunks[n++] = c;
+      prev = c;
+    }
+    n_sel = n;
+    if (bad) flag_error(err, kErrChunkIdx);
+  }
+  routing_query<T, D>(q, p, b, h, r0, nr, qbar, part);  // syncs: n_sel and chunks visible
+
+  const int n_cand = n_sel * p.Ng;
+  const float* base = group_sum + static_cast<size_t>(bh) * p.n_chunks * p.Ng * D;
+  score_rows<D>(n_cand, qbar, sc, [&](int i) {
+    const int c = chunks[i / p.Ng], gi = i % p.Ng;
+    return base + (static_cast<size_t>(c) * p.Ng + gi) * D;
+  });
+  __syncthreads();
+  const int ns = block_topk<kThreads>(sc, n_cand, p.kg, sel, tsm);
+  for (int i = threadIdx.x; i < p.kg; i += kThreads) {
+    if (i < ns) {
+      const int s = sel[i];
+      out[i] = chunks[s / p.Ng] * p.Ng + s % p.Ng;
+      if (out_sc) out_sc[i] = sc[s];
+    } else {
+      out[i] = -1;
+      if (out_sc) out_sc[i] = CUDART_NAN_F;
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_route_chunks_t(const LayerParams& p, const void* q, const int64_t* pos,
+                                  const float* chunk_sum, int32_t* chunk_idx, float* chunk_score,
+                                  unsigned* err, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(p.n_chunks) * sizeof(float) + p.kc * sizeof(int);
+  auto kern = route_chunks_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<p.B * p.Hkv * p.nblk, kThreads, smem, s>>>(static_cast<const T*>(q), pos, chunk_sum, p,
+                                                    chunk_idx, chunk_score, err);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_route_groups_t(const LayerParams& p, const void* q, const int64_t* pos,
+                                  const float* group_sum, const int32_t* chunk_idx,
+                                  int32_t* group_idx, float* group_score, unsigned* err,
+                                  cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(p.kc) * p.Ng * sizeof(float) +
+                      static_cast<size_t>(p.kg + p.kc) * sizeof(int);
+  auto kern = route_groups_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<p.B * p.Hkv * p.nblk, kThreads, smem, s>>>(static_cast<const T*>(q), pos, group_sum,
+                                                    chunk_idx, p, group_idx, group_score, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_chunks(const LayerParams& p, int dtype, const void* q, const int64_t* pos,
+                                const float* chunk_sum, int32_t* chunk_idx, float* chunk_score,
+                                unsigned* err, cudaStream_t s) {
+  if (dtype == 0)
+    return p.D == 64 ? launch_route_chunks_t<float, 64>(p, q, pos, chunk_sum, chunk_idx, chunk_score, err, s)
+                     : launch_route_chunks_t<float, 128>(p, q, pos, chunk_sum, chunk_idx, chunk_score, err, s);
+  return p.D == 64
+             ? launch_route_chunks_t<__nv_bfloat16, 64>(p, q, pos, chunk_sum, chunk_idx, chunk_score, err, s)
+             : launch_route_chunks_t<__nv_bfloat16, 128>(p, q, pos, chunk_sum, chunk_idx, chunk_score, err, s);
+}
+
+cudaError_t launch_route_groups(const LayerParams& p, int dtype, const void* q, const int64_t* pos,
+                                const float* group_sum, const int32_t* chunk_idx,
+                                int32_t* group_idx, float* group_score, unsigned* err,
+                                cudaStream_t s) {
+  if (dtype == 0)
+    return p.D == 64 ? launch_route_groups_t<float, 64>(p, q, pos, group_sum, chunk_idx, group_idx, group_score, err, s)
+                     : launch_route_groups_t<float, 128>(p, q, pos, group_sum, chunk_idx, group_idx, group_score, err, s);
+  return p.D == 64
+             ? launch_route_groups_t<__nv_bfloat16, 64>(p, q, pos, group_sum, chunk_idx, group_idx, group_score, err, s)
+             : launch_route_groups_t<__nv_bfloat16, 128>(p, q, pos, group_sum, chunk_idx, group_idx, group_score, err, s);
+}
+
+}  // namespace hga

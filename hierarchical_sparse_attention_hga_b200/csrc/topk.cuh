@@ -1,0 +1,139 @@
+// Block-wide deterministic top-k over float scores held in shared memory.
+//
+// Selects the k largest of n scores, equal scores going to the lower index, and
+// writes the chosen indices in ascending order.  A 4-pass 8-bit radix select
+// finds the k-th largest order key T and how many keys equal to T are still
+// needed; one ordered block scan then takes those in index order.  No sort, no
+// atomics outside the shared-memory histogram, no inter-block communication.
+#pragma once
+
+#include "common.cuh"
+
+namespace hga {
+
+struct TopkSmem {
+  unsigned hist[256];
+  int warp_tot[32];
+  unsigned pick[2];
+};
+
+// Order-preserving map of a float to uint32 (larger float -> larger key);
+// -0.0 is folded onto +0.0 so that the two compare equal, as they do as floats.
+__device__ __forceinline__ unsigned order_key(float f) {
+  unsigned u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix sum of one int per thread, in thread order.  Every thread of
+// the block must call it.  NT = blockDim.x, a multiple of 32.
+template <int NT>
+__device__ __forceinline__ int block_exclusive_scan(int v, TopkSmem& sm, int* total = nullptr) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) sm.warp_tot[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int w = lane < NW ? sm.warp_tot[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    if (lane < NW) sm.warp_tot[lane] = wi - w;  // exclusive warp offsets
+    if (lane == NW - 1 && total) sm.pick[1] = static_cast<unsigned>(wi);
+  }
+  __syncthreads();
+  const int res = sm.warp_tot[wid] + incl - v;
+  if (total) *total = static_cast<int>(sm.pick[1]);
+  __syncthreads();
+  return res;
+}
+
+// Indices of the top k of sc[0..n) (ties to the lower index), ascending, into
+// sel[0..min(n,k)).  Returns min(n, k).  Every thread of the block must call it;
+// sc and sel are shared memory; sel is complete on return.
+template <int NT>
+__device__ int block_topk(const float* sc, int n, int k, int* sel, TopkSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (n <= k) {
+    for (int i = tid; i < n; i += NT) sel[i] = i;
+    __syncthreads();
+    return n;
+  }
+  unsigned prefix = 0u, pmask = 0u;
+  unsigned krem = static_cast<unsigned>(k);
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += NT) sm.hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += NT) {
+      const unsigned key = order_key(sc[i]);
+      if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (wid == 0) {
+      // lane l owns digits 255-8l .. 248-8l, visited from the largest down
+      unsigned c[8], tot = 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { c[j] = sm.hist[255 - 8 * lane - j]; tot += c[j]; }
+      unsigned incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      unsigned run = incl - tot;  // keys with a larger digit
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (run < krem && krem <= run + c[j]) {
+          sm.pick[0] = 255u - 8u * lane - j;
+          sm.pick[1] = run;
+        }
+        run += c[j];
+      }
+    }
+    __syncthreads();
+    const unsigned d = sm.pick[0];
+    krem -= sm.pick[1];
+    prefix |= d << shift;
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  const unsigned thr = prefix;  // k-th largest key; krem of the keys equal to it are taken
+  const int ipt = (n + NT - 1) / NT;
+  const int beg = min(n, tid * ipt), end = min(n, beg + ipt);
+  int n_eq = 0;
+  for (int i = beg; i < end; ++i) n_eq += order_key(sc[i]) == thr;
+  const int eq_before = block_exclusive_scan<NT>(n_eq, sm);
+  int n_sel = 0;
+  {
+    int eq = eq_before;
+    for (int i = beg; i < end; ++i) {
+      const unsigned key = order_key(sc[i]);
+      const bool take = key > thr || (key == thr && static_cast<unsigned>(eq) < krem);
+      eq += key == thr;
+      n_sel += take;
+    }
+  }
+  int w = block_exclusive_scan<NT>(n_sel, sm);
+  {
+    int eq = eq_before;
+    for (int i = beg; i < end; ++i) {
+      const unsigned key = order_key(sc[i]);
+      const bool take = key > thr || (key == thr && static_cast<unsigned>(eq) < krem);
+      eq += key == thr;
+      if (take) sel[w++] = i;
+    }
+  }
+  __syncthreads();
+  return k;
+}
+
+}  // namespace hga

@@ -1,0 +1,222 @@
+/*
+ * hga.h - C ABI of the Hierarchical Global Attention (HGA) hot path on B200.
+ *
+ * HGA replaces dense causal attention over a long K/V cache without touching
+ * the model's weights (technical summary of "Hierarchical Global Attention
+ * (HGA)", gist.science paper 2606.30709, section "Metodologia", and "Contributi
+ * Chiave" item 1: drop-in compatibility).  One layer's decode or prefill step
+ * is four calls, in this order:
+ *
+ *   hga_build_summaries  RoPE-aware chunk and group key summaries
+ *   hga_route_chunks     level-1 routing against the chunk-summary table
+ *   hga_route_groups     level-2 routing inside the selected chunks
+ *   hga_attend           exact softmax over the routed tokens' original K/V
+ *
+ * Conventions shared by every call
+ *  - Plain pointers and sizes only.  Device pointers are CUDA device memory of
+ *    the current device; the caller owns and frees every buffer.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).  They validate what they can on the
+ *    host and return a status; they never abort the process.
+ *  - Conditions only the device can see (a position out of range, an index
+ *    set that breaks its contract) set a sticky device error word, read and
+ *    cleared by hga_device_status().  The offending work item writes -1
+ *    indices / zero outputs instead of faulting.
+ *  - Layouts are row-major and contiguous:
+ *      q      [B, Hq, q_len, D]   post-RoPE queries (dtype)
+ *      k, v   [B, Hkv, n_alloc, D] post-RoPE key cache and value cache (dtype);
+ *             token t sits at row t and at RoPE position t
+ *      chunk_sum [B, Hkv, n_alloc/C, D]          float32
+ *      group_sum [B, Hkv, n_alloc/C, C/g, D]     float32
+ *      chunk_idx [B, Hkv, nblk, kc] int32, group_idx [B, Hkv, nblk, kg] int32
+ *      out    [B, Hq, q_len, D] (out_dtype), lse [B, Hq, q_len] float32
+ *    Query head hq reads KV head hq / (Hq/Hkv).
+ *  - Query blocks.  The queries of sequence b sit at positions
+ *    pos[b]-q_len+1 .. pos[b].  Decode is q_len == 1 (one block).  Prefill
+ *    takes q_len a multiple of C with pos[b]+1 a multiple of C; every chunk of
+ *    C queries is one routing block (nblk = q_len / C).
+ *  - pos is a DEVICE array int64[B] so that a decode loop can advance it on
+ *    the GPU; 0 <= pos[b] < n_alloc and pos[b] >= q_len-1 is checked on the
+ *    device.
+ *  - All sequences share n_alloc (the cache capacity in tokens, a multiple of
+ *    C).
+ */
+#ifndef HGA_H_
+#define HGA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HGA_ABI_VERSION 1
+
+typedef enum hga_status {
+  HGA_OK = 0,
+  HGA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum */
+  HGA_ERR_SHAPE = 2,         /* inconsistent sizes (Hq % Hkv, n_alloc % C, ...) */
+  HGA_ERR_UNSUPPORTED = 3,   /* valid but not built: head_dim, chunk, group, k limits */
+  HGA_ERR_CUDA = 4,          /* a CUDA runtime call failed; see hga_last_error() */
+  HGA_ERR_TIMEOUT = 5,       /* a bounded wait ran out */
+  HGA_ERR_DEVICE_CHECK = 6,  /* a device-side argument check failed */
+  HGA_ERR_WORKSPACE = 7      /* workspace missing or smaller than hga_workspace_size() */
+} hga_status;
+
+typedef enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype;
+
+typedef enum hga_kv_loc { HGA_KV_DEVICE = 0, HGA_KV_HOST_PINNED = 1 } hga_kv_loc;
+
+/* Layer shape and method parameters.  Field names follow the pages' notation. */
+typedef struct hga_config {
+  int32_t batch;          /* B */
+  int32_t heads_q;        /* Hq */
+  int32_t heads_kv;       /* Hkv; G = Hq / Hkv query heads share one KV head (1..16) */
+  int32_t head_dim;       /* D: 64 or 128 */
+  int32_t chunk;          /* C: fixed chunk size, 64 or 128 */
+  int32_t group;          /* g: tokens per group inside a chunk; 16 */
+  int32_t sink_chunks;    /* initial chunks that are always visible (>= 0) */
+  int32_t local_chunks;   /* recent chunks before the current one that are always visible (>= 0) */
+  int32_t topk_chunks;    /* kc: level-1 top-k, 1..256 */
+  int32_t topk_groups;    /* kg: level-2 top-k, 1..1024 */
+  int32_t n_high_pairs;   /* RoPE pairs i < n_high_pairs are "high frequency" (0..D/2) */
+  int32_t dtype;          /* hga_dtype of q, k, v */
+  int32_t out_dtype;      /* hga_dtype of out */
+  int32_t kv_loc;         /* hga_kv_loc of k and v (HGA_KV_DEVICE for the calls below) */
+  double rope_theta;      /* RoPE base: omega_i = rope_theta^(-2i/D) */
+} hga_config;
+
+/* Version of this ABI (HGA_ABI_VERSION of the built library). */
+int32_t hga_abi_version(void);
+
+/* Human-readable name of a status. Never NULL. */
+const char* hga_status_string(hga_status status);
+
+/* Detail message of the last failing call on this host thread ("" if none). */
+const char* hga_last_error(void);
+
+/*
+ * Synchronises `stream`, then returns HGA_ERR_DEVICE_CHECK if any kernel of this
+ * library on the current device has set the device error word since the last
+ * call, and clears it; HGA_OK otherwise (HGA_ERR_CUDA if the sync failed).
+ */
+hga_status hga_device_status(void* stream);
+
+/*
+ * Bytes of device workspace hga_attend needs for (cfg, n_alloc, q_len).  Zero
+ * is a valid answer.  The workspace holds per-split partial results of the
+ * split-K decode; its contents need no initialisation and are scratch.
+ */
+hga_status hga_workspace_size(const hga_config* cfg, int64_t n_alloc, int32_t q_len,
+                              size_t* bytes);
+
+/*
+ * Step 1 - RoPE-aware key summaries (HGA technical summary, "Metodologia ->
+ * Meccanismo Core", item 1 partitioning and item 3 RoPE-aware summaries).
+ *
+ * For every chunk (C tokens) and every group (g tokens) whose LAST token lies
+ * in [t_begin, t_end), computes its summary row from the keys in k and stores
+ * it; rows whose last token is outside that range are left untouched, so a
+ * whole cache is summarised with (0, n) and a decode step appending token p
+ * calls (p, p+1) (a no-op unless p closes a group).  Each row is computed from
+ * the cache alone, the same way whatever the call pattern, so appending token
+ * by token gives bit-identical rows to one batch call.
+ *
+ * Summary of the span t0..t0+L-1 with centre r = t0 + (L-1)/2:
+ *   high-frequency pairs (i < n_high_pairs): mean of the stored (rotated) keys;
+ *   low-frequency pairs: mean of the raw keys R(-t) k[t], rotated to r;
+ *   equivalently mean over t of R(r - t) k[t] on those pairs.
+ *
+ *   k          device, [B, Hkv, n_alloc, D] of cfg->dtype, post-RoPE keys
+ *   n_alloc    cache capacity in tokens (multiple of C)
+ *   t_begin, t_end   0 <= t_begin <= t_end <= n_alloc (same for every sequence)
+ *   chunk_sum  device float32 [B, Hkv, n_alloc/C, D] (written rows only)
+ *   group_sum  device float32 [B, Hkv, n_alloc/C, C/g, D] (written rows only)
+ * Errors: INVALID_ARG / SHAPE / UNSUPPORTED for bad arguments, CUDA on launch
+ * failure.  No workspace.
+ */
+hga_status hga_build_summaries(const hga_config* cfg, const void* k, int64_t n_alloc,
+                               int64_t t_begin, int64_t t_end, float* chunk_sum,
+                               float* group_sum, void* stream);
+
+/*
+ * Step 2 - level-1 chunk routing with deterministic visibility (HGA technical
+ * summary, "Metodologia -> Meccanismo Core", item 2: "Livello 1 (Chunk
+ * Routing)" and "Visibilita Deterministica"; "Contributi Chiave" item 3).
+ *
+ * For each (sequence b, KV head h, query block): the routing query is the mean
+ * of the block's post-RoPE query vectors over the G query heads of h.  With
+ * cur = the chunk of the block's last query, the candidates are the chunks j
+ * with sink_chunks <= j < cur - local_chunks (the always-visible sink, local
+ * and current chunks are not candidates: they are attended in full).  Each
+ * candidate is scored by the dot product of the routing query with its chunk
+ * summary; the kc best are kept (equal scores: lower chunk index first) and
+ * written in ascending order, padded with -1.
+ *
+ *   q          device [B, Hq, q_len, D] (cfg->dtype)
+ *   pos        device int64 [B], position of each sequence's last query
+ *   chunk_sum  device float32 [B, Hkv, n_alloc/C, D]; candidate rows complete
+ *   chunk_idx  device int32 [B, Hkv, nblk, kc] (output)
+ *   chunk_score optional device float32 [B, Hkv, nblk, kc]: the selected
+ *              chunks' scores (NaN on padding); may be NULL
+ * Limits: n_alloc / C <= 32768.  No workspace.
+ */
+hga_status hga_route_chunks(const hga_config* cfg, const void* q, int32_t q_len,
+                            const int64_t* pos, const float* chunk_sum, int64_t n_alloc,
+                            int32_t* chunk_idx, float* chunk_score, void* stream);
+
+/*
+ * Step 3 - level-2 group routing inside the selected chunks (HGA technical
+ * summary, "Metodologia -> Meccanismo Core", item 2: "Livello 2 (Group
+ * Routing)").
+ *
+ * Scores every group of every selected chunk (skipping -1 entries) against
+ * the same routing query as step 2 and keeps the kg best over all of them
+ * (equal scores: lower global group id first).  A group is named by its global
+ * id chunk * (C/g) + group-in-chunk; ids are written ascending, padded with -1.
+ *
+ *   chunk_idx  device int32 [B, Hkv, nblk, kc], ascending, as step 2 writes it;
+ *              every entry must be a complete candidate chunk (checked on the
+ *              device)
+ *   group_sum  device float32 [B, Hkv, n_alloc/C, C/g, D]
+ *   group_idx  device int32 [B, Hkv, nblk, kg] (output)
+ *   group_score optional device float32 [B, Hkv, nblk, kg]; may be NULL
+ * Limits: kc * C/g <= 8192.  No workspace.
+ */
+hga_status hga_route_groups(const hga_config* cfg, const void* q, int32_t q_len,
+                            const int64_t* pos, const float* group_sum, int64_t n_alloc,
+                            const int32_t* chunk_idx, int32_t* group_idx, float* group_score,
+                            void* stream);
+
+/*
+ * Steps 4-5 - gather of the selected tokens' original K/V and exact softmax
+ * attention over that bounded set (HGA technical summary, "Metodologia ->
+ * Meccanismo Core", item 4 "Attenzione Esatta per Token"; "Contributi Chiave"
+ * item 2: only retrieval is approximated, never the attention output).
+ *
+ * Each query at position p attends, with scale 1/sqrt(D), to: every token of
+ * the sink chunks and of the local chunks, the tokens <= p of its own chunk,
+ * and the g tokens of every group in its block's group_idx row.  No summary
+ * value enters the output.
+ *
+ *   k, v       device [B, Hkv, n_alloc, D] (cfg->dtype)
+ *   group_idx  device int32 [B, Hkv, nblk, kg] from step 3; entries must be
+ *              groups of candidate chunks (checked on the device; a bad entry
+ *              is skipped and flagged)
+ *   out        device [B, Hq, q_len, D] of cfg->out_dtype
+ *   lse        optional device float32 [B, Hq, q_len]: natural-log
+ *              log-sum-exp of the scaled scores; may be NULL
+ *   workspace  device scratch of at least hga_workspace_size() bytes
+ *              (may be NULL when that size is 0)
+ */
+hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const int64_t* pos,
+                      const void* k, const void* v, int64_t n_alloc, const int32_t* group_idx,
+                      void* out, float* lse, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HGA_H_ */

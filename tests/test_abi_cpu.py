@@ -1,0 +1,112 @@
+"""The C-ABI library builds, loads and exports every symbol include/hga.h declares.
+
+No compute call is made here: only entry points that fail host-side argument
+validation (before any CUDA call) or are pure host functions run.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    from hierarchical_sparse_attention_hga_b200.build import build
+    build()
+    return B.load_library()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "hga.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hga_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_steps():
+    names = declared_symbols()
+    for step in ("hga_build_summaries", "hga_route_chunks", "hga_route_groups", "hga_attend"):
+        assert step in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    names = declared_symbols()
+    assert sorted(B.SYMBOLS) == names
+    for name in names:
+        assert getattr(lib, name) is not None
+
+
+def test_abi_version_and_status_strings(lib):
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    assert B.hga_abi_version() == 1
+    assert B.hga_status_string(0) == "HGA_OK"
+    assert B.hga_status_string(6) == "HGA_ERR_DEVICE_CHECK"
+    assert B.hga_status_string(99) == "HGA_ERR_UNKNOWN"
+
+
+def test_config_struct_layout_matches_header(lib):
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    assert ctypes.sizeof(B.HGAConfig) == 14 * 4 + 8
+    assert B.HGAConfig.rope_theta.offset == 56
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(heads_q=3, heads_kv=2), 2),          # Hq % Hkv
+    (dict(head_dim=96), 3),                     # unsupported D
+    (dict(chunk=32), 3),                        # unsupported C
+    (dict(group=8), 3),                         # unsupported g
+    (dict(topk_chunks=0), 1),                   # non-positive k
+    (dict(n_high_pairs=65), 2),                 # more pairs than D/2
+    (dict(rope_theta=0.5), 1),
+    (dict(heads_q=64, heads_kv=2), 3),          # G = 32 > 16
+    (dict(dtype=7), 1),
+])
+def test_host_validation_errors(lib, kw, status):
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    base = dict(batch=1, heads_q=32, heads_kv=8, head_dim=128)
+    base.update(kw)
+    with pytest.raises(B.HGAError) as e:
+        B.hga_workspace_size(B.Layer(**base), 4096, 1)
+    assert e.value.status == status
+    assert B.load_library().hga_last_error()  # detail message is set
+
+
+def test_shape_errors_of_sizes(lib):
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    layer = B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128)
+    for n_alloc, q_len, status in [(4000, 1, 2), (4096, 0, 1), (4096, 100, 3), (0, 1, 2)]:
+        with pytest.raises(B.HGAError) as e:
+            B.hga_workspace_size(layer, n_alloc, q_len)
+        assert e.value.status == status
+
+
+def test_null_pointers_rejected_before_any_cuda_call(lib):
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    layer = B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128)
+    with pytest.raises(B.HGAError) as e:
+        B.hga_build_summaries(layer, None, 4096, 0, 4096, None, None, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(B.HGAError) as e:
+        B.hga_build_summaries(layer, 16, 4096, 10, 5, 16, 16, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(B.HGAError) as e:
+        B.hga_route_chunks(layer, None, 1, None, None, 4096, None, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(B.HGAError) as e:
+        B.hga_attend(layer, 16, 1, 16, 16, 16, 4096, 16, 16, workspace=None, workspace_bytes=0,
+                     stream=0)
+    assert e.value.status == 7  # decode needs split-K workspace
+
+
+def test_workspace_size_is_zero_for_prefill_and_grows_with_batch(lib):
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    small = B.hga_workspace_size(B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128), 32768, 1)
+    big = B.hga_workspace_size(B.Layer(batch=16, heads_q=32, heads_kv=8, head_dim=128), 32768, 1)
+    assert 0 < small < big
+    assert B.hga_workspace_size(B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128), 32768,
+                                1024) == 0

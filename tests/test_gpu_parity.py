@@ -1,0 +1,171 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Routed indices must equal the oracle's except where the oracle's own scores put
+the differing candidates within a 1e-4 relative window of the k-th score (a
+near-tie, then the GPU selection is validated and attention is compared on
+it).  Outputs: max-abs 2e-2 for bf16 K/V with fp32 accumulation, 1e-4 for
+fp32 inputs.
+"""
+
+import numpy as np
+import pytest
+
+import hga_synth as S
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU too
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from gpu_harness import compare_head, compare_summaries, run_gpu  # noqa: E402
+from hierarchical_sparse_attention_hga_b200 import binding as B  # noqa: E402
+from oracle import hga_oracle as O  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from hierarchical_sparse_attention_hga_b200.build import build
+    build()
+    B.load_library()
+
+
+# ------------------------------------------------------------- tiny fp32 layer
+
+def test_tiny_fp32_decode():
+    wl = S.workload("tiny_f32_1k")
+    x = S.make_inputs(wl, S.seed_for(0))
+    res = run_gpu(wl, x)
+    compare_summaries(wl, x, res, 0, 0)
+    compare_head(wl, x, res, 0, 0)
+    toks = O.visible_tokens(1023, 15, res["group_idx"][0, 0, 0], O.HGAParams(
+        head_dim=64, heads_q=1, heads_kv=1, chunk=64, group=16, sink=1, local=2,
+        topk_chunks=4, topk_groups=8))
+    assert len(toks) == 384
+
+
+def test_tiny_fp32_prefill_all_blocks():
+    wl = S.workload("tiny_f32_1k", prefill=True)
+    x = S.make_inputs(wl, S.seed_for(0))
+    res = run_gpu(wl, x)
+    assert res["chunk_idx"].shape[2] == 16
+    compare_head(wl, x, res, 0, 0)
+
+
+# ------------------------------------------------------- bf16 decode variants
+
+@pytest.mark.parametrize("chunk", [64, 128])
+def test_bf16_decode_small_context(chunk):
+    wl = S.workload("llama3_8b_decode_32k", batch=2, context=4096, chunk=chunk)
+    x = S.make_inputs(wl, 11)
+    res = run_gpu(wl, x)
+    for b in range(2):
+        for h in (0, 5):
+            compare_summaries(wl, x, res, b, h)
+            compare_head(wl, x, res, b, h)
+    # planted needles are routed (sanity)
+    for b in range(2):
+        for h in range(wl.heads_kv):
+            assert set(S.needle_chunks(wl, 11, b, h)) <= set(res["chunk_idx"][b, h, 0])
+
+
+def test_decode_ragged_positions_and_empty_candidates():
+    """Per-sequence positions: mid-chunk, mid-group, and too early for any candidate."""
+    wl = S.workload("llama3_8b_decode_32k", batch=5, context=2048, heads_q=8, heads_kv=2,
+                    needles=0)
+    x = S.make_inputs(wl, 12)
+    pos = np.array([2047, 2047 - 37, 700, 100, 5], dtype=np.int64)
+    x["pos"] = pos
+    res = run_gpu(wl, x)
+    for b in range(5):
+        for h in range(2):
+            compare_head(wl, x, res, b, h)
+    assert (res["chunk_idx"][3:] == -1).all()      # cur - local <= sink: no candidates
+    assert (res["group_idx"][3:] == -1).all()
+
+
+@pytest.mark.parametrize("kc,chunk", [(8, 64), (64, 64), (32, 128), (64, 128)])
+def test_wide_head_sweep_small(kc, chunk):
+    wl = S.workload("wide_head_decode_64k", batch=2, context=16384, topk_chunks=kc,
+                    topk_groups=2 * kc, chunk=chunk)
+    x = S.make_inputs(wl, 13)
+    res = run_gpu(wl, x)
+    for b in range(2):
+        for h in (0, 7):
+            compare_head(wl, x, res, b, h)
+
+
+@pytest.mark.parametrize("g_heads", [1, 16])
+def test_gqa_extremes(g_heads):
+    wl = S.workload("llama3_8b_decode_32k", batch=2, context=2048, heads_q=2 * g_heads,
+                    heads_kv=2, needles=0, topk_chunks=4, topk_groups=8)
+    x = S.make_inputs(wl, 14)
+    res = run_gpu(wl, x)
+    for b in range(2):
+        for h in range(2):
+            compare_head(wl, x, res, b, h)
+
+
+def test_bf16_output_dtype():
+    wl = S.workload("llama3_8b_decode_32k", batch=2, context=2048, needles=0)
+    x = S.make_inputs(wl, 15)
+    res = run_gpu(wl, x, out_dtype=B.HGA_BF16)
+    compare_head(wl, x, res, 1, 3)
+
+
+def test_bf16_prefill_small():
+    wl = S.workload("llama3_8b_prefill_64k", context=1024, heads_q=8, heads_kv=2,
+                    topk_chunks=4, topk_groups=8)
+    x = S.make_inputs(wl, 16)
+    res = run_gpu(wl, x)
+    for h in range(2):
+        compare_head(wl, x, res, 0, h)
+
+
+# ----------------------------------------------------------- summaries / ABI
+
+def test_incremental_summaries_equal_batch_bitwise():
+    """Appending tokens one call at a time writes the same bits as one batch call."""
+    wl = S.workload("llama3_8b_decode_32k", batch=2, context=2048, heads_q=8, heads_kv=2,
+                    needles=0)
+    x = S.make_inputs(wl, 17)
+    layer = __import__("gpu_harness").layer_of(wl)
+    from gpu_harness import to_device
+    k = to_device(x["k"], wl.dtype)
+    n = wl.context
+    shape_c = (2 * 2, n // 64, 128)
+    shape_g = (2 * 2, n // 64, 4, 128)
+    cs_a = torch.zeros(shape_c, device="cuda"); gs_a = torch.zeros(shape_g, device="cuda")
+    cs_b = torch.zeros(shape_c, device="cuda"); gs_b = torch.zeros(shape_g, device="cuda")
+    B.hga_build_summaries(layer, k, n, 0, n, cs_a, gs_a)
+    start = n - 200
+    B.hga_build_summaries(layer, k, n, 0, start, cs_b, gs_b)
+    for t in range(start, n):
+        B.hga_build_summaries(layer, k, n, t, t + 1, cs_b, gs_b)
+    torch.cuda.synchronize()
+    assert torch.equal(cs_a, cs_b) and torch.equal(gs_a, gs_b)
+
+
+def test_invalid_position_sets_device_error_and_recovers():
+    wl = S.workload("llama3_8b_decode_32k", batch=2, context=1024, heads_q=8, heads_kv=2,
+                    needles=0, topk_chunks=4, topk_groups=8)
+    x = S.make_inputs(wl, 18)
+    bad = np.array([1023, 1024], dtype=np.int64)   # second sequence past the cache
+    res = run_gpu(wl, x, pos=bad, check_status=False)
+    assert res["status"] == 6  # HGA_ERR_DEVICE_CHECK
+    assert (res["chunk_idx"][1] == -1).all() and (res["group_idx"][1] == -1).all()
+    assert np.all(res["out"][1] == 0)
+    x["pos"] = np.array([1023, 1023], dtype=np.int64)
+    res = run_gpu(wl, x)  # status is clear again
+    compare_head(wl, x, res, 1, 1)
+
+
+def test_host_side_argument_errors():
+    layer = B.Layer(batch=1, heads_q=3, heads_kv=2, head_dim=128)
+    with pytest.raises(B.HGAError) as e:
+        B.hga_workspace_size(layer, 4096, 1)
+    assert e.value.status == 2
+    layer = B.Layer(batch=1, heads_q=4, heads_kv=2, head_dim=96)
+    with pytest.raises(B.HGAError) as e:
+        B.hga_workspace_size(layer, 4096, 1)
+    assert e.value.status == 3

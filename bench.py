@@ -193,55 +193,67 @@ def run_hga(args, rank: int, world: int):
     # prefix summaries (setup, untimed): every row closed before the new token
     B.hga_build_summaries(layer, k, n, 0, p, cs, gs, stream=sh)
 
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    parts = {
+        "summaries": lambda st: B.hga_build_summaries(layer, k, n, p, p + 1, cs, gs, stream=st),
+        "route_chunks": lambda st: B.hga_route_chunks(layer, q, 1, pos, cs, n, ci, stream=st),
+        "route_groups": lambda st: B.hga_route_groups(layer, q, 1, pos, gs, n, ci, gi, stream=st),
+        "attend": lambda st: B.hga_attend(layer, q, 1, pos, k, v, n, gi, out, lse, ws, wsb,
+                                          stream=st),
+    }
 
-    def step(record: bool):
-        if record:
-            ev[0].record(stream)
-        B.hga_build_summaries(layer, k, n, p, p + 1, cs, gs, stream=sh)
-        if record:
-            ev[1].record(stream)
-        B.hga_route_chunks(layer, q, 1, pos, cs, n, ci, stream=sh)
-        if record:
-            ev[2].record(stream)
-        B.hga_route_groups(layer, q, 1, pos, gs, n, ci, gi, stream=sh)
-        if record:
-            ev[3].record(stream)
-        B.hga_attend(layer, q, 1, pos, k, v, n, gi, out, lse, ws, wsb, stream=sh)
-        if record:
-            ev[4].record(stream)
+    def step(st):
+        for fn in parts.values():
+            fn(st)
+
+    # eager warm-up, then one CUDA graph for the whole step and one per call
+    for _ in range(max(1, args.warmup)):
+        step(sh)
+    torch.cuda.synchronize()
+    assert B.hga_device_status(sh) == 0
+    graphs = {}
+    for name, fn in list(parts.items()) + [("step", step)]:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(torch.cuda.current_stream().cuda_stream)
+        graphs[name] = g
+    torch.cuda.synchronize()
+
+    def timed(g, iters):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(iters)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(iters)]
+        for i in range(iters):
+            flush.zero_()              # L2 flush, outside the timed events
+            starts[i].record(stream)
+            g.replay()
+            ends[i].record(stream)
+        return starts, ends
 
     for _ in range(args.warmup):
         flush.zero_()
-        step(False)
-    torch.cuda.synchronize()
-    assert B.hga_device_status(sh) == 0
-
+        graphs["step"].replay()
     dist = None
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    per = {"step": [], "summaries": [], "route_chunks": [], "route_groups": [], "attend": []}
     with ClockSampler(torch.cuda.current_device()) as clk:
-        for _ in range(args.steps):
-            flush.zero_()
-            step(True)
-            ev[4].synchronize()
-            per["step"].append(ev[0].elapsed_time(ev[4]))
-            per["summaries"].append(ev[0].elapsed_time(ev[1]))
-            per["route_chunks"].append(ev[1].elapsed_time(ev[2]))
-            per["route_groups"].append(ev[2].elapsed_time(ev[3]))
-            per["attend"].append(ev[3].elapsed_time(ev[4]))
-    torch.cuda.synchronize()
+        starts, ends = timed(graphs["step"], args.steps)
+        torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    ms = {kk: sum(vv) / len(vv) for kk, vv in per.items()}
-    ms_step = ms["step"]
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    ms_step = sum(step_ms) / len(step_ms)
     if dist:
         t = torch.tensor([ms_step], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step = float(t.item())
+    assert B.hga_device_status(sh) == 0
+    # per-call breakdown: each call's graph replayed alone after an L2 flush
+    ms = {}
+    for name in parts:
+        a_, b_ = timed(graphs[name], min(args.steps, 200))
+        torch.cuda.synchronize()
+        ms[name] = sum(x.elapsed_time(y) for x, y in zip(a_, b_)) / len(a_)
 
     # ---- e2e: host (pinned) q and new K/V rows in, output back, every step
     q_host = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).pin_memory() \
@@ -259,7 +271,7 @@ def run_hga(args, rank: int, world: int):
         qv.copy_(q_host, non_blocking=True)
         k[:, :, p].copy_(kv_new[0], non_blocking=True)
         v[:, :, p].copy_(kv_new[1], non_blocking=True)
-        step(False)
+        graphs["step"].replay()
         out_host.copy_(out, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -309,6 +321,7 @@ def run_hga(args, rank: int, world: int):
         "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "decode tokens/s (one attention layer)",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
+        "timing": "CUDA graph of the step replayed per timed step; CUDA events on the launch stream",
         "clocks": clk.report(),
     }
     return line, wl, seed, x

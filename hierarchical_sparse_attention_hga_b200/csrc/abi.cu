@@ -135,7 +135,7 @@ hga_status hga_workspace_size(const hga_config* cfg, int64_t n_alloc, int32_t q_
   LayerParams p;
   hga_status st = make_params(cfg, n_alloc, q_len, &p);
   if (st != HGA_OK) return st;
-  *bytes = attend_workspace_bytes(p);
+  *bytes = attend_workspace_bytes(p, cfg->dtype);
   return HGA_OK;
 }
 
@@ -191,7 +191,7 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
   hga_status st = make_params(cfg, n_alloc, q_len, &p);
   if (st != HGA_OK) return st;
   if (!q || !pos || !k || !v || !group_idx || !out) return fail(HGA_ERR_INVALID_ARG, "null pointer");
-  const size_t need = attend_workspace_bytes(p);
+  const size_t need = attend_workspace_bytes(p, cfg->dtype);
   if (need && (!workspace || workspace_bytes < need))
     return fail(HGA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
   unsigned* err = nullptr;

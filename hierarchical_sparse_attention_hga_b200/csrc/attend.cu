@@ -18,6 +18,8 @@
 // CTA per (query row, KV head, split).  Decode splits the list (split-K flash
 // decoding) and a second kernel merges the partial (o, m, l) by log-sum-exp;
 // prefill rows run unsplit and write the output directly.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -250,6 +252,23 @@ combine_kernel(LayerParams p, int nsplit, const float* __restrict__ ws_o,
   if (lse && d == 0) lse[row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
 }
 
+}  // namespace
+
+cudaError_t launch_combine(const LayerParams& p, int out_dtype, int nsplit, const float* ws_o,
+                           const float* ws_ml, void* out, float* lse, cudaStream_t s) {
+  using bf = __nv_bfloat16;
+  if (p.D == 64) {
+    if (out_dtype == 0) combine_kernel<64, float><<<p.B * p.Hq, 64, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<float*>(out), lse);
+    else combine_kernel<64, bf><<<p.B * p.Hq, 64, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<bf*>(out), lse);
+  } else {
+    if (out_dtype == 0) combine_kernel<128, float><<<p.B * p.Hq, 128, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<float*>(out), lse);
+    else combine_kernel<128, bf><<<p.B * p.Hq, 128, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<bf*>(out), lse);
+  }
+  return cudaGetLastError();
+}
+
+namespace {
+
 template <typename T, int D, typename TO>
 cudaError_t launch_attend_t(const LayerParams& p, const void* q, const int64_t* pos, const void* k,
                             const void* v, const int32_t* group_idx, void* out, float* lse,
@@ -259,18 +278,15 @@ cudaError_t launch_attend_t(const LayerParams& p, const void* q, const int64_t* 
   float* ws_o = static_cast<float*>(ws);
   float* ws_ml = ws_o ? ws_o + static_cast<size_t>(p.B) * p.Hkv * nsplit * p.G * D : nullptr;
   const size_t smem = static_cast<size_t>(p.kg) * sizeof(int);
-  auto kern = attend_kernel<T, D, TO>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_smem<attend_kernel<T, D, TO>>(smem);
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(static_cast<int64_t>(p.B) * p.Hkv * p.q_len), nsplit);
-  kern<<<grid, kThreads, smem, s>>>(static_cast<const T*>(q), pos, static_cast<const T*>(k),
+  attend_kernel<T, D, TO><<<grid, kThreads, smem, s>>>(static_cast<const T*>(q), pos, static_cast<const T*>(k),
                                     static_cast<const T*>(v), group_idx, p, nsplit, split_tokens,
                                     static_cast<TO*>(out), lse, ws_o, ws_ml, err);
   e = cudaGetLastError();
   if (e != cudaSuccess || nsplit == 1) return e;
-  combine_kernel<D, TO><<<p.B * p.Hq, D, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<TO*>(out), lse);
-  return cudaGetLastError();
+  return launch_combine(p, std::is_same<TO, float>::value ? 0 : 1, nsplit, ws_o, ws_ml, out, lse, s);
 }
 
 template <typename T, typename TO>
@@ -283,7 +299,14 @@ cudaError_t launch_attend_d(const LayerParams& p, const void* q, const int64_t* 
 
 }  // namespace
 
-size_t attend_workspace_bytes(const LayerParams& p) {
+static bool use_decode_fast(const LayerParams& p, int dtype) {
+  return decode_fast_path(p, dtype) &&
+         static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc < (static_cast<int64_t>(1) << 31);
+}
+
+size_t attend_workspace_bytes(const LayerParams& p, int dtype) {
+  if (use_decode_fast(p, dtype))
+    return static_cast<size_t>(p.B) * p.Hkv * decode_fast_nsplit(p) * p.G * (p.D + 2) * sizeof(float);
   int nsplit = 1;
   choose_split_tokens(p, &nsplit);
   if (nsplit == 1) return 0;
@@ -295,6 +318,8 @@ cudaError_t launch_attend(const LayerParams& p, int dtype, int out_dtype, const 
                           const int32_t* group_idx, void* out, float* lse, void* ws,
                           unsigned* err, cudaStream_t s) {
   using bf = __nv_bfloat16;
+  if (use_decode_fast(p, dtype))
+    return launch_attend_decode_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, ws, err, s);
   if (dtype == 0)
     return out_dtype == 0 ? launch_attend_d<float, float>(p, q, pos, k, v, group_idx, out, lse, ws, err, s)
                           : launch_attend_d<float, bf>(p, q, pos, k, v, group_idx, out, lse, ws, err, s);

@@ -1,0 +1,398 @@
+// Steps 4-5 for decode, bf16 K/V with D = 128: fused gather + split-K flash
+// decoding on sm_100a.
+//
+// HGA technical summary ("Hierarchical Global Attention (HGA)", gist.science
+// 2606.30709), "Metodologia -> Meccanismo Core", item 4: the original K/V of
+// the selected tokens are fetched and attended exactly with a standard softmax.
+//
+// Every part of a decode query's token list starts on a group boundary, so the
+// list is a sequence of 16-token units, each a contiguous 16 x 256 B segment of
+// the cache: the sink chunks, the local chunks, the current chunk up to the
+// query (last unit partial) and the routed groups.  One warp owns a split of
+// consecutive units (a warp-split) and streams them through a private
+// double-buffered shared-memory ring:
+//   - lane 0 issues two 2-D TMA box loads per unit and tensor (16 rows x 64
+//     columns each, 128-byte swizzle), completing on the stage's mbarrier;
+//   - S^T = Q K^T runs on the tensor cores (mma.sync m16n8k16, bf16 -> fp32),
+//     with the G <= 16 query heads as the M rows and K fragments read with
+//     ldmatrix from the swizzled tile;
+//   - online softmax in registers (log2 domain); P stays in registers and is
+//     reused as the A operand of O += P V (V fragments via ldmatrix.trans).
+// The warp writes its partial (o, m, l); the log-sum-exp merge kernel of
+// attend.cu combines the splits.  No cluster multicast is used anywhere.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace hga {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kUnit = 16;                       // tokens per unit (= group size)
+constexpr int kWarps = 4;
+constexpr int kStages = 2;
+constexpr int kBoxBytes = kUnit * 64 * 2;       // 16 rows x 64 bf16 = 2 KB
+constexpr int kTileBytes = 2 * kBoxBytes;       // one tensor, 128 dims
+constexpr int kStageBytes = 2 * kTileBytes;     // K and V
+constexpr int kWarpBytes = kStages * kStageBytes;
+constexpr int kSmemBytes = kWarps * kWarpBytes + 1024;  // + alignment slack
+constexpr uint32_t kWaitLimit = 1u << 26;       // bounded mbarrier polls
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecodeArgs {
+  const __nv_bfloat16* q;
+  const int64_t* pos;
+  const int32_t* group_idx;
+  float* ws_o;
+  float* ws_ml;
+  unsigned* err;
+  int units_per_split;
+  int nsplit;
+};
+
+// Address of the 16-byte chunk `chunk` (0..15 over 128 dims) of row `row` in a
+// tile stored as two 128B-swizzled boxes of 64 columns.
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int chunk) {
+  const int box = chunk >> 3, c = chunk & 7;
+  return tile + box * kBoxBytes + row * 128 + ((c ^ (row & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, DecodeArgs a, LayerParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bars[kWarps][kStages];
+  __shared__ int s_gl[1024];
+  __shared__ int s_ng;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  const int split = blockIdx.x * kWarps + warp;
+
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tensormap(&tm_k);
+    ptx::prefetch_tensormap(&tm_v);
+    for (int w = 0; w < kWarps; ++w)
+      for (int s = 0; s < kStages; ++s) ptx::mbar_init(&bars[w][s], 1);
+    ptx::fence_barrier_init();
+  }
+
+  const int64_t pb = a.pos[b];
+  const bool ok = valid_position(pb, p, threadIdx.x == 0 && blockIdx.x == 0 ? a.err : nullptr);
+  const int cur = ok ? static_cast<int>(pb / p.C) : 0;
+  const int b0 = max(0, cur - p.local);
+
+  // Routed groups kept, in order: warp 0 validates and compacts them.  An id
+  // is kept when it names a group of a candidate chunk and exceeds every id
+  // kept before it (so the list is strictly ascending and has no duplicates).
+  if (warp == 0) {
+    int n = 0;
+    bool bad = false;
+    if (ok) {
+      const int32_t* gl = a.group_idx + static_cast<size_t>(bh) * p.kg;
+      int run_max = -1;
+      for (int base = 0; base < p.kg; base += 32) {
+        const int i = base + lane;
+        const int gid = i < p.kg ? gl[i] : -1;
+        const int c = gid >= 0 ? gid / p.Ng : -1;
+        const bool in_range = gid >= 0 && c >= p.sink && c < cur - p.local;
+        int incl = in_range ? gid : -1;  // inclusive prefix max over lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int x = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl = max(incl, x);
+        }
+        int excl = __shfl_up_sync(0xffffffffu, incl, 1);
+        excl = max(lane == 0 ? -1 : excl, run_max);
+        const bool keep = in_range && gid > excl;
+        bad |= __any_sync(0xffffffffu, gid >= 0 && !keep);
+        const unsigned km = __ballot_sync(0xffffffffu, keep);
+        if (keep) s_gl[n + __popc(km & ((1u << lane) - 1u))] = gid;
+        n += __popc(km);
+        run_max = max(run_max, __shfl_sync(0xffffffffu, incl, 31));
+      }
+    }
+    if (lane == 0) {
+      s_ng = n;
+      if (bad && blockIdx.x == 0) flag_error(a.err, kErrGroupIdx);
+    }
+  }
+  __syncthreads();
+
+  // Unit list: sink units [0, su), local+current units [su, su+lu), routed groups.
+  const int ng_per_c = p.C / kUnit;
+  const int su = ok ? min(p.sink, b0) * ng_per_c : 0;
+  const int u_first_local = b0 * ng_per_c;
+  const int lu = ok ? static_cast<int>(pb / kUnit) - u_first_local + 1 : 0;
+  const int n_units = su + lu + s_ng;
+  const int u_lo = split * a.units_per_split;
+  const int u_hi = min(n_units, u_lo + a.units_per_split);
+  const size_t slot = static_cast<size_t>(bh) * a.nsplit + split;
+
+  if (split >= a.nsplit) return;
+  if (u_lo >= u_hi) {
+    if (lane < p.G) {
+      a.ws_ml[(slot * p.G + lane) * 2] = -CUDART_INF_F;
+      a.ws_ml[(slot * p.G + lane) * 2 + 1] = 0.f;
+    }
+    return;
+  }
+
+  const int64_t row_base = static_cast<int64_t>(bh) * p.n_alloc;
+  auto unit_token = [&](int u) -> int64_t {
+    if (u < su) return static_cast<int64_t>(u) * kUnit;
+    u -= su;
+    if (u < lu) return static_cast<int64_t>(u_first_local + u) * kUnit;
+    return static_cast<int64_t>(s_gl[u - lu]) * kUnit;
+  };
+  // Valid tokens in unit u (only the unit holding the query can be partial).
+  auto unit_valid = [&](int u) -> int {
+    if (u == su + lu - 1) return static_cast<int>(pb % kUnit) + 1;
+    return kUnit;
+  };
+
+  uint8_t* wsm = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023) + warp * kWarpBytes;
+  const uint32_t wsm_u32 = ptx::smem_u32(wsm);
+  uint64_t* wbar = bars[warp];
+
+  auto issue = [&](int u, int stage) {
+    if (lane == 0) {
+      const int32_t y = static_cast<int32_t>(row_base + unit_token(u));
+      uint8_t* st = wsm + stage * kStageBytes;
+      ptx::mbar_expect_tx(&wbar[stage], kStageBytes);
+      ptx::tma_load_2d(st, &tm_k, &wbar[stage], 0, y);
+      ptx::tma_load_2d(st + kBoxBytes, &tm_k, &wbar[stage], 64, y);
+      ptx::tma_load_2d(st + kTileBytes, &tm_v, &wbar[stage], 0, y);
+      ptx::tma_load_2d(st + kTileBytes + kBoxBytes, &tm_v, &wbar[stage], 64, y);
+    }
+  };
+  issue(u_lo, 0);
+  if (u_lo + 1 < u_hi) issue(u_lo + 1, 1);
+
+  // Q as m16n8k16 A fragments: rows = query heads (g, g+8), k = dims.
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t qa[8][4];
+  {
+    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(
+        a.q + (static_cast<size_t>(b) * p.Hq + h * p.G + g) * kD);
+    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(
+        a.q + (static_cast<size_t>(b) * p.Hq + h * p.G + g + 8) * kD);
+    const bool r0 = g < p.G, r1 = g + 8 < p.G;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      qa[kk][0] = r0 ? __ldg(q0 + kk * 8 + t) : 0u;
+      qa[kk][1] = r1 ? __ldg(q1 + kk * 8 + t) : 0u;
+      qa[kk][2] = r0 ? __ldg(q0 + kk * 8 + 4 + t) : 0u;
+      qa[kk][3] = r1 ? __ldg(q1 + kk * 8 + 4 + t) : 0u;
+    }
+  }
+  const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
+
+  float o[16][4];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F;  // rows g and g+8
+  float l0 = 0.f, l1 = 0.f;                      // this lane's partial sums
+
+  // ldmatrix lane roles
+  const int mi = lane >> 3, ri = lane & 7;
+  bool timed_out = false;
+
+  for (int u = u_lo; u < u_hi; ++u) {
+    const int it = u - u_lo;
+    const int stage = it & 1;
+    if (!ptx::mbar_wait(&wbar[stage], (it >> 1) & 1, kWaitLimit)) { timed_out = true; break; }
+    const uint32_t kt = wsm_u32 + stage * kStageBytes;
+    const uint32_t vt = kt + kTileBytes;
+    const int valid = unit_valid(u);
+
+    // S^T[head, token] for tokens 0-7 (s[0]) and 8-15 (s[1])
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t r[4];
+      const int tok = (mi >> 1) * 8 + ri;
+      ptx::ldmatrix_x4(swz(kt, tok, kk * 2 + (mi & 1)), r);
+      ptx::mma_bf16_16816(s[0], qa[kk], r[0], r[1]);
+      ptx::mma_bf16_16816(s[1], qa[kk], r[2], r[3]);
+    }
+    // scale into log2 units, mask tokens past the query
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = nt * 8 + 2 * t + (e & 1);
+        s[nt][e] = tok < valid ? s[nt][e] * sc : -CUDART_INF_F;
+      }
+    }
+    float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+    float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+    const float c0 = exp2f(m0 - n0), c1 = exp2f(m1 - n1);  // 0 while m is -inf
+    m0 = n0;
+    m1 = n1;
+    float pr[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      pr[nt][0] = exp2f(s[nt][0] - n0);
+      pr[nt][1] = exp2f(s[nt][1] - n0);
+      pr[nt][2] = exp2f(s[nt][2] - n1);
+      pr[nt][3] = exp2f(s[nt][3] - n1);
+    }
+    l0 = l0 * c0 + pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
+    l1 = l1 * c1 + pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      o[j][0] *= c0; o[j][1] *= c0;
+      o[j][2] *= c1; o[j][3] *= c1;
+    }
+    uint32_t pa[4];
+    pa[0] = ptx::pack_bf16x2(pr[0][0], pr[0][1]);
+    pa[1] = ptx::pack_bf16x2(pr[0][2], pr[0][3]);
+    pa[2] = ptx::pack_bf16x2(pr[1][0], pr[1][1]);
+    pa[3] = ptx::pack_bf16x2(pr[1][2], pr[1][3]);
+    // Tokens past the query may hold anything (even NaN) in the cache: their
+    // V rows must not reach the product, so zero them in the tile.
+    if (valid < kUnit) {
+      __syncwarp();
+      for (int i = lane; i < (kUnit - valid) * 16; i += 32) {
+        const int row = valid + i / 16, chunk = i % 16;
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(swz(vt, row, chunk)), "r"(0u));
+      }
+      ptx::fence_proxy_async();  // the stage is refilled by TMA later
+      __syncwarp();
+    }
+#pragma unroll
+    for (int nn = 0; nn < 8; ++nn) {
+      uint32_t r[4];
+      const int tok = (mi & 1) * 8 + ri;
+      ptx::ldmatrix_x4_trans(swz(vt, tok, nn * 2 + (mi >> 1)), r);
+      ptx::mma_bf16_16816(o[2 * nn], pa, r[0], r[1]);
+      ptx::mma_bf16_16816(o[2 * nn + 1], pa, r[2], r[3]);
+    }
+    __syncwarp();
+    if (u + 2 < u_hi) issue(u + 2, stage);
+  }
+
+  if (timed_out) {
+    if (lane == 0) flag_error(a.err, kErrTimeout);
+    return;
+  }
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  if (g < p.G) {
+    float* dst = a.ws_o + (slot * p.G + g) * kD;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      *reinterpret_cast<float2*>(dst + j * 8 + 2 * t) = make_float2(o[j][0], o[j][1]);
+    if (t == 0) {
+      a.ws_ml[(slot * p.G + g) * 2] = m0;
+      a.ws_ml[(slot * p.G + g) * 2 + 1] = l0;
+    }
+  }
+  if (g + 8 < p.G) {
+    float* dst = a.ws_o + (slot * p.G + g + 8) * kD;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      *reinterpret_cast<float2*>(dst + j * 8 + 2 * t) = make_float2(o[j][2], o[j][3]);
+    if (t == 0) {
+      a.ws_ml[(slot * p.G + g + 8) * 2] = m1;
+      a.ws_ml[(slot * p.G + g + 8) * 2 + 1] = l1;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// Tensor map of a [rows, 128] bf16 cache, boxes of 16 rows x 64 columns, 128B swizzle.
+cudaError_t make_map(CUtensorMap* map, const void* base, int64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  const cuuint32_t box[2] = {64, kUnit};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int max_units(const LayerParams& p) {
+  return (p.sink + p.local + 1) * (p.C / kUnit) + p.kg;
+}
+
+int choose_units_per_split(const LayerParams& p) {
+  const int64_t total = static_cast<int64_t>(p.B) * p.Hkv * max_units(p);
+  const int64_t warps = 148 * 12;  // ~3 CTAs of 4 warps per SM
+  int64_t u = (total + warps - 1) / warps;
+  return static_cast<int>(u < 1 ? 1 : (u > 16 ? 16 : u));
+}
+
+}  // namespace
+
+bool decode_fast_path(const LayerParams& p, int dtype) {
+  return dtype == 1 && p.D == kD && p.q_len == 1 && p.g == kUnit && p.kg <= 1024 && p.G <= 16;
+}
+
+int decode_fast_nsplit(const LayerParams& p) {
+  const int u = choose_units_per_split(p);
+  return (max_units(p) + u - 1) / u;
+}
+
+cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const void* q,
+                                      const int64_t* pos, const void* k, const void* v,
+                                      const int32_t* group_idx, void* out, float* lse, void* ws,
+                                      unsigned* err, cudaStream_t s) {
+  CUtensorMap tk, tv;
+  const int64_t rows = static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc;
+  cudaError_t e = make_map(&tk, k, rows);
+  if (e == cudaSuccess) e = make_map(&tv, v, rows);
+  if (e != cudaSuccess) return e;
+  const int ups = choose_units_per_split(p);
+  const int nsplit = decode_fast_nsplit(p);
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.pos = pos;
+  a.group_idx = group_idx;
+  a.ws_o = static_cast<float*>(ws);
+  a.ws_ml = a.ws_o + static_cast<size_t>(p.B) * p.Hkv * nsplit * p.G * kD;
+  a.err = err;
+  a.units_per_split = ups;
+  a.nsplit = nsplit;
+  e = ensure_smem<attend_decode_bf16_kernel>(kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((nsplit + kWarps - 1) / kWarps, p.B * p.Hkv);
+  attend_decode_bf16_kernel<<<grid, kWarps * 32, kSmemBytes, s>>>(tk, tv, a, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_combine(p, out_dtype, nsplit, a.ws_o, a.ws_ml, out, lse, s);
+}
+
+}  // namespace hga

@@ -5,9 +5,32 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace hga {
+
+// Raises the dynamic shared-memory limit of kernel Kern on the current device
+// to at least `bytes`, calling cudaFuncSetAttribute only the first time a
+// larger value is needed on that device.
+template <auto Kern>
+cudaError_t ensure_smem(size_t bytes) {
+  static std::atomic<int> done[64];
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int want = static_cast<int>(bytes);
+  if (dev >= 0 && dev < 64 && done[dev].load() >= want) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, want);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) {
+    int cur = done[dev].load();
+    while (cur < want && !done[dev].compare_exchange_weak(cur, want)) {
+    }
+  }
+  return e;
+}
 
 // dtype: 0 = float32, 1 = bfloat16 (hga_dtype values).
 cudaError_t launch_summaries(const LayerParams& p, int dtype, const void* k, int64_t t_begin,
@@ -23,7 +46,19 @@ cudaError_t launch_route_groups(const LayerParams& p, int dtype, const void* q, 
                                 cudaStream_t s);
 
 // Workspace bytes of launch_attend for p (0 when the launch needs none).
-size_t attend_workspace_bytes(const LayerParams& p);
+size_t attend_workspace_bytes(const LayerParams& p, int dtype);
+
+// The bf16, D = 128 decode kernel (TMA + mma.sync) applies to p.
+bool decode_fast_path(const LayerParams& p, int dtype);
+int decode_fast_nsplit(const LayerParams& p);
+cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const void* q,
+                                      const int64_t* pos, const void* k, const void* v,
+                                      const int32_t* group_idx, void* out, float* lse, void* ws,
+                                      unsigned* err, cudaStream_t s);
+
+// Log-sum-exp merge of nsplit decode partials into out / lse.
+cudaError_t launch_combine(const LayerParams& p, int out_dtype, int nsplit, const float* ws_o,
+                           const float* ws_ml, void* out, float* lse, cudaStream_t s);
 
 cudaError_t launch_attend(const LayerParams& p, int dtype, int out_dtype, const void* q,
                           const int64_t* pos, const void* k, const void* v,

@@ -10,7 +10,7 @@
 // One CTA per (sequence, KV head, query block).  The routing query is the mean
 // of the block's post-RoPE query rows over the G heads sharing the KV head,
 // summed in a fixed order (deterministic).  Summary rows are streamed with
-// 16-byte loads, one row per D/4 lanes, four rows in flight per lane; scores
+// 16-byte loads, one row per D/4 lanes, eight rows in flight per lane; scores
 // land in shared memory and a block radix select keeps the top-k.
 #include "common.cuh"
 #include "kernels.h"
@@ -58,7 +58,7 @@ template <int D, typename RowFn>
 __device__ void score_rows(int n, const float* qbar, float* sc, RowFn row) {
   constexpr int LPR = D / 4;          // lanes per row
   constexpr int RPW = 32 / LPR;       // rows per warp step
-  constexpr int UNR = 4;
+  constexpr int UNR = 8;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int sub = lane / LPR, l = lane % LPR;
   const float4 qv = reinterpret_cast<const float4*>(qbar)[l];
@@ -211,11 +211,9 @@ cudaError_t launch_route_chunks_t(const LayerParams& p, const void* q, const int
                                   const float* chunk_sum, int32_t* chunk_idx, float* chunk_score,
                                   unsigned* err, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(p.n_chunks) * sizeof(float) + p.kc * sizeof(int);
-  auto kern = route_chunks_kernel<T, D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_smem<route_chunks_kernel<T, D>>(smem);
   if (e != cudaSuccess) return e;
-  kern<<<p.B * p.Hkv * p.nblk, kThreads, smem, s>>>(static_cast<const T*>(q), pos, chunk_sum, p,
+  route_chunks_kernel<T, D><<<p.B * p.Hkv * p.nblk, kThreads, smem, s>>>(static_cast<const T*>(q), pos, chunk_sum, p,
                                                     chunk_idx, chunk_score, err);
   return cudaGetLastError();
 }
@@ -227,11 +225,9 @@ cudaError_t launch_route_groups_t(const LayerParams& p, const void* q, const int
                                   cudaStream_t s) {
   const size_t smem = static_cast<size_t>(p.kc) * p.Ng * sizeof(float) +
                       static_cast<size_t>(p.kg + p.kc) * sizeof(int);
-  auto kern = route_groups_kernel<T, D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_smem<route_groups_kernel<T, D>>(smem);
   if (e != cudaSuccess) return e;
-  kern<<<p.B * p.Hkv * p.nblk, kThreads, smem, s>>>(static_cast<const T*>(q), pos, group_sum,
+  route_groups_kernel<T, D><<<p.B * p.Hkv * p.nblk, kThreads, smem, s>>>(static_cast<const T*>(q), pos, group_sum,
                                                     chunk_idx, p, group_idx, group_score, err);
   return cudaGetLastError();
 }

@@ -169,3 +169,34 @@ def test_host_side_argument_errors():
     with pytest.raises(B.HGAError) as e:
         B.hga_workspace_size(layer, 4096, 1)
     assert e.value.status == 3
+
+
+def test_bf16_head_dim_64_decode():
+    """bf16 with D=64 takes the general kernel; parity holds there too."""
+    wl = S.workload("llama3_8b_decode_32k", batch=2, context=2048, head_dim=64, n_high_pairs=16,
+                    heads_q=8, heads_kv=2, needles=0)
+    x = S.make_inputs(wl, 19)
+    res = run_gpu(wl, x)
+    for b in range(2):
+        for h in range(2):
+            compare_summaries(wl, x, res, b, h)
+            compare_head(wl, x, res, b, h)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_cache_past_the_query_is_never_read_into_the_output(dtype):
+    """Rows after the query position may hold anything (here NaN): outputs stay exact."""
+    wl = S.workload("llama3_8b_decode_32k", batch=2, context=2048, heads_q=8, heads_kv=2,
+                    needles=0, dtype=dtype)
+    x = S.make_inputs(wl, 20)
+    pos = np.array([2047 - 5, 2047 - 16 - 9], dtype=np.int64)
+    x["pos"] = pos
+    nan = np.uint16(0x7FC0) if dtype == "bf16" else np.float32("nan")
+    for b in range(2):
+        x["k"][b, :, pos[b] + 1:] = nan
+        x["v"][b, :, pos[b] + 1:] = nan
+    res = run_gpu(wl, x, summaries_range=(0, int(pos.min()) + 1))
+    assert np.isfinite(res["out"]).all()
+    for b in range(2):
+        for h in range(2):
+            compare_head(wl, x, res, b, h)

@@ -93,6 +93,8 @@ attend_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos, const T*
   const int h = bh % p.Hkv, b = bh / p.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int d = tid % D;
+  pdl_wait();
+  pdl_trigger();
 
   const int64_t pb = pos[b];
   const bool ok = valid_position(pb, p, tid == 0 && split == 0 ? err : nullptr);
@@ -234,6 +236,8 @@ combine_kernel(LayerParams p, int nsplit, const float* __restrict__ ws_o,
   const int h = hq / p.G, hh = hq % p.G;
   const int bh = b * p.Hkv + h;
   const int d = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   float m = -CUDART_INF_F;
   for (int s = 0; s < nsplit; ++s) m = fmaxf(m, ws_ml[((static_cast<size_t>(bh) * nsplit + s) * p.G + hh) * 2]);
   float l = 0.f, o = 0.f;
@@ -257,14 +261,18 @@ combine_kernel(LayerParams p, int nsplit, const float* __restrict__ ws_o,
 cudaError_t launch_combine(const LayerParams& p, int out_dtype, int nsplit, const float* ws_o,
                            const float* ws_ml, void* out, float* lse, cudaStream_t s) {
   using bf = __nv_bfloat16;
-  if (p.D == 64) {
-    if (out_dtype == 0) combine_kernel<64, float><<<p.B * p.Hq, 64, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<float*>(out), lse);
-    else combine_kernel<64, bf><<<p.B * p.Hq, 64, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<bf*>(out), lse);
-  } else {
-    if (out_dtype == 0) combine_kernel<128, float><<<p.B * p.Hq, 128, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<float*>(out), lse);
-    else combine_kernel<128, bf><<<p.B * p.Hq, 128, 0, s>>>(p, nsplit, ws_o, ws_ml, static_cast<bf*>(out), lse);
-  }
-  return cudaGetLastError();
+  const dim3 grid(p.B * p.Hq);
+  if (p.D == 64)
+    return out_dtype == 0
+               ? launch_pdl(combine_kernel<64, float>, grid, dim3(64), 0, s, 1, p, nsplit, ws_o,
+                            ws_ml, static_cast<float*>(out), lse)
+               : launch_pdl(combine_kernel<64, bf>, grid, dim3(64), 0, s, 1, p, nsplit, ws_o,
+                            ws_ml, static_cast<bf*>(out), lse);
+  return out_dtype == 0
+             ? launch_pdl(combine_kernel<128, float>, grid, dim3(128), 0, s, 1, p, nsplit, ws_o,
+                          ws_ml, static_cast<float*>(out), lse)
+             : launch_pdl(combine_kernel<128, bf>, grid, dim3(128), 0, s, 1, p, nsplit, ws_o,
+                          ws_ml, static_cast<bf*>(out), lse);
 }
 
 namespace {
@@ -281,10 +289,10 @@ cudaError_t launch_attend_t(const LayerParams& p, const void* q, const int64_t* 
   cudaError_t e = ensure_smem<attend_kernel<T, D, TO>>(smem);
   if (e != cudaSuccess) return e;
   dim3 grid(static_cast<unsigned>(static_cast<int64_t>(p.B) * p.Hkv * p.q_len), nsplit);
-  attend_kernel<T, D, TO><<<grid, kThreads, smem, s>>>(static_cast<const T*>(q), pos, static_cast<const T*>(k),
-                                    static_cast<const T*>(v), group_idx, p, nsplit, split_tokens,
-                                    static_cast<TO*>(out), lse, ws_o, ws_ml, err);
-  e = cudaGetLastError();
+  e = launch_pdl(attend_kernel<T, D, TO>, grid, dim3(kThreads), smem, s, 1,
+                 static_cast<const T*>(q), pos, static_cast<const T*>(k),
+                 static_cast<const T*>(v), group_idx, p, nsplit, split_tokens,
+                 static_cast<TO*>(out), lse, ws_o, ws_ml, err);
   if (e != cudaSuccess || nsplit == 1) return e;
   return launch_combine(p, std::is_same<TO, float>::value ? 0 : 1, nsplit, ws_o, ws_ml, out, lse, s);
 }

@@ -81,11 +81,76 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
       for (int s = 0; s < kStages; ++s) ptx::mbar_init(&bars[w][s], 1);
     ptx::fence_barrier_init();
   }
+  __syncthreads();
 
+  // Everything up to pdl_wait() reads only pos, k and v (never written by this
+  // library), so it overlaps the routing kernel still running ahead of us.
   const int64_t pb = a.pos[b];
   const bool ok = valid_position(pb, p, threadIdx.x == 0 && blockIdx.x == 0 ? a.err : nullptr);
   const int cur = ok ? static_cast<int>(pb / p.C) : 0;
   const int b0 = max(0, cur - p.local);
+  // Unit list: sink units [0, su), local+current units [su, su+lu), routed groups.
+  const int ng_per_c = p.C / kUnit;
+  const int su = ok ? min(p.sink, b0) * ng_per_c : 0;
+  const int u_first_local = b0 * ng_per_c;
+  const int lu = ok ? static_cast<int>(pb / kUnit) - u_first_local + 1 : 0;
+  const int n_forced = su + lu;
+  const int u_lo = split * a.units_per_split;
+  const int u_cap = u_lo + a.units_per_split;
+  const int64_t row_base = static_cast<int64_t>(bh) * p.n_alloc;
+  auto unit_token = [&](int u) -> int64_t {
+    if (u < su) return static_cast<int64_t>(u) * kUnit;
+    u -= su;
+    if (u < lu) return static_cast<int64_t>(u_first_local + u) * kUnit;
+    return static_cast<int64_t>(s_gl[u - lu]) * kUnit;
+  };
+  // Valid tokens in unit u (only the unit holding the query can be partial).
+  auto unit_valid = [&](int u) -> int {
+    if (u == n_forced - 1) return static_cast<int>(pb % kUnit) + 1;
+    return kUnit;
+  };
+  uint8_t* wsm = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023) + warp * kWarpBytes;
+  const uint32_t wsm_u32 = ptx::smem_u32(wsm);
+  uint64_t* wbar = bars[warp];
+  auto issue = [&](int u, int stage) {
+    if (lane == 0) {
+      const int32_t y = static_cast<int32_t>(row_base + unit_token(u));
+      uint8_t* st = wsm + stage * kStageBytes;
+      ptx::mbar_expect_tx(&wbar[stage], kStageBytes);
+      ptx::tma_load_2d(st, &tm_k, &wbar[stage], 0, y);
+      ptx::tma_load_2d(st + kBoxBytes, &tm_k, &wbar[stage], 64, y);
+      ptx::tma_load_2d(st + kTileBytes, &tm_v, &wbar[stage], 0, y);
+      ptx::tma_load_2d(st + kTileBytes + kBoxBytes, &tm_v, &wbar[stage], 64, y);
+    }
+  };
+  // Forced units (sink, local, current) do not depend on routing: start them now.
+  const bool live = split < a.nsplit;
+  const int pre0 = live && u_lo < n_forced ? 1 : 0;
+  const int pre1 = live && u_lo + 1 < n_forced && u_lo + 1 < u_cap ? 1 : 0;
+  if (pre0) issue(u_lo, 0);
+  if (pre1) issue(u_lo + 1, 1);
+
+  // Q as m16n8k16 A fragments: rows = query heads (g, g+8), k = dims.
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t qa[8][4];
+  {
+    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(
+        a.q + (static_cast<size_t>(b) * p.Hq + h * p.G + g) * kD);
+    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(
+        a.q + (static_cast<size_t>(b) * p.Hq + h * p.G + g + 8) * kD);
+    const bool r0 = g < p.G, r1 = g + 8 < p.G;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      qa[kk][0] = r0 ? __ldg(q0 + kk * 8 + t) : 0u;
+      qa[kk][1] = r1 ? __ldg(q1 + kk * 8 + t) : 0u;
+      qa[kk][2] = r0 ? __ldg(q0 + kk * 8 + 4 + t) : 0u;
+      qa[kk][3] = r1 ? __ldg(q1 + kk * 8 + 4 + t) : 0u;
+    }
+  }
+  const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
+
+  pdl_wait();
+  pdl_trigger();
 
   // Routed groups kept, in order: warp 0 validates and compacts them.  An id
   // is kept when it names a group of a candidate chunk and exceeds every id
@@ -124,17 +189,11 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
   __syncthreads();
 
-  // Unit list: sink units [0, su), local+current units [su, su+lu), routed groups.
-  const int ng_per_c = p.C / kUnit;
-  const int su = ok ? min(p.sink, b0) * ng_per_c : 0;
-  const int u_first_local = b0 * ng_per_c;
-  const int lu = ok ? static_cast<int>(pb / kUnit) - u_first_local + 1 : 0;
-  const int n_units = su + lu + s_ng;
-  const int u_lo = split * a.units_per_split;
-  const int u_hi = min(n_units, u_lo + a.units_per_split);
+  const int n_units = n_forced + s_ng;
+  const int u_hi = min(n_units, u_cap);
   const size_t slot = static_cast<size_t>(bh) * a.nsplit + split;
 
-  if (split >= a.nsplit) return;
+  if (!live) return;
   if (u_lo >= u_hi) {
     if (lane < p.G) {
       a.ws_ml[(slot * p.G + lane) * 2] = -CUDART_INF_F;
@@ -142,56 +201,9 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     return;
   }
+  if (!pre0) issue(u_lo, 0);
+  if (!pre1 && u_lo + 1 < u_hi) issue(u_lo + 1, 1);
 
-  const int64_t row_base = static_cast<int64_t>(bh) * p.n_alloc;
-  auto unit_token = [&](int u) -> int64_t {
-    if (u < su) return static_cast<int64_t>(u) * kUnit;
-    u -= su;
-    if (u < lu) return static_cast<int64_t>(u_first_local + u) * kUnit;
-    return static_cast<int64_t>(s_gl[u - lu]) * kUnit;
-  };
-  // Valid tokens in unit u (only the unit holding the query can be partial).
-  auto unit_valid = [&](int u) -> int {
-    if (u == su + lu - 1) return static_cast<int>(pb % kUnit) + 1;
-    return kUnit;
-  };
-
-  uint8_t* wsm = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023) + warp * kWarpBytes;
-  const uint32_t wsm_u32 = ptx::smem_u32(wsm);
-  uint64_t* wbar = bars[warp];
-
-  auto issue = [&](int u, int stage) {
-    if (lane == 0) {
-      const int32_t y = static_cast<int32_t>(row_base + unit_token(u));
-      uint8_t* st = wsm + stage * kStageBytes;
-      ptx::mbar_expect_tx(&wbar[stage], kStageBytes);
-      ptx::tma_load_2d(st, &tm_k, &wbar[stage], 0, y);
-      ptx::tma_load_2d(st + kBoxBytes, &tm_k, &wbar[stage], 64, y);
-      ptx::tma_load_2d(st + kTileBytes, &tm_v, &wbar[stage], 0, y);
-      ptx::tma_load_2d(st + kTileBytes + kBoxBytes, &tm_v, &wbar[stage], 64, y);
-    }
-  };
-  issue(u_lo, 0);
-  if (u_lo + 1 < u_hi) issue(u_lo + 1, 1);
-
-  // Q as m16n8k16 A fragments: rows = query heads (g, g+8), k = dims.
-  const int g = lane >> 2, t = lane & 3;
-  uint32_t qa[8][4];
-  {
-    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(
-        a.q + (static_cast<size_t>(b) * p.Hq + h * p.G + g) * kD);
-    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(
-        a.q + (static_cast<size_t>(b) * p.Hq + h * p.G + g + 8) * kD);
-    const bool r0 = g < p.G, r1 = g + 8 < p.G;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      qa[kk][0] = r0 ? __ldg(q0 + kk * 8 + t) : 0u;
-      qa[kk][1] = r1 ? __ldg(q1 + kk * 8 + t) : 0u;
-      qa[kk][2] = r0 ? __ldg(q0 + kk * 8 + 4 + t) : 0u;
-      qa[kk][3] = r1 ? __ldg(q1 + kk * 8 + 4 + t) : 0u;
-    }
-  }
-  const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
 
   float o[16][4];
 #pragma unroll
@@ -389,8 +401,8 @@ cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const
   e = ensure_smem<attend_decode_bf16_kernel>(kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((nsplit + kWarps - 1) / kWarps, p.B * p.Hkv);
-  attend_decode_bf16_kernel<<<grid, kWarps * 32, kSmemBytes, s>>>(tk, tv, a, p);
-  e = cudaGetLastError();
+  e = launch_pdl(attend_decode_bf16_kernel, grid, dim3(kWarps * 32), kSmemBytes, s, 1, tk, tv, a,
+                 p);
   if (e != cudaSuccess) return e;
   return launch_combine(p, out_dtype, nsplit, a.ws_o, a.ws_ml, out, lse, s);
 }

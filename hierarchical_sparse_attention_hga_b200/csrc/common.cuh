@@ -58,6 +58,17 @@ __device__ __forceinline__ void load2(const __nv_bfloat16* p, float (&o)[2]) {
   o[0] = __uint_as_float(v << 16); o[1] = __uint_as_float(v & 0xffff0000u);
 }
 
+// Programmatic dependent launch.  Every kernel of the library launches with the
+// programmatic-serialization attribute, waits for its stream predecessor before
+// reading anything a predecessor may have written, and only then lets its own
+// dependents launch.  So the code a kernel runs before pdl_wait() overlaps the
+// tail of its predecessor and may read only data no kernel of this library
+// writes (q, pos, k, v).  Without the attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void flag_error(unsigned* err, unsigned bit) {
   if (err) atomicOr(err, bit);
 }

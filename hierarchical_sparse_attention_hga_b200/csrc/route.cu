@@ -12,15 +12,22 @@
 // summed in a fixed order (deterministic).  Summary rows are streamed with
 // 16-byte loads, one row per D/4 lanes, eight rows in flight per lane; scores
 // land in shared memory and a block radix select keeps the top-k.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "topk.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace hga {
 namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+// Below this many candidates the one-pass rank count beats the 4-pass radix
+// select; above it the rank count's O(n) serial compare chain per thread loses.
+constexpr int kRankTopkMax = 128;
 
 // qbar[0..D) = mean of the q rows (G heads x nr rows) of (b, KV head h).
 template <typename T, int D>
@@ -94,6 +101,10 @@ __device__ __forceinline__ void block_rows(const LayerParams& p, int64_t pos, in
   *cur = static_cast<int>((first + *r0 + *nr - 1) / p.C);
 }
 
+// One cluster of `cl` CTAs per (sequence, KV head, block): CTA r scores the
+// r-th slice of the candidates into its own shared memory; after a cluster
+// barrier, CTA 0 gathers every slice through distributed shared memory and
+// runs the top-k.  With cl == 1 this is a plain single-CTA scan.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 route_chunks_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
@@ -104,31 +115,53 @@ route_chunks_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
   __shared__ float part[kWarps][D];
   __shared__ TopkSmem tsm;
   extern __shared__ __align__(16) float dyn[];
-  const int item = blockIdx.x;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int cl = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int item = blockIdx.x / cl;
   const int blk = item % p.nblk;
   const int bh = item / p.nblk;
   const int h = bh % p.Hkv, b = bh / p.Hkv;
   int32_t* out = chunk_idx + static_cast<size_t>(item) * p.kc;
   float* out_sc = chunk_score ? chunk_score + static_cast<size_t>(item) * p.kc : nullptr;
   const int64_t pb = pos[b];
-  if (!valid_position(pb, p, threadIdx.x == 0 ? err : nullptr)) {
+  const bool ok = valid_position(pb, p, threadIdx.x == 0 && rank == 0 ? err : nullptr);
+  int r0 = 0, nr = 0, cur = 0;
+  if (ok) {
+    block_rows(p, pb, blk, &r0, &nr, &cur);
+    routing_query<T, D>(q, p, b, h, r0, nr, qbar, part);  // q is never written by this library
+  }
+  pdl_wait();
+  pdl_trigger();
+
+  const int n_cand = ok ? max(0, cur - p.local - p.sink) : 0;
+  const int per = ((p.n_chunks + cl - 1) / cl + 3) & ~3;  // slice capacity (keeps sc 16 B aligned)
+  float* local = dyn;                                 // [per]: this CTA's slice
+  float* sc = cl == 1 ? dyn : dyn + per;              // [n_chunks]: gathered (rank 0)
+  int* sel = reinterpret_cast<int*>(sc + p.n_chunks); // [kc]
+  const int slice = (n_cand + cl - 1) / cl;
+  const int lo = min(n_cand, rank * slice), hi = min(n_cand, lo + slice);
+  const float* rows = chunk_sum + (static_cast<size_t>(bh) * p.n_chunks + p.sink + lo) * D;
+  score_rows<D>(hi - lo, qbar, local, [&](int i) { return rows + static_cast<size_t>(i) * D; });
+  cluster.sync();
+  if (rank == 0 && cl > 1) {
+    for (int i = threadIdx.x; i < n_cand; i += kThreads) {
+      const int r = i / slice;
+      const float* src = cluster.map_shared_rank(local, r);
+      sc[i] = src[i - r * slice];
+    }
+  }
+  cluster.sync();  // remote slices read; the other CTAs may leave
+  if (rank != 0) return;
+  if (!ok) {
     for (int i = threadIdx.x; i < p.kc; i += kThreads) {
       out[i] = -1;
       if (out_sc) out_sc[i] = CUDART_NAN_F;
     }
     return;
   }
-  int r0, nr, cur;
-  block_rows(p, pb, blk, &r0, &nr, &cur);
-  routing_query<T, D>(q, p, b, h, r0, nr, qbar, part);
-
-  const int n_cand = max(0, cur - p.local - p.sink);
-  float* sc = dyn;                                   // [n_chunks]
-  int* sel = reinterpret_cast<int*>(dyn + p.n_chunks);  // [kc]
-  const float* rows = chunk_sum + (static_cast<size_t>(bh) * p.n_chunks + p.sink) * D;
-  score_rows<D>(n_cand, qbar, sc, [&](int i) { return rows + static_cast<size_t>(i) * D; });
-  __syncthreads();
-  const int ns = block_topk<kThreads>(sc, n_cand, p.kc, sel, tsm);
+  const int ns = n_cand <= kRankTopkMax ? block_topk_rank<kThreads>(sc, n_cand, p.kc, sel, tsm)
+                                       : block_topk<kThreads>(sc, n_cand, p.kc, sel, tsm);
   for (int i = threadIdx.x; i < p.kc; i += kThreads) {
     out[i] = i < ns ? sel[i] + p.sink : -1;
     if (out_sc) out_sc[i] = i < ns ? sc[sel[i]] : CUDART_NAN_F;
@@ -154,6 +187,8 @@ route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
   float* out_sc = group_score ? group_score + static_cast<size_t>(item) * p.kg : nullptr;
   const int64_t pb = pos[b];
   if (!valid_position(pb, p, threadIdx.x == 0 ? err : nullptr)) {
+    pdl_wait();
+    pdl_trigger();
     for (int i = threadIdx.x; i < p.kg; i += kThreads) {
       out[i] = -1;
       if (out_sc) out_sc[i] = CUDART_NAN_F;
@@ -162,29 +197,26 @@ route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
   }
   int r0, nr, cur;
   block_rows(p, pb, blk, &r0, &nr, &cur);
+  routing_query<T, D>(q, p, b, h, r0, nr, qbar, part);  // q is never written by this library
+  pdl_wait();
+  pdl_trigger();
 
   const int n_cand_max = p.kc * p.Ng;
   float* sc = dyn;                                        // [kc * Ng]
   int* sel = reinterpret_cast<int*>(dyn + n_cand_max);    // [kg]
   int* chunks = sel + p.kg;                               // [kc]
   const int32_t* cidx = chunk_idx + static_cast<size_t>(item) * p.kc;
-  for (int i = threadIdx.x; i < p.kc; i += kThreads) chunks[i] = cidx[i];
-  __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
     // Keep the ascending complete candidate chunks; flag anything else.
-    int n = 0, prev = -1;
     bool bad = false;
-    for (int i = 0; i < p.kc; ++i) {
-      const int c = chunks[i];
-      if (c < 0) continue;
-      if (c < p.sink || c >= cur - p.local || c <= prev) { bad = true; continue; }
-      chunks[n++] = c;
-      prev = c;
+    const int n = warp_keep_ascending(
+        cidx, p.kc, [&](int c) { return c >= p.sink && c < cur - p.local; }, chunks, &bad);
+    if (threadIdx.x == 0) {
+      n_sel = n;
+      if (bad) flag_error(err, kErrChunkIdx);
     }
-    n_sel = n;
-    if (bad) flag_error(err, kErrChunkIdx);
   }
-  routing_query<T, D>(q, p, b, h, r0, nr, qbar, part);  // syncs: n_sel and chunks visible
+  __syncthreads();
 
   const int n_cand = n_sel * p.Ng;
   const float* base = group_sum + static_cast<size_t>(bh) * p.n_chunks * p.Ng * D;
@@ -193,7 +225,8 @@ route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
     return base + (static_cast<size_t>(c) * p.Ng + gi) * D;
   });
   __syncthreads();
-  const int ns = block_topk<kThreads>(sc, n_cand, p.kg, sel, tsm);
+  const int ns = n_cand <= kRankTopkMax ? block_topk_rank<kThreads>(sc, n_cand, p.kg, sel, tsm)
+                                       : block_topk<kThreads>(sc, n_cand, p.kg, sel, tsm);
   for (int i = threadIdx.x; i < p.kg; i += kThreads) {
     if (i < ns) {
       const int s = sel[i];
@@ -206,16 +239,28 @@ route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
   }
 }
 
+// CTAs per cluster for the chunk scan: enough CTAs to cover the SMs a few
+// times, at most 8 (the portable cluster size), slices of at least 32 rows.
+int chunk_cluster_size(const LayerParams& p) {
+  const int64_t items = static_cast<int64_t>(p.B) * p.Hkv * p.nblk;
+  int cl = 1;
+  while (cl < 8 && items * cl * 2 <= 148 * 8 && p.n_chunks / (cl * 2) >= 32) cl *= 2;
+  return cl;
+}
+
 template <typename T, int D>
 cudaError_t launch_route_chunks_t(const LayerParams& p, const void* q, const int64_t* pos,
                                   const float* chunk_sum, int32_t* chunk_idx, float* chunk_score,
                                   unsigned* err, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(p.n_chunks) * sizeof(float) + p.kc * sizeof(int);
+  const int cl = chunk_cluster_size(p);
+  const int per = ((p.n_chunks + cl - 1) / cl + 3) & ~3;
+  const size_t smem = static_cast<size_t>(per + (cl > 1 ? p.n_chunks : 0)) * sizeof(float) +
+                      p.kc * sizeof(int);
   cudaError_t e = ensure_smem<route_chunks_kernel<T, D>>(smem);
   if (e != cudaSuccess) return e;
-  route_chunks_kernel<T, D><<<p.B * p.Hkv * p.nblk, kThreads, smem, s>>>(static_cast<const T*>(q), pos, chunk_sum, p,
-                                                    chunk_idx, chunk_score, err);
-  return cudaGetLastError();
+  return launch_pdl(route_chunks_kernel<T, D>, dim3(p.B * p.Hkv * p.nblk * cl), dim3(kThreads),
+                    smem, s, cl, static_cast<const T*>(q), pos, chunk_sum, p, chunk_idx,
+                    chunk_score, err);
 }
 
 template <typename T, int D>
@@ -227,9 +272,9 @@ cudaError_t launch_route_groups_t(const LayerParams& p, const void* q, const int
                       static_cast<size_t>(p.kg + p.kc) * sizeof(int);
   cudaError_t e = ensure_smem<route_groups_kernel<T, D>>(smem);
   if (e != cudaSuccess) return e;
-  route_groups_kernel<T, D><<<p.B * p.Hkv * p.nblk, kThreads, smem, s>>>(static_cast<const T*>(q), pos, group_sum,
-                                                    chunk_idx, p, group_idx, group_score, err);
-  return cudaGetLastError();
+  return launch_pdl(route_groups_kernel<T, D>, dim3(p.B * p.Hkv * p.nblk), dim3(kThreads), smem,
+                    s, 1, static_cast<const T*>(q), pos, group_sum, chunk_idx, p, group_idx,
+                    group_score, err);
 }
 
 }  // namespace

@@ -52,7 +52,11 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   constexpr int PPL = P / 32;
   extern __shared__ float2 smem_tab[];
   __shared__ float s_gsum[8][D];             // raw group sums of one chunk
+  __shared__ double s_omega[P];
   const int n_lo = P - p.n_high;
+  for (int i = threadIdx.x; i < n_lo; i += blockDim.x)
+    s_omega[i] = pow(p.theta, -2.0 * (p.n_high + i) / D);
+  __syncthreads();
   float2* tab_g = smem_tab;                  // [g][n_lo]: rotation by (g-1)/2 - o
   float2* tab_s = smem_tab + kGroup * n_lo;  // [Ng][n_lo]: rotation by (C-g)/2 - w*g
   // Angles are formed in double from omega_i = theta^(-2i/D) and the exact
@@ -61,14 +65,15 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
     const bool is_g = idx < kGroup * n_lo;
     const int j = is_g ? idx : idx - kGroup * n_lo;
     const int o = j / n_lo;
-    const int i = p.n_high + j % n_lo;
-    const double omega = pow(p.theta, -2.0 * i / D);
+    const double omega = s_omega[j % n_lo];
     const double off = is_g ? 0.5 * (kGroup - 1) - o : 0.5 * (p.C - kGroup) - o * kGroup;
     float s, c;
     sincosf(static_cast<float>(off * omega), &s, &c);
     smem_tab[idx] = make_float2(c, s);
   }
   __syncthreads();
+  pdl_wait();
+  pdl_trigger();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
@@ -164,9 +169,9 @@ cudaError_t launch_summaries_t(const LayerParams& p, const void* k, int64_t t_be
   dim3 grid(gx, bh);
   const int n_lo = D / 2 - p.n_high;
   const size_t smem = static_cast<size_t>(kGroup + p.Ng) * n_lo * sizeof(float2);
-  summaries_kernel<T, D><<<grid, 32 * p.Ng, smem, stream>>>(
-      static_cast<const T*>(k), p, t_begin, t_end, c_first, c_count, chunk_sum, group_sum);
-  return cudaGetLastError();
+  return launch_pdl(summaries_kernel<T, D>, grid, dim3(32 * p.Ng), smem, stream, 1,
+                    static_cast<const T*>(k), p, t_begin, t_end, c_first, c_count, chunk_sum,
+                    group_sum);
 }
 
 }  // namespace

@@ -57,6 +57,83 @@ __device__ __forceinline__ int block_exclusive_scan(int v, TopkSmem& sm, int* to
   return res;
 }
 
+// Warp-cooperative compaction of an id list: keeps, in order, every id with
+// in_range(id) true that exceeds every id kept before it (so the output is
+// strictly ascending and free of duplicates).  Called by all 32 lanes of one
+// warp; writes out[0..count) and returns count in every lane; *bad is set when
+// a non-negative id was dropped.
+template <typename InRange>
+__device__ int warp_keep_ascending(const int32_t* ids, int n, InRange in_range, int* out,
+                                   bool* bad) {
+  const int lane = threadIdx.x & 31;
+  int count = 0, run_max = -1;
+  bool dropped = false;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const int id = i < n ? ids[i] : -1;
+    const bool ok = id >= 0 && in_range(id);
+    int incl = ok ? id : -1;  // inclusive prefix max over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl = max(incl, x);
+    }
+    int excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    excl = max(lane == 0 ? -1 : excl, run_max);
+    const bool keep = ok && id > excl;
+    dropped |= __any_sync(0xffffffffu, id >= 0 && !keep);
+    const unsigned km = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[count + __popc(km & ((1u << lane) - 1u))] = id;
+    count += __popc(km);
+    run_max = max(run_max, __shfl_sync(0xffffffffu, incl, 31));
+  }
+  *bad = dropped;
+  return count;
+}
+
+// Top-k by rank counting, for small n (each thread compares its candidates
+// against all n): candidate i is taken when fewer than k candidates beat it,
+// where j beats i if s_j > s_i, or s_j == s_i and j < i.  Same result and
+// contract as block_topk.
+template <int NT>
+__device__ int block_topk_rank(const float* sc, int n, int k, int* sel, TopkSmem& sm) {
+  const int tid = threadIdx.x;
+  if (n <= k) {
+    for (int i = tid; i < n; i += NT) sel[i] = i;
+    __syncthreads();
+    return n;
+  }
+  const int ipt = (n + NT - 1) / NT;
+  const int beg = min(n, tid * ipt), end = min(n, beg + ipt);
+  unsigned take_bits = 0u;  // ipt <= 32 (n <= 32 * NT)
+  int n_take = 0;
+  for (int i = beg; i < end; ++i) {
+    const float si = sc[i];
+    int beats = 0;
+    int j = 0;
+    for (; j + 4 <= n; j += 4) {  // sc is 16-byte aligned shared memory
+      const float4 v = *reinterpret_cast<const float4*>(sc + j);
+      beats += (v.x > si) || (v.x == si && j < i);
+      beats += (v.y > si) || (v.y == si && j + 1 < i);
+      beats += (v.z > si) || (v.z == si && j + 2 < i);
+      beats += (v.w > si) || (v.w == si && j + 3 < i);
+    }
+    for (; j < n; ++j) {
+      const float sj = sc[j];
+      beats += (sj > si) || (sj == si && j < i);
+    }
+    if (beats < k) {
+      take_bits |= 1u << (i - beg);
+      ++n_take;
+    }
+  }
+  int w = block_exclusive_scan<NT>(n_take, sm);
+  for (int i = beg; i < end; ++i)
+    if (take_bits >> (i - beg) & 1u) sel[w++] = i;
+  __syncthreads();
+  return k;
+}
+
 // Indices of the top k of sc[0..n) (ties to the lower index), ascending, into
 // sel[0..min(n,k)).  Returns min(n, k).  Every thread of the block must call it;
 // sc and sel are shared memory; sel is complete on return.

@@ -200,3 +200,15 @@ def test_cache_past_the_query_is_never_read_into_the_output(dtype):
     for b in range(2):
         for h in range(2):
             compare_head(wl, x, res, b, h)
+
+
+@pytest.mark.parametrize("context,batch", [(6400, 1), (100 * 64 * 5, 1), (3200, 3)])
+def test_router_with_odd_chunk_counts(context, batch):
+    """Chunk counts that split unevenly over a CTA cluster; small and large candidate sets."""
+    wl = S.workload("llama3_8b_decode_32k", batch=batch, context=context, heads_q=8, heads_kv=2,
+                    needles=0)
+    x = S.make_inputs(wl, 21)
+    res = run_gpu(wl, x)
+    for b in range(batch):
+        for h in range(2):
+            compare_head(wl, x, res, b, h)

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_SHAPE", 3: "H
 # Exported symbols of the C ABI, in header order.
 SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device_status",
            "hga_workspace_size", "hga_build_summaries", "hga_route_chunks", "hga_route_groups",
-           "hga_attend")
+           "hga_attend", "hga_attend_noalloc")
 
 
 class HGAConfig(ctypes.Structure):
@@ -70,6 +70,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_route_chunks": (ctypes.c_int, [C, P, I32, P, P, I64, P, P, P]),
         "hga_route_groups": (ctypes.c_int, [C, P, I32, P, P, I64, P, P, P, P]),
         "hga_attend": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, SZ, P]),
+        "hga_attend_noalloc": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -180,3 +181,21 @@ def hga_attend(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=
                                      _ptr(v), n_alloc, _ptr(group_idx), _ptr(out), _ptr(lse),
                                      _ptr(workspace), workspace_bytes, _stream(stream)),
            "hga_attend")
+
+
+def hga_attend_noalloc(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=None,
+                       stream=None) -> None:
+    """hga_attend without a caller workspace, for callers that cannot allocate.
+
+    Frameworks that own all device memory and hand a plugin only its inputs and
+    outputs, or loops where cudaMalloc/cudaFree (which may synchronise the
+    device) is not allowed, can use this call: the split-K scratch lives in a
+    fixed 8 MiB array inside the library.  Larger shapes raise HGAError
+    (HGA_ERR_WORKSPACE).  The first call on a device looks up the array's
+    address, so make it before any stream capture; calls that overlap on the
+    GPU share the array and race.
+    """
+    _check(load_library().hga_attend_noalloc(ctypes.byref(_cfg(cfg)), _ptr(q), q_len, _ptr(pos),
+                                             _ptr(k), _ptr(v), n_alloc, _ptr(group_idx),
+                                             _ptr(out), _ptr(lse), _stream(stream)),
+           "hga_attend_noalloc")

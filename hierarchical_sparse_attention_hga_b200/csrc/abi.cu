@@ -92,6 +92,11 @@ hga_status make_params(const hga_config* cfg, int64_t n_alloc, int32_t q_len, La
 }
 
 }  // namespace
+
+// Sets the message hga_last_error() returns on this thread (for entry points
+// defined in other files of the library).
+void set_last_error(const char* msg) { snprintf(g_msg, sizeof(g_msg), "%s", msg); }
+
 }  // namespace hga
 
 using namespace hga;

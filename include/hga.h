@@ -215,6 +215,33 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
                       void* out, float* lse, void* workspace, size_t workspace_bytes,
                       void* stream);
 
+/*
+ * hga_attend for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is a deployment convenience of this library.
+ *
+ * Some callers cannot provide the workspace hga_attend needs: frameworks that
+ * own all device memory through their own pool and give an attention plugin
+ * only its input and output buffers, and latency-critical loops where a
+ * cudaMalloc / cudaFree (which may synchronise the device) is not allowed.
+ * This call computes exactly what hga_attend computes, with the same
+ * arguments minus the workspace: its split-K scratch lives in one fixed 8 MiB
+ * array inside the library (present on every GPU that loads the library, until
+ * the process exits).  It calls no allocator.
+ *
+ *  - Shapes whose hga_workspace_size() exceeds 8 MiB are rejected with
+ *    HGA_ERR_WORKSPACE (use hga_attend with a caller workspace instead).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the array, which keeps the last call's
+ *    contents (nothing in it has to start at zero).  Calls whose kernels
+ *    overlap on the GPU (other streams, other host threads) race on it and
+ *    produce wrong results: serialise them.
+ */
+hga_status hga_attend_noalloc(const hga_config* cfg, const void* q, int32_t q_len,
+                              const int64_t* pos, const void* k, const void* v, int64_t n_alloc,
+                              const int32_t* group_idx, void* out, float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

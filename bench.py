@@ -197,25 +197,31 @@ def run_hga(args, rank: int, world: int):
 
     parts = {
         "summaries": lambda st: B.hga_build_summaries(layer, k, n, p, p + 1, cs, gs, stream=st),
-        "route_chunks": lambda st: B.hga_route_chunks(layer, q, 1, pos, cs, n, ci, stream=st),
-        "route_groups": lambda st: B.hga_route_groups(layer, q, 1, pos, gs, n, ci, gi, stream=st),
+        "route": lambda st: B.hga_route(layer, q, 1, pos, cs, gs, n, ci, gi, stream=st),
         "attend": lambda st: B.hga_attend(layer, q, 1, pos, k, v, n, gi, out, lse, ws, wsb,
                                           stream=st),
+        "route_chunks": lambda st: B.hga_route_chunks(layer, q, 1, pos, cs, n, ci, stream=st),
+        "route_groups": lambda st: B.hga_route_groups(layer, q, 1, pos, gs, n, ci, gi, stream=st),
     }
 
     side = torch.cuda.Stream()
 
-    def step(st):
-        # The rows the new token closes belong to the current chunk, which this
-        # step never routes (it is always visible), so the append runs on a
-        # side stream, concurrently with routing and attention.
-        main = torch.cuda.current_stream()
-        side.wait_stream(main)
-        with torch.cuda.stream(side):
-            parts["summaries"](side.cuda_stream)
-        for name in ("route_chunks", "route_groups", "attend"):
-            parts[name](st)
-        main.wait_stream(side)
+    def make_step(chain):
+        def step(st):
+            # The rows the new token closes belong to the current chunk, which
+            # this step never routes (it is always visible), so the append runs
+            # on a side stream, concurrently with routing and attention.
+            main = torch.cuda.current_stream()
+            side.wait_stream(main)
+            with torch.cuda.stream(side):
+                parts["summaries"](side.cuda_stream)
+            for name in chain:
+                parts[name](st)
+            main.wait_stream(side)
+        return step
+
+    step = make_step(("route", "attend"))
+    step4 = make_step(("route_chunks", "route_groups", "attend"))
 
     # eager warm-up, then one CUDA graph for the whole step and one per call
     for _ in range(max(1, args.warmup)):
@@ -223,7 +229,7 @@ def run_hga(args, rank: int, world: int):
     torch.cuda.synchronize()
     assert B.hga_device_status(sh) == 0
     graphs = {}
-    for name, fn in list(parts.items()) + [("step", step)]:
+    for name, fn in list(parts.items()) + [("step", step), ("step4", step4)]:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             fn(torch.cuda.current_stream().cuda_stream)
@@ -255,6 +261,9 @@ def run_hga(args, rank: int, world: int):
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     ms_step = sum(step_ms) / len(step_ms)
+    a4, b4 = timed(graphs["step4"], min(args.steps, 200))
+    torch.cuda.synchronize()
+    ms_step4 = sum(x.elapsed_time(y) for x, y in zip(a4, b4)) / len(a4)
     if dist:
         t = torch.tensor([ms_step], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -306,12 +315,13 @@ def run_hga(args, rank: int, world: int):
     d2h = out_host.numel() * out_host.element_size()
 
     nb = step_bytes(wl)
-    kern = max(("route_chunks", "route_groups", "attend", "summaries"), key=lambda kk: ms[kk])
+    nb["route"] = nb["route_chunks"] + nb["route_groups"]
+    kern = max(("route", "attend"), key=lambda kk: ms[kk])
     hbm, peak_kind = peaks()
     achieved = nb[kern] / (ms[kern] * 1e-3) / 1e9
-    total_bytes = nb["summaries"] + nb["route_chunks"] + nb["route_groups"] + nb["attend"]
+    total_bytes = nb["summaries"] + nb["route"] + nb["attend"]
     nsplit_combine = 1 if wsb > 0 else 0
-    launches_per_step = 1 + 1 + 1 + 1 + nsplit_combine
+    launches_per_step = 1 + 1 + 1 + nsplit_combine   # summaries, route, attend (+ merge)
     tokens = wl.batch * world
     line = {
         "metric": METRIC,
@@ -332,7 +342,8 @@ def run_hga(args, rank: int, world: int):
                    "tokens_attended_per_kv_head": nb["tokens"],
                    "l2": "flushed (256 MB write) before every timed step",
                    "parallelism": f"replicas x{world} (independent sequences per GPU)"},
-        "per_kernel_us": {kk: ms[kk] * 1e3 for kk in ("summaries", "route_chunks", "route_groups", "attend")},
+        "per_kernel_us": {kk: ms[kk] * 1e3 for kk in parts},
+        "four_call_step_us": ms_step4 * 1e3,
         "timing_floor_us": floor_us,
         "step_hbm_bytes": total_bytes,
         "step_hbm_gbs": total_bytes / (ms_step * 1e-3) / 1e9,

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_SHAPE", 3: "H
 # Exported symbols of the C ABI, in header order.
 SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device_status",
            "hga_workspace_size", "hga_build_summaries", "hga_route_chunks", "hga_route_groups",
-           "hga_attend", "hga_attend_noalloc")
+           "hga_route", "hga_attend", "hga_attend_noalloc")
 
 
 class HGAConfig(ctypes.Structure):
@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_build_summaries": (ctypes.c_int, [C, P, I64, I64, I64, P, P, P]),
         "hga_route_chunks": (ctypes.c_int, [C, P, I32, P, P, I64, P, P, P]),
         "hga_route_groups": (ctypes.c_int, [C, P, I32, P, P, I64, P, P, P, P]),
+        "hga_route": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, P]),
         "hga_attend": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, SZ, P]),
         "hga_attend_noalloc": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P]),
     }
@@ -173,6 +174,15 @@ def hga_route_groups(cfg, q, q_len: int, pos, group_sum, n_alloc: int, chunk_idx
                                            _ptr(group_sum), n_alloc, _ptr(chunk_idx),
                                            _ptr(group_idx), _ptr(group_score), _stream(stream)),
            "hga_route_groups")
+
+
+def hga_route(cfg, q, q_len: int, pos, chunk_sum, group_sum, n_alloc: int, chunk_idx, group_idx,
+              chunk_score=None, group_score=None, stream=None) -> None:
+    """Both routing levels in one launch (same results as the two separate calls)."""
+    _check(load_library().hga_route(ctypes.byref(_cfg(cfg)), _ptr(q), q_len, _ptr(pos),
+                                    _ptr(chunk_sum), _ptr(group_sum), n_alloc, _ptr(chunk_idx),
+                                    _ptr(chunk_score), _ptr(group_idx), _ptr(group_score),
+                                    _stream(stream)), "hga_route")
 
 
 def hga_attend(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=None,

@@ -188,6 +188,22 @@ hga_status hga_route_groups(const hga_config* cfg, const void* q, int32_t q_len,
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route_groups");
 }
 
+hga_status hga_route(const hga_config* cfg, const void* q, int32_t q_len, const int64_t* pos,
+                     const float* chunk_sum, const float* group_sum, int64_t n_alloc,
+                     int32_t* chunk_idx, float* chunk_score, int32_t* group_idx,
+                     float* group_score, void* stream) {
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, q_len, &p);
+  if (st != HGA_OK) return st;
+  if (!q || !pos || !chunk_sum || !group_sum || !chunk_idx || !group_idx)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_route(p, cfg->dtype, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score,
+                               group_idx, group_score, err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route");
+}
+
 hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const int64_t* pos,
                       const void* k, const void* v, int64_t n_alloc, const int32_t* group_idx,
                       void* out, float* lse, void* workspace, size_t workspace_bytes,

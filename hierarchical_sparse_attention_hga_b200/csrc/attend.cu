@@ -94,7 +94,6 @@ attend_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos, const T*
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int d = tid % D;
   pdl_wait();
-  pdl_trigger();
 
   const int64_t pb = pos[b];
   const bool ok = valid_position(pb, p, tid == 0 && split == 0 ? err : nullptr);
@@ -224,6 +223,7 @@ attend_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos, const T*
       if (d == 0) { ws_ml[slot * 2] = m; ws_ml[slot * 2 + 1] = l; }
     }
   }
+  pdl_trigger();
 }
 
 // Log-sum-exp merge of the split partials of one decode query head.
@@ -237,7 +237,6 @@ combine_kernel(LayerParams p, int nsplit, const float* __restrict__ ws_o,
   const int bh = b * p.Hkv + h;
   const int d = threadIdx.x;
   pdl_wait();
-  pdl_trigger();
   float m = -CUDART_INF_F;
   for (int s = 0; s < nsplit; ++s) m = fmaxf(m, ws_ml[((static_cast<size_t>(bh) * nsplit + s) * p.G + hh) * 2]);
   float l = 0.f, o = 0.f;
@@ -254,6 +253,7 @@ combine_kernel(LayerParams p, int nsplit, const float* __restrict__ ws_o,
   const size_t row = static_cast<size_t>(b) * p.Hq + hq;  // q_len == 1
   store_out(out + row * D + d, l > 0.f ? o / l : 0.f);
   if (lse && d == 0) lse[row] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+  pdl_trigger();
 }
 
 }  // namespace
@@ -313,8 +313,7 @@ static bool use_decode_fast(const LayerParams& p, int dtype) {
 }
 
 size_t attend_workspace_bytes(const LayerParams& p, int dtype) {
-  if (use_decode_fast(p, dtype))
-    return static_cast<size_t>(p.B) * p.Hkv * decode_fast_nsplit(p) * p.G * (p.D + 2) * sizeof(float);
+  if (use_decode_fast(p, dtype)) return 0;  // partials merge inside a thread-block cluster
   int nsplit = 1;
   choose_split_tokens(p, &nsplit);
   if (nsplit == 1) return 0;
@@ -327,7 +326,7 @@ cudaError_t launch_attend(const LayerParams& p, int dtype, int out_dtype, const 
                           unsigned* err, cudaStream_t s) {
   using bf = __nv_bfloat16;
   if (use_decode_fast(p, dtype))
-    return launch_attend_decode_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, ws, err, s);
+    return launch_attend_decode_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, err, s);
   if (dtype == 0)
     return out_dtype == 0 ? launch_attend_d<float, float>(p, q, pos, k, v, group_idx, out, lse, ws, err, s)
                           : launch_attend_d<float, bf>(p, q, pos, k, v, group_idx, out, lse, ws, err, s);

@@ -18,14 +18,21 @@
 //     ldmatrix from the swizzled tile;
 //   - online softmax in registers (log2 domain); P stays in registers and is
 //     reused as the A operand of O += P V (V fragments via ldmatrix.trans).
-// The warp writes its partial (o, m, l); the log-sum-exp merge kernel of
-// attend.cu combines the splits.  No cluster multicast is used anywhere.
+// The CTAs of one (sequence, KV head) form a thread-block cluster.  Each warp's
+// partial (o, m, l) is merged by log-sum-exp first inside its CTA (shared
+// memory), then across the cluster by CTA rank 0 reading the other CTAs'
+// partials through distributed shared memory: no workspace, no second kernel.
+// No cluster multicast is used anywhere.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace hga {
 
@@ -42,16 +49,18 @@ constexpr int kWarpBytes = kStages * kStageBytes;
 constexpr int kSmemBytes = kWarps * kWarpBytes + 1024;  // + alignment slack
 constexpr uint32_t kWaitLimit = 1u << 26;       // bounded mbarrier polls
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
+template <typename TO>
 struct DecodeArgs {
   const __nv_bfloat16* q;
   const int64_t* pos;
   const int32_t* group_idx;
-  float* ws_o;
-  float* ws_ml;
+  TO* out;
+  float* lse;
   unsigned* err;
   int units_per_split;
-  int nsplit;
+  int nsplit;   // warp-splits per (sequence, KV head) = kWarps * cluster size
 };
 
 // Address of the 16-byte chunk `chunk` (0..15 over 128 dims) of row `row` in a
@@ -61,18 +70,25 @@ __device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int chunk) {
   return tile + box * kBoxBytes + row * 128 + ((c ^ (row & 7)) << 4);
 }
 
+template <typename TO>
 __global__ void __launch_bounds__(kWarps * 32)
 attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, DecodeArgs a, LayerParams p) {
+                          const __grid_constant__ CUtensorMap tm_v, DecodeArgs<TO> a,
+                          LayerParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bars[kWarps][kStages];
   __shared__ int s_gl[1024];
   __shared__ int s_ng;
+  __shared__ float s_ml[kWarps][16][2];   // per-warp (m, l) of each query head
+  __shared__ float s_rml[8][16][2];       // rank 0: (m, l) pushed by each CTA of the cluster
 
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());  // grid.x == cluster size
+  const int n_cta = static_cast<int>(cluster.num_blocks());
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int b = bh / p.Hkv, h = bh % p.Hkv;
-  const int split = blockIdx.x * kWarps + warp;
+  const int split = rank * kWarps + warp;
 
   if (threadIdx.x == 0) {
     ptx::prefetch_tensormap(&tm_k);
@@ -86,7 +102,7 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   // Everything up to pdl_wait() reads only pos, k and v (never written by this
   // library), so it overlaps the routing kernel still running ahead of us.
   const int64_t pb = a.pos[b];
-  const bool ok = valid_position(pb, p, threadIdx.x == 0 && blockIdx.x == 0 ? a.err : nullptr);
+  const bool ok = valid_position(pb, p, threadIdx.x == 0 && rank == 0 ? a.err : nullptr);
   const int cur = ok ? static_cast<int>(pb / p.C) : 0;
   const int b0 = max(0, cur - p.local);
   // Unit list: sink units [0, su), local+current units [su, su+lu), routed groups.
@@ -124,9 +140,8 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
   };
   // Forced units (sink, local, current) do not depend on routing: start them now.
-  const bool live = split < a.nsplit;
-  const int pre0 = live && u_lo < n_forced ? 1 : 0;
-  const int pre1 = live && u_lo + 1 < n_forced && u_lo + 1 < u_cap ? 1 : 0;
+  const int pre0 = u_lo < n_forced ? 1 : 0;
+  const int pre1 = u_lo + 1 < n_forced && u_lo + 1 < u_cap ? 1 : 0;
   if (pre0) issue(u_lo, 0);
   if (pre1) issue(u_lo + 1, 1);
 
@@ -150,7 +165,6 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
 
   pdl_wait();
-  pdl_trigger();
 
   // Routed groups kept, in order: warp 0 validates and compacts them.  An id
   // is kept when it names a group of a candidate chunk and exceeds every id
@@ -184,26 +198,17 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     if (lane == 0) {
       s_ng = n;
-      if (bad && blockIdx.x == 0) flag_error(a.err, kErrGroupIdx);
+      if (bad && rank == 0) flag_error(a.err, kErrGroupIdx);
     }
   }
   __syncthreads();
 
   const int n_units = n_forced + s_ng;
   const int u_hi = min(n_units, u_cap);
-  const size_t slot = static_cast<size_t>(bh) * a.nsplit + split;
-
-  if (!live) return;
-  if (u_lo >= u_hi) {
-    if (lane < p.G) {
-      a.ws_ml[(slot * p.G + lane) * 2] = -CUDART_INF_F;
-      a.ws_ml[(slot * p.G + lane) * 2 + 1] = 0.f;
-    }
-    return;
+  if (u_lo < u_hi) {
+    if (!pre0) issue(u_lo, 0);
+    if (!pre1 && u_lo + 1 < u_hi) issue(u_lo + 1, 1);
   }
-  if (!pre0) issue(u_lo, 0);
-  if (!pre1 && u_lo + 1 < u_hi) issue(u_lo + 1, 1);
-
 
   float o[16][4];
 #pragma unroll
@@ -214,11 +219,16 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   // ldmatrix lane roles
   const int mi = lane >> 3, ri = lane & 7;
   bool timed_out = false;
+  int stuck_it = 0;
 
   for (int u = u_lo; u < u_hi; ++u) {
     const int it = u - u_lo;
     const int stage = it & 1;
-    if (!ptx::mbar_wait(&wbar[stage], (it >> 1) & 1, kWaitLimit)) { timed_out = true; break; }
+    if (!ptx::mbar_wait(&wbar[stage], (it >> 1) & 1, kWaitLimit)) {
+      timed_out = true;
+      stuck_it = it;
+      break;
+    }
     const uint32_t kt = wsm_u32 + stage * kStageBytes;
     const uint32_t vt = kt + kTileBytes;
     const int valid = unit_valid(u);
@@ -296,33 +306,104 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
 
   if (timed_out) {
+    // The warp gave up waiting on its copies: its partial is dropped (the
+    // output is wrong and flagged), it waits once more, again bounded, for the
+    // copies it still has in flight, and it still joins the merge barriers.
     if (lane == 0) flag_error(a.err, kErrTimeout);
-    return;
+    for (int it = stuck_it; it < stuck_it + 2 && u_lo + it < u_hi; ++it)
+      ptx::mbar_wait(&wbar[it & 1], (it >> 1) & 1, kWaitLimit);
+    m0 = m1 = -CUDART_INF_F;
+    l0 = l1 = 0.f;
   }
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  if (g < p.G) {
-    float* dst = a.ws_o + (slot * p.G + g) * kD;
+
+  // ---- merge 1: the CTA's warps, through shared memory.  Every issued TMA
+  // copy has been waited for, so a warp's own ring now holds its partial o.
+  float* wo = reinterpret_cast<float*>(wsm);  // [16 heads][128] floats
+  if (u_lo >= u_hi) {
+    m0 = m1 = -CUDART_INF_F;
+    l0 = l1 = 0.f;
+  } else {
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      *reinterpret_cast<float2*>(dst + j * 8 + 2 * t) = make_float2(o[j][0], o[j][1]);
-    if (t == 0) {
-      a.ws_ml[(slot * p.G + g) * 2] = m0;
-      a.ws_ml[(slot * p.G + g) * 2 + 1] = l0;
+    for (int j = 0; j < 16; ++j) {
+      *reinterpret_cast<float2*>(wo + g * kD + j * 8 + 2 * t) = make_float2(o[j][0], o[j][1]);
+      *reinterpret_cast<float2*>(wo + (g + 8) * kD + j * 8 + 2 * t) = make_float2(o[j][2], o[j][3]);
     }
   }
-  if (g + 8 < p.G) {
-    float* dst = a.ws_o + (slot * p.G + g + 8) * kD;
+  if (t == 0) {
+    s_ml[warp][g][0] = m0;
+    s_ml[warp][g][1] = l0;
+    s_ml[warp][g + 8][0] = m1;
+    s_ml[warp][g + 8][1] = l1;
+  }
+  __syncthreads();
+  const int d = threadIdx.x;  // one output dim per thread (blockDim == D == 128)
+  uint8_t* ring0 = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
+  float cta_m[16], cta_l[16], cta_o[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      *reinterpret_cast<float2*>(dst + j * 8 + 2 * t) = make_float2(o[j][2], o[j][3]);
-    if (t == 0) {
-      a.ws_ml[(slot * p.G + g + 8) * 2] = m1;
-      a.ws_ml[(slot * p.G + g + 8) * 2 + 1] = l1;
+  for (int hh = 0; hh < 16; ++hh) {
+    cta_m[hh] = -CUDART_INF_F;
+    cta_l[hh] = 0.f;
+    cta_o[hh] = 0.f;
+    if (hh >= p.G) continue;
+    float mm = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, s_ml[w][hh][0]);
+    if (mm == -CUDART_INF_F) continue;
+    float ll = 0.f, oo = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = s_ml[w][hh][0];
+      if (mw == -CUDART_INF_F) continue;
+      const float f = exp2f(mw - mm);
+      ll += s_ml[w][hh][1] * f;
+      oo += reinterpret_cast<const float*>(ring0 + w * kWarpBytes)[hh * kD + d] * f;
+    }
+    cta_m[hh] = mm;
+    cta_l[hh] = ll;
+    cta_o[hh] = oo;
+  }
+  // ---- merge 2: the cluster's CTAs.  After the first barrier every CTA has
+  // finished reading its own ring, so rank 0's ring is free; every CTA then
+  // pushes its partial into rank 0's ring (remote shared-memory stores), and
+  // after the second barrier rank 0 merges from its own shared memory.
+  cluster.sync();
+  float* recv = cluster.map_shared_rank(reinterpret_cast<float*>(ring0), 0);  // [8][16][128]
+  float (*recv_ml)[16][2] = cluster.map_shared_rank(s_rml, 0);
+#pragma unroll
+  for (int hh = 0; hh < 16; ++hh) {
+    if (hh >= p.G) continue;
+    recv[(rank * 16 + hh) * kD + d] = cta_o[hh];
+    if (d == 0) {
+      recv_ml[rank][hh][0] = cta_m[hh];
+      recv_ml[rank][hh][1] = cta_l[hh];
     }
   }
+  cluster.sync();
+  if (rank == 0) {
+    const float* mine = reinterpret_cast<const float*>(ring0);
+    for (int hh = 0; hh < p.G; ++hh) {
+      float mm = -CUDART_INF_F;
+      for (int r = 0; r < n_cta; ++r) mm = fmaxf(mm, s_rml[r][hh][0]);
+      float ll = 0.f, oo = 0.f;
+      if (mm != -CUDART_INF_F) {
+        for (int r = 0; r < n_cta; ++r) {
+          const float mr = s_rml[r][hh][0];
+          if (mr == -CUDART_INF_F) continue;
+          const float f = exp2f(mr - mm);
+          ll += s_rml[r][hh][1] * f;
+          oo += mine[(r * 16 + hh) * kD + d] * f;
+        }
+      }
+      const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + hh;
+      store_out(a.out + row * kD + d, ll > 0.f ? oo / ll : 0.f);
+      if (a.lse && d == 0) a.lse[row] = ll > 0.f ? (mm + log2f(ll)) * kLn2 : -CUDART_INF_F;
+    }
+  }
+  pdl_trigger();
 }
 
 // ------------------------------------------------------------------ host side
@@ -360,51 +441,62 @@ int max_units(const LayerParams& p) {
   return (p.sink + p.local + 1) * (p.C / kUnit) + p.kg;
 }
 
-int choose_units_per_split(const LayerParams& p) {
-  const int64_t total = static_cast<int64_t>(p.B) * p.Hkv * max_units(p);
-  const int64_t warps = 148 * 12;  // ~3 CTAs of 4 warps per SM
-  int64_t u = (total + warps - 1) / warps;
-  return static_cast<int>(u < 1 ? 1 : (u > 16 ? 16 : u));
+// CTAs per (sequence, KV head), at most 8 (the portable cluster size): enough
+// warps for ~12 per SM over the whole batch, but never more CTAs than fit at
+// once (3 per SM, bounded by registers and shared memory), so the grid runs
+// in a single wave.
+int cluster_size(const LayerParams& p) {
+  const int64_t bh = static_cast<int64_t>(p.B) * p.Hkv;
+  const int64_t want = (148 * 12 + bh * kWarps - 1) / (bh * kWarps);
+  const int64_t fit = (148 * 3) / bh;
+  const int64_t useful = (max_units(p) + kWarps - 1) / kWarps;
+  int64_t cl = want < fit ? want : fit;
+  cl = cl < useful ? cl : useful;
+  return static_cast<int>(cl < 1 ? 1 : (cl > 8 ? 8 : cl));
+}
+
+template <typename TO>
+cudaError_t launch_t(const LayerParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const void* q, const int64_t* pos, const int32_t* group_idx, void* out,
+                     float* lse, unsigned* err, cudaStream_t s) {
+  const int cl = cluster_size(p);
+  DecodeArgs<TO> a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.pos = pos;
+  a.group_idx = group_idx;
+  a.out = static_cast<TO*>(out);
+  a.lse = lse;
+  a.err = err;
+  a.nsplit = cl * kWarps;
+  a.units_per_split = (max_units(p) + a.nsplit - 1) / a.nsplit;
+  cudaError_t e = ensure_smem<attend_decode_bf16_kernel<TO>>(kSmemBytes);
+  if (e != cudaSuccess) return e;
+  // A plain (non-programmatic) launch: measured faster here, because CTAs of
+  // this kernel launched early would hold SM slots while the routing kernel
+  // before it finishes.  pdl_wait() inside is then a no-op.
+  return launch_pdl(attend_decode_bf16_kernel<TO>, dim3(cl, p.B * p.Hkv), dim3(kWarps * 32),
+                    kSmemBytes, s, cl | kNoPdl, tk, tv, a, p);
 }
 
 }  // namespace
 
 bool decode_fast_path(const LayerParams& p, int dtype) {
-  return dtype == 1 && p.D == kD && p.q_len == 1 && p.g == kUnit && p.kg <= 1024 && p.G <= 16;
-}
-
-int decode_fast_nsplit(const LayerParams& p) {
-  const int u = choose_units_per_split(p);
-  return (max_units(p) + u - 1) / u;
+  return dtype == 1 && p.D == kD && p.q_len == 1 && p.g == kUnit && p.kg <= 1024 && p.G <= 16 &&
+         p.B * p.Hkv <= 65535;
 }
 
 cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const void* q,
                                       const int64_t* pos, const void* k, const void* v,
-                                      const int32_t* group_idx, void* out, float* lse, void* ws,
+                                      const int32_t* group_idx, void* out, float* lse,
                                       unsigned* err, cudaStream_t s) {
   CUtensorMap tk, tv;
   const int64_t rows = static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc;
   cudaError_t e = make_map(&tk, k, rows);
   if (e == cudaSuccess) e = make_map(&tv, v, rows);
   if (e != cudaSuccess) return e;
-  const int ups = choose_units_per_split(p);
-  const int nsplit = decode_fast_nsplit(p);
-  DecodeArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.pos = pos;
-  a.group_idx = group_idx;
-  a.ws_o = static_cast<float*>(ws);
-  a.ws_ml = a.ws_o + static_cast<size_t>(p.B) * p.Hkv * nsplit * p.G * kD;
-  a.err = err;
-  a.units_per_split = ups;
-  a.nsplit = nsplit;
-  e = ensure_smem<attend_decode_bf16_kernel>(kSmemBytes);
-  if (e != cudaSuccess) return e;
-  dim3 grid((nsplit + kWarps - 1) / kWarps, p.B * p.Hkv);
-  e = launch_pdl(attend_decode_bf16_kernel, grid, dim3(kWarps * 32), kSmemBytes, s, 1, tk, tv, a,
-                 p);
-  if (e != cudaSuccess) return e;
-  return launch_combine(p, out_dtype, nsplit, a.ws_o, a.ws_ml, out, lse, s);
+  return out_dtype == 0
+             ? launch_t<float>(p, tk, tv, q, pos, group_idx, out, lse, err, s)
+             : launch_t<__nv_bfloat16>(p, tk, tv, q, pos, group_idx, out, lse, err, s);
 }
 
 }  // namespace hga

@@ -60,10 +60,12 @@ __device__ __forceinline__ void load2(const __nv_bfloat16* p, float (&o)[2]) {
 
 // Programmatic dependent launch.  Every kernel of the library launches with the
 // programmatic-serialization attribute, waits for its stream predecessor before
-// reading anything a predecessor may have written, and only then lets its own
-// dependents launch.  So the code a kernel runs before pdl_wait() overlaps the
-// tail of its predecessor and may read only data no kernel of this library
-// writes (q, pos, k, v).  Without the attribute both are no-ops.
+// reading anything a predecessor may have written, and lets its own dependents
+// launch only after that wait, near the end of its work (so that waiting
+// dependent CTAs do not take SM slots the kernel still needs).  The code a
+// kernel runs before pdl_wait() overlaps the tail of its predecessor and may
+// read only data no kernel of this library writes (q, pos, k, v).  Without
+// the attribute both are no-ops.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -12,11 +12,14 @@
 
 namespace hga {
 
-// Launches `kern` with programmatic stream serialization (see pdl_wait in
-// common.cuh) and, when cluster > 1, with that many CTAs per cluster along x.
+// Launches `kern`, with programmatic stream serialization (see pdl_wait in
+// common.cuh) unless kNoPdl is passed as `cluster` flag bit, and, when the
+// cluster size is > 1, with that many CTAs per cluster along x.
+constexpr int kNoPdl = 1 << 16;
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, int cluster, Args&&... args) {
+                       cudaStream_t stream, int cluster_and_flags, Args&&... args) {
+  const int cluster = cluster_and_flags & 0xffff;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -24,7 +27,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].val.programmaticStreamSerializationAllowed = (cluster_and_flags & kNoPdl) ? 0 : 1;
   int n = 1;
   if (cluster > 1) {
     attr[1].id = cudaLaunchAttributeClusterDimension;
@@ -72,15 +75,21 @@ cudaError_t launch_route_groups(const LayerParams& p, int dtype, const void* q, 
                                 int32_t* group_idx, float* group_score, unsigned* err,
                                 cudaStream_t s);
 
+// Both routing levels in one launch (same results as the two launches above).
+cudaError_t launch_route(const LayerParams& p, int dtype, const void* q, const int64_t* pos,
+                         const float* chunk_sum, const float* group_sum, int32_t* chunk_idx,
+                         float* chunk_score, int32_t* group_idx, float* group_score,
+                         unsigned* err, cudaStream_t s);
+
 // Workspace bytes of launch_attend for p (0 when the launch needs none).
 size_t attend_workspace_bytes(const LayerParams& p, int dtype);
 
-// The bf16, D = 128 decode kernel (TMA + mma.sync) applies to p.
+// The bf16, D = 128 decode kernel (TMA + mma.sync, in-cluster merge, no
+// workspace) applies to p.
 bool decode_fast_path(const LayerParams& p, int dtype);
-int decode_fast_nsplit(const LayerParams& p);
 cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const void* q,
                                       const int64_t* pos, const void* k, const void* v,
-                                      const int32_t* group_idx, void* out, float* lse, void* ws,
+                                      const int32_t* group_idx, void* out, float* lse,
                                       unsigned* err, cudaStream_t s);
 
 // Log-sum-exp merge of nsplit decode partials into out / lse.

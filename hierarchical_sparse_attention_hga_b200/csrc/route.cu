@@ -101,21 +101,52 @@ __device__ __forceinline__ void block_rows(const LayerParams& p, int64_t pos, in
   *cur = static_cast<int>((first + *r0 + *nr - 1) / p.C);
 }
 
+// Dynamic shared memory of route_chunks_kernel, in 4-byte words (every part a
+// multiple of 4 words, so each part stays 16-byte aligned):
+//   local [per] | lsel [lsel_n] | pushed scores, pushed ids, merged scores,
+//   merged ids [4 x 8 x kc4] | sel [kc4]
+struct RouteSmem {
+  int per, lsel_n, kc4;
+  __host__ __device__ size_t words() const { return per + lsel_n + 4 * 8 * kc4 + kc4; }
+};
+__host__ __device__ inline RouteSmem route_smem(const LayerParams& p, int cl, bool fuse) {
+  RouteSmem L;
+  L.kc4 = (p.kc + 3) & ~3;
+  L.per = ((p.n_chunks + cl - 1) / cl + 3) & ~3;
+  if (fuse && L.per < p.kc * p.Ng) L.per = (p.kc * p.Ng + 3) & ~3;  // level-2 scores reuse it
+  L.lsel_n = fuse && p.kg > L.kc4 ? ((p.kg + 3) & ~3) : L.kc4;       // level-2 ids reuse it
+  return L;
+}
+
 // One cluster of `cl` CTAs per (sequence, KV head, block): CTA r scores the
 // r-th slice of the candidates into its own shared memory; after a cluster
 // barrier, CTA 0 gathers every slice through distributed shared memory and
 // runs the top-k.  With cl == 1 this is a plain single-CTA scan.
-template <typename T, int D>
+// With FUSE, CTA rank 0 continues into level 2 (the work of route_groups_kernel)
+// with the selected chunks still in shared memory; results are identical to the
+// two separate launches.
+// One cluster of `cl` CTAs per (sequence, KV head, block): CTA r scores the
+// r-th slice of the candidates and selects that slice's top-kc, then pushes
+// those (score, index) pairs into CTA 0's shared memory (distributed shared
+// memory stores).  CTA 0 takes the top-kc of the pushed pairs: the global
+// top-kc is always among the slices' top-kc, and the slices are pushed in
+// candidate order, so ties still go to the lower index.  With FUSE, CTA 0
+// continues into level 2 (the work of route_groups_kernel) with the selected
+// chunks still in shared memory; results are identical to the two launches.
+template <typename T, int D, bool FUSE>
 __global__ void __launch_bounds__(kThreads)
 route_chunks_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
-                    const float* __restrict__ chunk_sum, LayerParams p,
-                    int32_t* __restrict__ chunk_idx, float* __restrict__ chunk_score,
-                    unsigned* err) {
+                    const float* __restrict__ chunk_sum, const float* __restrict__ group_sum,
+                    LayerParams p, int32_t* __restrict__ chunk_idx,
+                    float* __restrict__ chunk_score, int32_t* __restrict__ group_idx,
+                    float* __restrict__ group_score, unsigned* err) {
   __shared__ __align__(16) float qbar[D];
   __shared__ float part[kWarps][D];
   __shared__ TopkSmem tsm;
+  __shared__ int s_cnt[8];
   extern __shared__ __align__(16) float dyn[];
   cg::cluster_group cluster = cg::this_cluster();
+  cluster.barrier_arrive();  // paired with barrier_wait() before the first remote store
   const int cl = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   const int item = blockIdx.x / cl;
@@ -132,39 +163,93 @@ route_chunks_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
     routing_query<T, D>(q, p, b, h, r0, nr, qbar, part);  // q is never written by this library
   }
   pdl_wait();
-  pdl_trigger();
 
   const int n_cand = ok ? max(0, cur - p.local - p.sink) : 0;
-  const int per = ((p.n_chunks + cl - 1) / cl + 3) & ~3;  // slice capacity (keeps sc 16 B aligned)
-  float* local = dyn;                                 // [per]: this CTA's slice
-  float* sc = cl == 1 ? dyn : dyn + per;              // [n_chunks]: gathered (rank 0)
-  int* sel = reinterpret_cast<int*>(sc + p.n_chunks); // [kc]
+  const RouteSmem L = route_smem(p, cl, FUSE);
+  const int kc4 = L.kc4;
+  float* local = dyn;                                             // [per]
+  int* lsel = reinterpret_cast<int*>(local + L.per);              // [lsel_n]
+  float* rsc = reinterpret_cast<float*>(lsel + L.lsel_n);         // [8 * kc4] pushed scores
+  int* ridx = reinterpret_cast<int*>(rsc + 8 * kc4);              // [8 * kc4] pushed indices
+  float* msc = reinterpret_cast<float*>(ridx + 8 * kc4);          // [8 * kc4] merged, compact
+  int* midx = reinterpret_cast<int*>(msc + 8 * kc4);              // [8 * kc4]
+  int* sel = reinterpret_cast<int*>(midx + 8 * kc4);              // [kc4]
   const int slice = (n_cand + cl - 1) / cl;
   const int lo = min(n_cand, rank * slice), hi = min(n_cand, lo + slice);
   const float* rows = chunk_sum + (static_cast<size_t>(bh) * p.n_chunks + p.sink + lo) * D;
   score_rows<D>(hi - lo, qbar, local, [&](int i) { return rows + static_cast<size_t>(i) * D; });
-  cluster.sync();
-  if (rank == 0 && cl > 1) {
-    for (int i = threadIdx.x; i < n_cand; i += kThreads) {
-      const int r = i / slice;
-      const float* src = cluster.map_shared_rank(local, r);
-      sc[i] = src[i - r * slice];
+  __syncthreads();
+  const int nl = hi - lo <= kRankTopkMax ? block_topk_rank<kThreads>(local, hi - lo, p.kc, lsel, tsm)
+                                         : block_topk<kThreads>(local, hi - lo, p.kc, lsel, tsm);
+  cluster.barrier_wait();  // every CTA of the cluster is running
+  {
+    float* dst_sc = cluster.map_shared_rank(rsc, 0);
+    int* dst_idx = cluster.map_shared_rank(ridx, 0);
+    for (int j = threadIdx.x; j < nl; j += kThreads) {
+      dst_sc[rank * kc4 + j] = local[lsel[j]];
+      dst_idx[rank * kc4 + j] = lo + lsel[j];
     }
+    if (threadIdx.x == 0) cluster.map_shared_rank(s_cnt, 0)[rank] = nl;
   }
-  cluster.sync();  // remote slices read; the other CTAs may leave
+  cluster.sync();  // pushes visible to CTA 0
   if (rank != 0) return;
+  int32_t* gout = FUSE ? group_idx + static_cast<size_t>(item) * p.kg : nullptr;
+  float* gout_sc = FUSE && group_score ? group_score + static_cast<size_t>(item) * p.kg : nullptr;
   if (!ok) {
     for (int i = threadIdx.x; i < p.kc; i += kThreads) {
       out[i] = -1;
       if (out_sc) out_sc[i] = CUDART_NAN_F;
     }
+    if constexpr (FUSE) {
+      for (int i = threadIdx.x; i < p.kg; i += kThreads) {
+        gout[i] = -1;
+        if (gout_sc) gout_sc[i] = CUDART_NAN_F;
+      }
+    }
     return;
   }
-  const int ns = n_cand <= kRankTopkMax ? block_topk_rank<kThreads>(sc, n_cand, p.kc, sel, tsm)
-                                       : block_topk<kThreads>(sc, n_cand, p.kc, sel, tsm);
+  // compact the pushed lists in rank order (= ascending candidate index)
+  int n_m = 0;
+  for (int r = 0; r < cl; ++r) {
+    const int c = s_cnt[r];
+    for (int j = threadIdx.x; j < c; j += kThreads) {
+      msc[n_m + j] = rsc[r * kc4 + j];
+      midx[n_m + j] = ridx[r * kc4 + j];
+    }
+    n_m += c;
+  }
+  __syncthreads();
+  const int ns = n_m <= kRankTopkMax ? block_topk_rank<kThreads>(msc, n_m, p.kc, sel, tsm)
+                                     : block_topk<kThreads>(msc, n_m, p.kc, sel, tsm);
   for (int i = threadIdx.x; i < p.kc; i += kThreads) {
-    out[i] = i < ns ? sel[i] + p.sink : -1;
-    if (out_sc) out_sc[i] = i < ns ? sc[sel[i]] : CUDART_NAN_F;
+    out[i] = i < ns ? midx[sel[i]] + p.sink : -1;
+    if (out_sc) out_sc[i] = i < ns ? msc[sel[i]] : CUDART_NAN_F;
+  }
+  pdl_trigger();  // the other CTAs of the cluster have exited
+  if constexpr (FUSE) {
+    // level 2 over the groups of the ns selected chunks (ascending chunk ids)
+    float* gsc = local;                                      // reuse: [kc * Ng] (fits: see launcher)
+    int* gsel = lsel;                                        // reuse: [kg]
+    const int n_g = ns * p.Ng;
+    const float* gbase = group_sum + static_cast<size_t>(bh) * p.n_chunks * p.Ng * D;
+    __syncthreads();  // everyone is done with local / lsel
+    score_rows<D>(n_g, qbar, gsc, [&](int i) {
+      const int c = midx[sel[i / p.Ng]] + p.sink, gi = i % p.Ng;
+      return gbase + (static_cast<size_t>(c) * p.Ng + gi) * D;
+    });
+    __syncthreads();
+    const int ng = n_g <= kRankTopkMax ? block_topk_rank<kThreads>(gsc, n_g, p.kg, gsel, tsm)
+                                       : block_topk<kThreads>(gsc, n_g, p.kg, gsel, tsm);
+    for (int i = threadIdx.x; i < p.kg; i += kThreads) {
+      if (i < ng) {
+        const int sidx = gsel[i];
+        gout[i] = (midx[sel[sidx / p.Ng]] + p.sink) * p.Ng + sidx % p.Ng;
+        if (gout_sc) gout_sc[i] = gsc[sidx];
+      } else {
+        gout[i] = -1;
+        if (gout_sc) gout_sc[i] = CUDART_NAN_F;
+      }
+    }
   }
 }
 
@@ -188,7 +273,6 @@ route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
   const int64_t pb = pos[b];
   if (!valid_position(pb, p, threadIdx.x == 0 ? err : nullptr)) {
     pdl_wait();
-    pdl_trigger();
     for (int i = threadIdx.x; i < p.kg; i += kThreads) {
       out[i] = -1;
       if (out_sc) out_sc[i] = CUDART_NAN_F;
@@ -199,7 +283,6 @@ route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
   block_rows(p, pb, blk, &r0, &nr, &cur);
   routing_query<T, D>(q, p, b, h, r0, nr, qbar, part);  // q is never written by this library
   pdl_wait();
-  pdl_trigger();
 
   const int n_cand_max = p.kc * p.Ng;
   float* sc = dyn;                                        // [kc * Ng]
@@ -237,30 +320,30 @@ route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
       if (out_sc) out_sc[i] = CUDART_NAN_F;
     }
   }
+  pdl_trigger();
 }
 
-// CTAs per cluster for the chunk scan: enough CTAs to cover the SMs a few
-// times, at most 8 (the portable cluster size), slices of at least 32 rows.
+// CTAs per cluster for the chunk scan: at most 8 (the portable cluster size),
+// no more CTAs in total than fit at once (4 per SM), slices of >= 32 rows.
 int chunk_cluster_size(const LayerParams& p) {
   const int64_t items = static_cast<int64_t>(p.B) * p.Hkv * p.nblk;
   int cl = 1;
-  while (cl < 8 && items * cl * 2 <= 148 * 8 && p.n_chunks / (cl * 2) >= 32) cl *= 2;
+  while (cl < 8 && items * cl * 2 <= 148 * 4 && p.n_chunks / (cl * 2) >= 32) cl *= 2;
   return cl;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool FUSE>
 cudaError_t launch_route_chunks_t(const LayerParams& p, const void* q, const int64_t* pos,
-                                  const float* chunk_sum, int32_t* chunk_idx, float* chunk_score,
-                                  unsigned* err, cudaStream_t s) {
+                                  const float* chunk_sum, const float* group_sum,
+                                  int32_t* chunk_idx, float* chunk_score, int32_t* group_idx,
+                                  float* group_score, unsigned* err, cudaStream_t s) {
   const int cl = chunk_cluster_size(p);
-  const int per = ((p.n_chunks + cl - 1) / cl + 3) & ~3;
-  const size_t smem = static_cast<size_t>(per + (cl > 1 ? p.n_chunks : 0)) * sizeof(float) +
-                      p.kc * sizeof(int);
-  cudaError_t e = ensure_smem<route_chunks_kernel<T, D>>(smem);
+  const size_t smem = route_smem(p, cl, FUSE).words() * 4;
+  cudaError_t e = ensure_smem<route_chunks_kernel<T, D, FUSE>>(smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(route_chunks_kernel<T, D>, dim3(p.B * p.Hkv * p.nblk * cl), dim3(kThreads),
-                    smem, s, cl, static_cast<const T*>(q), pos, chunk_sum, p, chunk_idx,
-                    chunk_score, err);
+  return launch_pdl(route_chunks_kernel<T, D, FUSE>, dim3(p.B * p.Hkv * p.nblk * cl),
+                    dim3(kThreads), smem, s, cl, static_cast<const T*>(q), pos, chunk_sum,
+                    group_sum, p, chunk_idx, chunk_score, group_idx, group_score, err);
 }
 
 template <typename T, int D>
@@ -282,12 +365,24 @@ cudaError_t launch_route_groups_t(const LayerParams& p, const void* q, const int
 cudaError_t launch_route_chunks(const LayerParams& p, int dtype, const void* q, const int64_t* pos,
                                 const float* chunk_sum, int32_t* chunk_idx, float* chunk_score,
                                 unsigned* err, cudaStream_t s) {
+  using bf = __nv_bfloat16;
   if (dtype == 0)
-    return p.D == 64 ? launch_route_chunks_t<float, 64>(p, q, pos, chunk_sum, chunk_idx, chunk_score, err, s)
-                     : launch_route_chunks_t<float, 128>(p, q, pos, chunk_sum, chunk_idx, chunk_score, err, s);
-  return p.D == 64
-             ? launch_route_chunks_t<__nv_bfloat16, 64>(p, q, pos, chunk_sum, chunk_idx, chunk_score, err, s)
-             : launch_route_chunks_t<__nv_bfloat16, 128>(p, q, pos, chunk_sum, chunk_idx, chunk_score, err, s);
+    return p.D == 64 ? launch_route_chunks_t<float, 64, false>(p, q, pos, chunk_sum, nullptr, chunk_idx, chunk_score, nullptr, nullptr, err, s)
+                     : launch_route_chunks_t<float, 128, false>(p, q, pos, chunk_sum, nullptr, chunk_idx, chunk_score, nullptr, nullptr, err, s);
+  return p.D == 64 ? launch_route_chunks_t<bf, 64, false>(p, q, pos, chunk_sum, nullptr, chunk_idx, chunk_score, nullptr, nullptr, err, s)
+                   : launch_route_chunks_t<bf, 128, false>(p, q, pos, chunk_sum, nullptr, chunk_idx, chunk_score, nullptr, nullptr, err, s);
+}
+
+cudaError_t launch_route(const LayerParams& p, int dtype, const void* q, const int64_t* pos,
+                         const float* chunk_sum, const float* group_sum, int32_t* chunk_idx,
+                         float* chunk_score, int32_t* group_idx, float* group_score,
+                         unsigned* err, cudaStream_t s) {
+  using bf = __nv_bfloat16;
+  if (dtype == 0)
+    return p.D == 64 ? launch_route_chunks_t<float, 64, true>(p, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx, group_score, err, s)
+                     : launch_route_chunks_t<float, 128, true>(p, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx, group_score, err, s);
+  return p.D == 64 ? launch_route_chunks_t<bf, 64, true>(p, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx, group_score, err, s)
+                   : launch_route_chunks_t<bf, 128, true>(p, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx, group_score, err, s);
 }
 
 cudaError_t launch_route_groups(const LayerParams& p, int dtype, const void* q, const int64_t* pos,

@@ -73,7 +73,6 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   }
   __syncthreads();
   pdl_wait();
-  pdl_trigger();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
@@ -151,6 +150,7 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
     }
     __syncthreads();
   }
+  pdl_trigger();
 }
 
 template <typename T, int D>

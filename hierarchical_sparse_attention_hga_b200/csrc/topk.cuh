@@ -151,8 +151,13 @@ __device__ int block_topk(const float* sc, int n, int k, int* sel, TopkSmem& sm)
     for (int i = tid; i < 256; i += NT) sm.hist[i] = 0u;
     __syncthreads();
     for (int i = tid; i < n; i += NT) {
+      // lanes hitting the same bin add once, with the lane count (similar
+      // scores share their top bits, so this avoids serialised atomics)
       const unsigned key = order_key(sc[i]);
-      if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
+      const bool hit = (key & pmask) == prefix;
+      const unsigned bin = hit ? (key >> shift) & 255u : 0xffffffffu;
+      const unsigned peers = __match_any_sync(__activemask(), bin);
+      if (hit && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], __popc(peers));
     }
     __syncthreads();
     if (wid == 0) {

@@ -105,8 +105,10 @@ hga_status hga_device_status(void* stream);
 
 /*
  * Bytes of device workspace hga_attend needs for (cfg, n_alloc, q_len).  Zero
- * is a valid answer.  The workspace holds per-split partial results of the
- * split-K decode; its contents need no initialisation and are scratch.
+ * is a valid answer (bf16 decode with D = 128 merges its split-K partials inside
+ * a thread-block cluster and needs none).  Otherwise the workspace holds the
+ * per-split partial results of the split-K decode; its contents need no
+ * initialisation and are scratch.
  */
 hga_status hga_workspace_size(const hga_config* cfg, int64_t n_alloc, int32_t q_len,
                               size_t* bytes);
@@ -188,6 +190,18 @@ hga_status hga_route_groups(const hga_config* cfg, const void* q, int32_t q_len,
                             const int64_t* pos, const float* group_sum, int64_t n_alloc,
                             const int32_t* chunk_idx, int32_t* group_idx, float* group_score,
                             void* stream);
+
+/*
+ * Steps 2 and 3 in one launch (same passages as hga_route_chunks and
+ * hga_route_groups).  Writes exactly what hga_route_chunks followed by
+ * hga_route_groups writes - bit for bit - with the level-2 stage continuing
+ * inside the level-1 kernel, so a decode step pays one launch for routing.
+ * chunk_score and group_score may be NULL.
+ */
+hga_status hga_route(const hga_config* cfg, const void* q, int32_t q_len, const int64_t* pos,
+                     const float* chunk_sum, const float* group_sum, int64_t n_alloc,
+                     int32_t* chunk_idx, float* chunk_score, int32_t* group_idx,
+                     float* group_score, void* stream);
 
 /*
  * Steps 4-5 - gather of the selected tokens' original K/V and exact softmax

@@ -97,16 +97,20 @@ def test_null_pointers_rejected_before_any_cuda_call(lib):
     with pytest.raises(B.HGAError) as e:
         B.hga_route_chunks(layer, None, 1, None, None, 4096, None, stream=0)
     assert e.value.status == 1
+    f32 = B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128, dtype=B.HGA_F32)
     with pytest.raises(B.HGAError) as e:
-        B.hga_attend(layer, 16, 1, 16, 16, 16, 4096, 16, 16, workspace=None, workspace_bytes=0,
+        B.hga_attend(f32, 16, 1, 16, 16, 16, 4096, 16, 16, workspace=None, workspace_bytes=0,
                      stream=0)
-    assert e.value.status == 7  # decode needs split-K workspace
+    assert e.value.status == 7  # fp32 decode needs split-K workspace
 
 
 def test_workspace_size_is_zero_for_prefill_and_grows_with_batch(lib):
     from hierarchical_sparse_attention_hga_b200 import binding as B
-    small = B.hga_workspace_size(B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128), 32768, 1)
-    big = B.hga_workspace_size(B.Layer(batch=16, heads_q=32, heads_kv=8, head_dim=128), 32768, 1)
+    f32 = dict(heads_q=32, heads_kv=8, head_dim=128, dtype=B.HGA_F32)
+    small = B.hga_workspace_size(B.Layer(batch=1, **f32), 32768, 1)
+    big = B.hga_workspace_size(B.Layer(batch=16, **f32), 32768, 1)
     assert 0 < small < big
-    assert B.hga_workspace_size(B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128), 32768,
-                                1024) == 0
+    assert B.hga_workspace_size(B.Layer(batch=1, **f32), 32768, 1024) == 0
+    # bf16, D = 128 decode merges its split-K partials inside a CTA cluster
+    assert B.hga_workspace_size(B.Layer(batch=16, heads_q=32, heads_kv=8, head_dim=128), 32768,
+                                1) == 0

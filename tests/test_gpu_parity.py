@@ -212,3 +212,41 @@ def test_router_with_odd_chunk_counts(context, batch):
     for b in range(batch):
         for h in range(2):
             compare_head(wl, x, res, b, h)
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("llama3_8b_decode_32k", dict(batch=3, context=8192)),
+    ("wide_head_decode_64k", dict(batch=2, context=8192, chunk=128, topk_chunks=32, topk_groups=64)),
+    ("llama3_8b_prefill_64k", dict(context=2048, heads_q=8, heads_kv=2)),
+    ("tiny_f32_1k", dict()),
+])
+def test_fused_route_is_bitwise_the_two_calls(name, kw):
+    from gpu_harness import layer_of, to_device
+    wl = S.workload(name, **kw)
+    x = S.make_inputs(wl, 22)
+    layer = layer_of(wl)
+    n = wl.context
+    q_len = x["q"].shape[2]
+    nblk = 1 if q_len == 1 else q_len // wl.chunk
+    bh = wl.batch * wl.heads_kv
+    q, k = to_device(x["q"], wl.dtype), to_device(x["k"], wl.dtype)
+    pos = torch.as_tensor(x["pos"], device="cuda")
+    cs = torch.empty(bh, n // wl.chunk, wl.head_dim, device="cuda")
+    gs = torch.empty(bh, n // wl.chunk, wl.chunk // wl.group, wl.head_dim, device="cuda")
+    B.hga_build_summaries(layer, k, n, 0, n, cs, gs)
+    outs = []
+    for fused in (False, True):
+        ci = torch.full((bh, nblk, wl.topk_chunks), -7, dtype=torch.int32, device="cuda")
+        gi = torch.full((bh, nblk, wl.topk_groups), -7, dtype=torch.int32, device="cuda")
+        csc = torch.empty((bh, nblk, wl.topk_chunks), device="cuda")
+        gsc = torch.empty((bh, nblk, wl.topk_groups), device="cuda")
+        if fused:
+            B.hga_route(layer, q, q_len, pos, cs, gs, n, ci, gi, csc, gsc)
+        else:
+            B.hga_route_chunks(layer, q, q_len, pos, cs, n, ci, csc)
+            B.hga_route_groups(layer, q, q_len, pos, gs, n, ci, gi, gsc)
+        torch.cuda.synchronize()
+        outs.append((ci.cpu(), gi.cpu(), csc.cpu(), gsc.cpu()))
+    assert B.hga_device_status() == 0
+    for a, b in zip(*outs):
+        assert torch.equal(a.nan_to_num(nan=-9.0), b.nan_to_num(nan=-9.0))

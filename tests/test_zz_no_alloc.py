@@ -66,8 +66,8 @@ def _attend_both(wl, layer, q, k, v, pos, gi):
 
 
 @pytest.mark.parametrize("name,kw", [
-    ("llama3_8b_decode_32k", dict(batch=4, context=4096)),          # bf16 TMA decode kernel
-    ("tiny_f32_1k", dict(batch=3, heads_q=4, heads_kv=2)),           # general split-K kernel
+    ("llama3_8b_decode_32k", dict(batch=4, context=4096, head_dim=64, n_high_pairs=16)),  # bf16
+    ("tiny_f32_1k", dict(batch=3, heads_q=4, heads_kv=2)),                                  # fp32
 ])
 def test_noalloc_matches_workspace_call_twice_in_a_row(name, kw):
     wl = S.workload(name, **kw)
@@ -83,7 +83,7 @@ def test_noalloc_matches_workspace_call_twice_in_a_row(name, kw):
 
 
 def test_noalloc_refuses_shapes_beyond_its_scratch():
-    wl = S.workload("wide_head_decode_64k", batch=256)
+    wl = S.workload("wide_head_decode_64k", batch=256, dtype="f32")  # general split-K kernel
     layer = layer_of(wl)
     assert B.hga_workspace_size(layer, wl.context, 1) > 8 << 20
     with pytest.raises(B.HGAError) as e:

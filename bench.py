@@ -161,7 +161,7 @@ def run_hga(args, rank: int, world: int):
     if args.batch:
         wl = wl.with_(batch=args.batch)
     if wl.prefill:
-        raise SystemExit("the decode bench takes a decode workload")
+        return run_prefill(args, rank, world, wl)
     dev = torch.device("cuda")
     seed = S.seed_for(list(S.WORKLOADS).index(args.workload)) + 7919 * rank
     x = S.make_inputs(wl, seed)
@@ -359,6 +359,211 @@ def run_hga(args, rank: int, world: int):
     return line, wl, seed, x
 
 
+# ------------------------------------------------------------------ prefill
+
+def prefill_flops(wl: S.Workload) -> float:
+    """Algorithmic FLOPs of the prefill attention (masked work excluded).
+
+    Per (sequence, KV head, block j) every query row sees the forced chunks
+    before the block, the routed groups and the causal part of its own chunk;
+    each visible (row, key) pair costs 4*D flops (Q K^T and P V).
+    """
+    c, g = wl.chunk, wl.group
+    ng = c // g
+    total_keys = 0
+    for j in range(wl.context // c):
+        b0 = max(0, j - wl.local)
+        forced = (min(wl.sink, b0) + (j - b0)) * c
+        n_cand = max(0, j - wl.local - wl.sink)
+        routed = min(wl.topk_groups, ng * min(wl.topk_chunks, n_cand)) * g
+        total_keys += c * (forced + routed) + c * (c + 1) // 2
+    return 4.0 * wl.head_dim * wl.gqa * total_keys * wl.batch * wl.heads_kv
+
+
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def run_prefill(args, rank: int, world: int, wl: S.Workload):
+    """One prefill step of one layer: summaries of the whole prompt, routing of
+    every 64-query block, attention of every query (steps 1-5)."""
+    import torch
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+
+    dev = torch.device("cuda")
+    seed = S.seed_for(list(S.WORKLOADS).index(args.workload)) + 7919 * rank
+    x = S.make_inputs(wl, seed)
+    n = wl.context
+    nblk = n // wl.chunk
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16))
+        return t.view(torch.bfloat16).to(dev)
+
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    pos = torch.as_tensor(x["pos"], device=dev)
+    layer = B.Layer(batch=wl.batch, heads_q=wl.heads_q, heads_kv=wl.heads_kv, head_dim=wl.head_dim,
+                    chunk=wl.chunk, group=wl.group, sink_chunks=wl.sink, local_chunks=wl.local,
+                    topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
+                    n_high_pairs=wl.n_high_pairs, rope_theta=wl.rope_theta, dtype=B.HGA_BF16,
+                    out_dtype=B.HGA_BF16)
+    bh = wl.batch * wl.heads_kv
+    cs = torch.empty(bh, n // wl.chunk, wl.head_dim, device=dev)
+    gs = torch.empty(bh, n // wl.chunk, wl.chunk // wl.group, wl.head_dim, device=dev)
+    ci = torch.empty(bh, nblk, wl.topk_chunks, dtype=torch.int32, device=dev)
+    gi = torch.empty(bh, nblk, wl.topk_groups, dtype=torch.int32, device=dev)
+    out = torch.empty(wl.batch, wl.heads_q, n, wl.head_dim, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(wl.batch, wl.heads_q, n, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    parts = {
+        "summaries": lambda: B.hga_build_summaries(layer, k, n, 0, n, cs, gs),
+        "route": lambda: B.hga_route(layer, q, n, pos, cs, gs, n, ci, gi),
+        "attend": lambda: B.hga_attend(layer, q, n, pos, k, v, n, gi, out, lse),
+    }
+
+    def step():
+        for fn in parts.values():
+            fn()
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert B.hga_device_status() == 0
+    graphs = {}
+    for name, fn in list(parts.items()) + [("step", step)]:
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_):
+            fn()
+        graphs[name] = g_
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def timed(g_, iters):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(iters)]
+        for a_, b_ in ev:
+            flush.zero_()
+            a_.record(stream)
+            g_.replay()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        return sum(a_.elapsed_time(b_) for a_, b_ in ev) / iters
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms_step = timed(graphs["step"], args.steps)
+    if dist:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    ms = {name: timed(graphs[name], max(3, min(args.steps, 20))) for name in parts}
+    assert B.hga_device_status() == 0
+
+    # e2e: host q in (pinned), host output back, every step; k/v resident
+    q_host = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e = []
+    for i in range(1 + min(args.steps, 5)):
+        flush.zero_()
+        e0.record(stream)
+        q.view(torch.int16).copy_(q_host, non_blocking=True)
+        graphs["step"].replay()
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i:
+            e2e.append(e0.elapsed_time(e1))
+    ms_e2e = sum(e2e) / len(e2e)
+
+    flops = prefill_flops(wl)
+    peak, peak_kind = tensor_peak()
+    achieved = flops / (ms["attend"] * 1e-3) / 1e12
+    tokens = wl.batch * n * world
+    line = {
+        "metric": METRIC + " (prefill)",
+        "value": tokens / (ms_step * 1e-3),
+        "unit": "prefill tokens/s (one attention layer)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "attn_us_per_layer": ms_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 q/k/v, fp32 accumulation (tcgen05)",
+        "data": "synthetic (seeded N(0,1) q/k/v)",
+        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": n,
+                   "heads_q": wl.heads_q, "heads_kv": wl.heads_kv, "head_dim": wl.head_dim,
+                   "chunk": wl.chunk, "query_block": wl.chunk, "topk_chunks": wl.topk_chunks,
+                   "topk_groups": wl.topk_groups,
+                   "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": f"replicas x{world}"},
+        "per_kernel_us": {kk: vv * 1e3 for kk, vv in ms.items()},
+        "attend_flops": flops,
+        "roofline": {"kernel": "attend", "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "algorithmic_flops": flops},
+        "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "prefill tokens/s (one attention layer)",
+                "ms_per_step": ms_e2e, "h2d_bytes_per_step": q_host.numel() * 2,
+                "d2h_bytes_per_step": out_host.numel() * 2},
+        "gpu_launches": 3 * args.steps,
+        "timing": "CUDA graph of the step replayed per timed step; CUDA events on the launch stream",
+        "clocks": clk.report(),
+    }
+    return line, wl, seed, x
+
+
+def oracle_prefill_rate(wl: S.Workload, seed: int, budget_s: float, x=None):
+    """Oracle prefill on a bounded sample of (KV head, query block) units: routing
+    of the block and attention of its G*C query rows.  Returns prompt tokens/s."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import hga_oracle as O
+    prm = O.HGAParams(head_dim=wl.head_dim, heads_q=wl.heads_q, heads_kv=wl.heads_kv,
+                      chunk=wl.chunk, group=wl.group, sink=wl.sink, local=wl.local,
+                      topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
+                      n_high_pairs=wl.n_high_pairs, rope_theta=wl.rope_theta)
+    g, c = wl.gqa, wl.chunk
+    nblk = wl.context // c
+    rng = np.random.default_rng(0)
+    units = [(h, int(j)) for h in range(wl.heads_kv) for j in rng.permutation(nblk)[:8]]
+    times, spent = [], 0.0
+    with threadpool_limits(limits=1):
+        cache = {}
+        for h, j in units:
+            if spent >= budget_s:
+                break
+            if h not in cache:
+                kb = x["k"][0, h] if x is not None else S.key_slice(wl, seed, 0, h)
+                vb = x["v"][0, h] if x is not None else S.value_slice(wl, seed, 0, h)
+                k64, v64 = S.widen(kb, wl.dtype), S.widen(vb, wl.dtype)
+                cache = {h: (k64, v64, O.build_summaries(k64, prm))}
+            k64, v64, (cs, gs) = cache[h]
+            qb = (x["q"][0, h * g:(h + 1) * g, j * c:(j + 1) * c] if x is not None else
+                  S.query_slice(wl, seed, 0)[h * g:(h + 1) * g, j * c:(j + 1) * c])
+            q64 = S.widen(qb, wl.dtype)
+            t0 = time.perf_counter()
+            qbar = O.routing_query(q64)
+            cidx, _, _ = O.route_chunks(qbar, cs, j, prm)
+            gidx, _, _ = O.route_groups(qbar, gs, cidx, prm)
+            for i in range(c):
+                toks = O.visible_tokens(j * c + i, j, gidx, prm)
+                for hh in range(g):
+                    O.attend(q64[hh, i], k64, v64, toks)
+            dt = time.perf_counter() - t0
+            times.append(dt)
+            spent += dt
+    per_unit = sum(times) / len(times)
+    step_s = per_unit * wl.heads_kv * nblk * wl.batch
+    sample = (f"{len(times)} (KV head, 64-query block) units of the {wl.context}-token prefill "
+              f"(routing + attention of every row), extrapolated ({sum(times):.1f} s of oracle time)")
+    return wl.batch * wl.context / step_s, sample, 1
+
+
 # ------------------------------------------------------------ oracle (CPU) arm
 
 def oracle_decode_rate(wl: S.Workload, seed: int, budget_s: float, x=None):
@@ -462,7 +667,8 @@ def main():
     line, wl, seed, x = run_hga(args, rank, world)
     if rank == 0:
         if not args.no_cpu_baseline:
-            val, sample, cores = oracle_decode_rate(wl, seed, args.cpu_seconds, x)
+            rate = oracle_prefill_rate if wl.prefill else oracle_decode_rate
+            val, sample, cores = rate(wl, seed, args.cpu_seconds, x)
             line["cpu_baseline"] = {"value": val, "unit": line["unit"], "cores": cores,
                                     "kind": "oracle", "sample": sample}
         print(json.dumps(line))

@@ -327,6 +327,8 @@ cudaError_t launch_attend(const LayerParams& p, int dtype, int out_dtype, const 
   using bf = __nv_bfloat16;
   if (use_decode_fast(p, dtype))
     return launch_attend_decode_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, err, s);
+  if (prefill_tc_path(p, dtype))
+    return launch_attend_prefill_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, err, s);
   if (dtype == 0)
     return out_dtype == 0 ? launch_attend_d<float, float>(p, q, pos, k, v, group_idx, out, lse, ws, err, s)
                           : launch_attend_d<float, bf>(p, q, pos, k, v, group_idx, out, lse, ws, err, s);

@@ -31,6 +31,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "tmap.h"
 
 namespace cg = cooperative_groups;
 
@@ -408,35 +409,6 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
 
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// Tensor map of a [rows, 128] bf16 cache, boxes of 16 rows x 64 columns, 128B swizzle.
-cudaError_t make_map(CUtensorMap* map, const void* base, int64_t rows) {
-  auto fn = encode_fn();
-  if (!fn) return cudaErrorNotSupported;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
-  const cuuint32_t box[2] = {64, kUnit};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 int max_units(const LayerParams& p) {
   return (p.sink + p.local + 1) * (p.C / kUnit) + p.kg;
 }
@@ -491,8 +463,8 @@ cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const
                                       unsigned* err, cudaStream_t s) {
   CUtensorMap tk, tv;
   const int64_t rows = static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc;
-  cudaError_t e = make_map(&tk, k, rows);
-  if (e == cudaSuccess) e = make_map(&tv, v, rows);
+  cudaError_t e = make_bf16_map(&tk, k, rows, kUnit);
+  if (e == cudaSuccess) e = make_bf16_map(&tv, v, rows, kUnit);
   if (e != cudaSuccess) return e;
   return out_dtype == 0
              ? launch_t<float>(p, tk, tv, q, pos, group_idx, out, lse, err, s)

@@ -1,0 +1,407 @@
+// Steps 4-5 for prefill, bf16 K/V with D = 128: gathered-tile attention of a
+// 64-query block on the 5th-generation tensor cores (tcgen05, TMEM).
+//
+// HGA technical summary ("Hierarchical Global Attention (HGA)", gist.science
+// 2606.30709), "Metodologia -> Meccanismo Core", item 4: every query attends
+// exactly, with a standard softmax, to the original K/V of the bounded token
+// set its block routed to (sink, local and current chunks plus the routed
+// groups), causal inside the current chunk.
+//
+// One CTA per (sequence, KV head, query block).  The block's G*C query rows
+// (G heads x C queries) form one or two M = 128 tiles.  Its token list is cut
+// into 16-token units ordered [sink | local | routed groups | current chunk],
+// and the units into KV tiles of 128 keys, so only the last tile(s) carry the
+// causal mask.  Warp roles (320 threads):
+//   warps 0-3, 4-7  softmax warpgroups of M-tile 0 and 1 (ping-pong): read
+//                   S = Q K^T from TMEM, masked online softmax in the log2
+//                   domain with lazy rescaling, write P (bf16) back over S;
+//   warp 8          TMA producer: Q once, then K and V tiles (two 16 x 64 boxes
+//                   per unit and tensor, 128B swizzle) into a 2-stage ring;
+//   warp 9          tcgen05.mma issuer and TMEM owner (512 columns: per M-tile
+//                   128 for S/P and 128 for O).
+// S_mt(t) = Q_mt K(t)^T and O_mt += P_mt(t) V(t) run on M = 128, N = 128,
+// K = 16 instructions; P is the A operand straight from TMEM, V the B operand
+// in MN-major layout.  O accumulates in TMEM; a row's O is rescaled only when
+// its running maximum grows by more than 2^8, so rescaling is rare.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+#include "tmap.h"
+#include "topk.cuh"
+
+namespace hga {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kUnit = 16;
+constexpr int kUnitsPerTile = 8;                // 128 keys
+constexpr int kMaxUnits = 512;
+constexpr int kChunkBytes = 128 * 128;          // 128 rows x 64 bf16
+constexpr int kTileBytes = 2 * kChunkBytes;     // 128 rows x 128 bf16
+constexpr int kStages = 2;
+constexpr int kThreads = 320;
+constexpr int kSmemBytes = (2 + 2 * kStages) * kTileBytes + 1024;
+constexpr uint32_t kWaitLimit = 1u << 26;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.f;
+
+// Routed groups of one block, kept if they name a group of a candidate chunk
+// and come in strictly ascending order; writes their first tokens to dst
+// (warp-collective; returns the count).
+__device__ __forceinline__ int warp_keep_ascending_groups(const int32_t* gl, int kg,
+                                                          const LayerParams& p, int cur, int* dst,
+                                                          bool* bad) {
+  const int m = warp_keep_ascending(
+      gl, kg,
+      [&](int gid) {
+        const int c = gid / p.Ng;
+        return c >= p.sink && c < cur - p.local;
+      },
+      dst, bad);
+  __syncwarp();
+  for (int i = threadIdx.x & 31; i < m; i += 32) dst[i] *= kUnit;
+  __syncwarp();
+  return m;
+}
+
+template <typename TO>
+struct PrefillArgs {
+  const int64_t* pos;
+  const int32_t* group_idx;
+  TO* out;
+  float* lse;
+  unsigned* err;
+};
+
+__device__ __forceinline__ void store_row(float* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4)
+    *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+}
+__device__ __forceinline__ void store_row(__nv_bfloat16* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    uint4 w;
+    w.x = ptx::pack_bf16x2(v[j], v[j + 1]);
+    w.y = ptx::pack_bf16x2(v[j + 2], v[j + 3]);
+    w.z = ptx::pack_bf16x2(v[j + 4], v[j + 5]);
+    w.w = ptx::pack_bf16x2(v[j + 6], v[j + 7]);
+    *reinterpret_cast<uint4*>(dst + j) = w;
+  }
+}
+
+template <typename TO>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, PrefillArgs<TO> a,
+                      LayerParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_q, bar_full[kStages], bar_empty[kStages];
+  __shared__ uint64_t bar_s[2], bar_p[2], bar_o[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_unit[kMaxUnits];  // first token of each unit of the list
+  __shared__ int s_nunits;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x;
+  const int blk = item % p.nblk;
+  const int bh = item / p.nblk;
+  const int h = bh % p.Hkv, b = bh / p.Hkv;
+  const int n_mt = p.G * p.C / 128;  // M-tiles (1 or 2)
+  const int heads_per_tile = 128 / p.C;
+
+  uint8_t* base = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sq = base;                                 // [2][32 KB] Q tiles
+  uint8_t* sk = base + 2 * kTileBytes;                // [kStages][32 KB] K ring
+  uint8_t* sv = sk + kStages * kTileBytes;            // [kStages][32 KB] V ring
+
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tensormap(&tm_q);
+    ptx::prefetch_tensormap(&tm_k);
+    ptx::prefetch_tensormap(&tm_v);
+    ptx::mbar_init(&bar_q, 1);
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(&bar_full[s], 1);
+      ptx::mbar_init(&bar_empty[s], 1);
+    }
+    for (int m = 0; m < 2; ++m) {
+      ptx::mbar_init(&bar_s[m], 1);
+      ptx::mbar_init(&bar_p[m], 128);
+      ptx::mbar_init(&bar_o[m], 1);
+    }
+    ptx::fence_barrier_init();
+  }
+  if (warp == 9) ptx::tmem_alloc(&s_tmem, 512);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  const int64_t pb = a.pos[b];  // never written by this library
+  const bool ok = valid_position(pb, p, threadIdx.x == 0 ? a.err : nullptr);
+  const int64_t first = pb - p.q_len + 1;
+  const int cur = ok ? static_cast<int>(first / p.C) + blk : 0;
+  const int64_t q_row0 = (static_cast<int64_t>(b) * p.Hq + h * p.G) * p.q_len +
+                         static_cast<int64_t>(blk) * p.C;  // row of head 0, query 0
+
+  // Q does not depend on routing: the producer starts it before the wait.
+  if (warp == 8 && lane == 0 && ok) {
+    ptx::mbar_expect_tx(&bar_q, n_mt * kTileBytes);
+    for (int mt = 0; mt < n_mt; ++mt)
+      for (int hs = 0; hs < heads_per_tile; ++hs)
+        for (int rb = 0; rb < p.C / 64; ++rb)
+          for (int kc = 0; kc < 2; ++kc) {
+            const int hh = mt * heads_per_tile + hs;
+            const int64_t row = q_row0 + static_cast<int64_t>(hh) * p.q_len + rb * 64;
+            ptx::tma_load_2d(sq + mt * kTileBytes + kc * kChunkBytes + (hs * p.C + rb * 64) * 128,
+                             &tm_q, &bar_q, kc * 64, static_cast<int32_t>(row));
+          }
+  }
+  pdl_wait();  // group_idx may come from the kernel just before
+
+  // Unit list: [sink | local | routed | current], first token of each unit.
+  if (warp == 0) {
+    int n = 0;
+    if (ok) {
+      const int b0 = max(0, cur - p.local);
+      const int a_end = min(p.sink, b0);
+      const int nf = (a_end + (cur - b0)) * p.Ng;  // sink and local units
+      for (int i = lane; i < nf; i += 32) {
+        const int ci = i / p.Ng, gi = i % p.Ng;
+        const int c = ci < a_end ? ci : b0 + (ci - a_end);
+        s_unit[i] = (c * p.Ng + gi) * kUnit;
+      }
+      n = nf;
+      bool bad = false;
+      const int32_t* gl = a.group_idx + static_cast<size_t>(item) * p.kg;
+      int* dst = s_unit + n;
+      const int m = warp_keep_ascending_groups(gl, p.kg, p, cur, dst, &bad);
+      n += m;
+      for (int i = lane; i < p.Ng; i += 32) s_unit[n + i] = (cur * p.Ng + i) * kUnit;
+      n += p.Ng;
+      if (bad && lane == 0) flag_error(a.err, kErrGroupIdx);
+    }
+    if (lane == 0) s_nunits = n;
+  }
+  __syncthreads();
+  const int n_units = s_nunits;
+  const int n_tiles = (n_units + kUnitsPerTile - 1) / kUnitsPerTile;
+  bool timed_out = false;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const int64_t kv_row0 = static_cast<int64_t>(bh) * p.n_alloc;
+      for (int t = 0; t < n_tiles && !timed_out; ++t) {
+        const int s = t % kStages;
+        if (t >= kStages &&
+            !ptx::mbar_wait(&bar_empty[s], ((t - kStages) / kStages) & 1, kWaitLimit)) {
+          timed_out = true;
+          break;
+        }
+        ptx::mbar_expect_tx(&bar_full[s], 2 * kTileBytes);
+        for (int us = 0; us < kUnitsPerTile; ++us) {
+          const int u = t * kUnitsPerTile + us;
+          // slots past the list reload unit 0 (finite data; masked to zero weight)
+          const int32_t y = static_cast<int32_t>(kv_row0 + s_unit[u < n_units ? u : 0]);
+          for (int kc = 0; kc < 2; ++kc) {
+            const int off = s * kTileBytes + kc * kChunkBytes + us * kUnit * 128;
+            ptx::tma_load_2d(sk + off, &tm_k, &bar_full[s], kc * 64, y);
+            ptx::tma_load_2d(sv + off, &tm_v, &bar_full[s], kc * 64, y);
+          }
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc_s = ptx::umma_idesc_bf16(128, 128, false, false);
+      const uint32_t idesc_o = ptx::umma_idesc_bf16(128, 128, false, true);
+      const uint32_t sq_a = ptx::smem_u32(sq), sk_a = ptx::smem_u32(sk), sv_a = ptx::smem_u32(sv);
+      auto issue_s = [&](int mt, int stage) {
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          const uint64_t ad = ptx::umma_desc_sw128(sq_a + mt * kTileBytes + koff, 16, 1024);
+          const uint64_t bd = ptx::umma_desc_sw128(sk_a + stage * kTileBytes + koff, 16, 1024);
+          ptx::umma_ss(tmem + mt * 256, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int mt, int stage, bool first_tile) {
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd =
+              ptx::umma_desc_sw128(sv_a + stage * kTileBytes + kk * kUnit * 128, kChunkBytes, 1024);
+          ptx::umma_ts(tmem + mt * 256 + 128, tmem + mt * 256 + kk * 8, bd, idesc_o,
+                       (!first_tile || kk > 0) ? 1u : 0u);
+        }
+      };
+      if (!ptx::mbar_wait(&bar_q, 0, kWaitLimit) || !ptx::mbar_wait(&bar_full[0], 0, kWaitLimit)) {
+        timed_out = true;
+      } else {
+        ptx::tc_fence_after();
+        for (int mt = 0; mt < n_mt; ++mt) {
+          issue_s(mt, 0);
+          ptx::umma_commit(&bar_s[mt]);
+        }
+        for (int t = 0; t < n_tiles && !timed_out; ++t) {
+          for (int mt = 0; mt < n_mt; ++mt) {
+            if (!ptx::mbar_wait(&bar_p[mt], t & 1, kWaitLimit)) { timed_out = true; break; }
+            ptx::tc_fence_after();
+            issue_pv(mt, t % kStages, t == 0);
+            if (mt == n_mt - 1) ptx::umma_commit(&bar_empty[t % kStages]);
+            if (t + 1 < n_tiles) {
+              if (mt == 0) {
+                if (!ptx::mbar_wait(&bar_full[(t + 1) % kStages], ((t + 1) / kStages) & 1,
+                                    kWaitLimit)) {
+                  timed_out = true;
+                  break;
+                }
+                ptx::tc_fence_after();
+              }
+              issue_s(mt, (t + 1) % kStages);
+              ptx::umma_commit(&bar_s[mt]);
+            } else {
+              ptx::umma_commit(&bar_o[mt]);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp < 4 * n_mt) {
+    // ----------------------------------------------------------- softmax (M-tile)
+    const int mt = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;                 // row of the M-tile = TMEM lane
+    const int hh = mt * heads_per_tile + r / p.C;         // query head within the group
+    const int qi = r % p.C;                               // query within the block
+    const int64_t qpos = static_cast<int64_t>(cur) * p.C + qi;
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + mt * 256;
+    const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
+    float m_used = -CUDART_INF_F, l = 0.f;
+    // key column c of tile t is valid when its unit exists and its token is <= qpos
+    auto col_ok = [&](int t, int c) -> bool {
+      const int u = t * kUnitsPerTile + (c >> 4);
+      return u < n_units && static_cast<int64_t>(s_unit[u] + (c & 15)) <= qpos;
+    };
+    for (int t = 0; t < n_tiles; ++t) {
+      if (!ptx::mbar_wait(&bar_s[mt], t & 1, kWaitLimit)) { timed_out = true; break; }
+      ptx::tc_fence_after();
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t v[32];
+        ptx::tmem_ld32(trow + ch * 32, v);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col_ok(t, ch * 32 + j)) mx = fmaxf(mx, __uint_as_float(v[j]) * sc);
+      }
+      if (mx > m_used + kRescaleLog2) {
+        if (m_used != -CUDART_INF_F) {  // O holds earlier tiles: rescale it
+          const float f = exp2f(m_used - mx);
+          l *= f;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t v[32];
+            ptx::tmem_ld32(trow + 128 + ch * 32, v);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+            ptx::tmem_st32(trow + 128 + ch * 32, v);
+          }
+        }
+        m_used = mx;
+      }
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t v[32], pk[16];
+        ptx::tmem_ld32(trow + ch * 32, v);
+        ptx::tmem_wait_ld();
+        float pr[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          pr[j] = col_ok(t, ch * 32 + j) && m_used != -CUDART_INF_F
+                      ? exp2f(__uint_as_float(v[j]) * sc - m_used)
+                      : 0.f;
+          l += pr[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = ptx::pack_bf16x2(pr[2 * j], pr[2 * j + 1]);
+        ptx::tmem_st16(trow + ch * 16, pk);  // P over the S columns already read
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bar_p[mt]);
+    }
+    // epilogue: O / l
+    const size_t orow = (static_cast<size_t>(b) * p.Hq + h * p.G + hh) * p.q_len +
+                        static_cast<size_t>(blk) * p.C + qi;
+    TO* dst = a.out + orow * kD;
+    const bool have = n_tiles > 0 && !timed_out && ptx::mbar_wait(&bar_o[mt], 0, kWaitLimit);
+    if (have) ptx::tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t v[32];
+      float o[32];
+      if (have) {
+        ptx::tmem_ld32(trow + 128 + ch * 32, v);
+        ptx::tmem_wait_ld();
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) o[j] = have ? __uint_as_float(v[j]) * inv : 0.f;
+      store_row(dst + ch * 32, o);
+    }
+    if (a.lse) a.lse[orow] = have && l > 0.f ? (m_used + log2f(l)) * kLn2 : -CUDART_INF_F;
+    if (n_tiles > 0 && !have) timed_out = true;
+  }
+  if (timed_out) flag_error(a.err, kErrTimeout);
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+  pdl_trigger();
+}
+
+template <typename TO>
+cudaError_t launch_t(const LayerParams& p, const void* q, const int64_t* pos, const void* k,
+                     const void* v, const int32_t* group_idx, void* out, float* lse,
+                     unsigned* err, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  const int64_t kv_rows = static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc;
+  const int64_t q_rows = static_cast<int64_t>(p.B) * p.Hq * p.q_len;
+  cudaError_t e = make_bf16_map(&tq, q, q_rows, 64);
+  if (e == cudaSuccess) e = make_bf16_map(&tk, k, kv_rows, kUnit);
+  if (e == cudaSuccess) e = make_bf16_map(&tv, v, kv_rows, kUnit);
+  if (e != cudaSuccess) return e;
+  PrefillArgs<TO> a{pos, group_idx, static_cast<TO*>(out), lse, err};
+  e = ensure_smem<attend_prefill_kernel<TO>>(kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(attend_prefill_kernel<TO>, dim3(p.B * p.Hkv * p.nblk), dim3(kThreads),
+                    kSmemBytes, s, 1, tq, tk, tv, a, p);
+}
+
+}  // namespace
+
+bool prefill_tc_path(const LayerParams& p, int dtype) {
+  const int64_t units = static_cast<int64_t>(p.sink + p.local + 1) * p.Ng + p.kg;
+  return dtype == 1 && p.D == kD && p.q_len > 1 && p.g == kUnit && p.C % 64 == 0 &&
+         (p.G * p.C == 128 || p.G * p.C == 256) && units <= kMaxUnits &&
+         static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc < (static_cast<int64_t>(1) << 31) &&
+         static_cast<int64_t>(p.B) * p.Hq * p.q_len < (static_cast<int64_t>(1) << 31);
+}
+
+cudaError_t launch_attend_prefill_bf16(const LayerParams& p, int out_dtype, const void* q,
+                                       const int64_t* pos, const void* k, const void* v,
+                                       const int32_t* group_idx, void* out, float* lse,
+                                       unsigned* err, cudaStream_t s) {
+  return out_dtype == 0 ? launch_t<float>(p, q, pos, k, v, group_idx, out, lse, err, s)
+                        : launch_t<__nv_bfloat16>(p, q, pos, k, v, group_idx, out, lse, err, s);
+}
+
+}  // namespace hga

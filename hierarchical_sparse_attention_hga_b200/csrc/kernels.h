@@ -92,6 +92,13 @@ cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const
                                       const int32_t* group_idx, void* out, float* lse,
                                       unsigned* err, cudaStream_t s);
 
+// The bf16, D = 128 prefill kernel (64-query blocks on tcgen05 / TMEM) applies to p.
+bool prefill_tc_path(const LayerParams& p, int dtype);
+cudaError_t launch_attend_prefill_bf16(const LayerParams& p, int out_dtype, const void* q,
+                                       const int64_t* pos, const void* k, const void* v,
+                                       const int32_t* group_idx, void* out, float* lse,
+                                       unsigned* err, cudaStream_t s);
+
 // Log-sum-exp merge of nsplit decode partials into out / lse.
 cudaError_t launch_combine(const LayerParams& p, int out_dtype, int nsplit, const float* ws_o,
                            const float* ws_ml, void* out, float* lse, cudaStream_t s);

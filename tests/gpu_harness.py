@@ -176,3 +176,43 @@ def compare_summaries(wl: S.Workload, x: dict, res: dict, b: int, h: int, n_vali
 
 def scale_of(x):
     return math.sqrt(float(np.mean(np.square(x))))
+
+
+def compare_prefill_blocks(wl: S.Workload, x: dict, res: dict, b: int, h: int, blocks,
+                           rows=(0, 1, 31, 63), tol: float | None = None):
+    """Prefill parity on chosen query blocks of one (b, h): routing of each block
+    and attention of the chosen rows, recomputed by the oracle for those only."""
+    prm = params_of(wl)
+    g, c = wl.gqa, wl.chunk
+    tol = TOL[wl.dtype] if tol is None else tol
+    k = S.widen(x["k"][b, h], wl.dtype)
+    v = S.widen(x["v"][b, h], wl.dtype)
+    pos_last = int(x["pos"][b])
+    q_len = x["q"].shape[2]
+    first = pos_last - q_len + 1
+    cs, gs = O.build_summaries(k, prm, n_valid=pos_last + 1)
+    for blk in blocks:
+        r0 = blk * c
+        cur = (first + r0) // c
+        q = S.widen(x["q"][b, h * g:(h + 1) * g, r0:r0 + c], wl.dtype)
+        qbar = O.routing_query(q)
+        cidx, ccand, cscore = O.route_chunks(qbar, cs, cur, prm)
+        scale = float(np.linalg.norm(qbar)) * max([float(np.linalg.norm(cs[j])) for j in ccand] or [1.0])
+        same = check_selection(res["chunk_idx"][b, h, blk], cidx, ccand, cscore, wl.topk_chunks,
+                               scale, f"prefill chunks b{b} h{h} blk{blk}")
+        chosen = cidx if same else list(res["chunk_idx"][b, h, blk])
+        gidx, gcand, gscore = O.route_groups(qbar, gs, chosen, prm)
+        gscale = float(np.linalg.norm(qbar)) * max(
+            [float(np.linalg.norm(gs[i // prm.groups_per_chunk, i % prm.groups_per_chunk]))
+             for i in gcand] or [1.0])
+        check_selection(res["group_idx"][b, h, blk], gidx, gcand, gscore, wl.topk_groups, gscale,
+                        f"prefill groups b{b} h{h} blk{blk}")
+        gsel = [int(i) for i in res["group_idx"][b, h, blk]]
+        for i in rows:
+            toks = O.visible_tokens(first + r0 + i, cur, gsel, prm)
+            for hh in range(g):
+                o, lse, _ = O.attend(q[hh, i], k, v, toks)
+                got = res["out"][b, h * g + hh, r0 + i]
+                err = float(np.max(np.abs(got - o)))
+                assert err <= tol, f"prefill out b{b} h{h} blk{blk} row{i} head{hh}: {err:.3e}"
+                assert abs(res["lse"][b, h * g + hh, r0 + i] - lse) <= max(tol, 1e-4)

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():  # pragma: no cover - collected on CPU too
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from gpu_harness import compare_head, compare_summaries, run_gpu  # noqa: E402
+from gpu_harness import compare_head, compare_prefill_blocks, compare_summaries, run_gpu  # noqa: E402
 from hierarchical_sparse_attention_hga_b200 import binding as B  # noqa: E402
 from oracle import hga_oracle as O  # noqa: E402
 
@@ -250,3 +250,28 @@ def test_fused_route_is_bitwise_the_two_calls(name, kw):
     assert B.hga_device_status() == 0
     for a, b in zip(*outs):
         assert torch.equal(a.nan_to_num(nan=-9.0), b.nan_to_num(nan=-9.0))
+
+
+# --------------------------------------------------------------- prefill (tcgen05)
+
+@pytest.mark.parametrize("heads_q,heads_kv,out_dtype", [(8, 2, B.HGA_F32), (4, 2, B.HGA_F32),
+                                                       (8, 2, B.HGA_BF16)])
+def test_prefill_tensor_core_path_small(heads_q, heads_kv, out_dtype):
+    """64-query blocks on tcgen05 (G*C = 256 or 128 rows), every block and row checked."""
+    wl = S.workload("llama3_8b_prefill_64k", context=1024, heads_q=heads_q, heads_kv=heads_kv,
+                    topk_chunks=4, topk_groups=8)
+    x = S.make_inputs(wl, 23)
+    res = run_gpu(wl, x, out_dtype=out_dtype)
+    for h in range(heads_kv):
+        compare_head(wl, x, res, 0, h)
+
+
+def test_prefill_tensor_core_path_8k_sampled_blocks():
+    """Llama-3-8B-shaped prefill at 8K context: many KV tiles per block, all workload k values."""
+    wl = S.workload("llama3_8b_prefill_64k", context=8192)
+    x = S.make_inputs(wl, 24)
+    res = run_gpu(wl, x)
+    assert np.isfinite(res["out"]).all()
+    for h in (0, 3, 7):
+        compare_prefill_blocks(wl, x, res, 0, h, blocks=(0, 1, 4, 5, 6, 37, 127),
+                               rows=(0, 9, 40, 63))

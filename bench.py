@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
     ap.add_argument("--workload", default="llama3_8b_decode_32k")
     ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--context", type=int, default=None, help="override the context length")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -160,6 +161,8 @@ def run_hga(args, rank: int, world: int):
     wl = S.workload(args.workload)
     if args.batch:
         wl = wl.with_(batch=args.batch)
+    if args.context:
+        wl = wl.with_(context=args.context)
     if wl.prefill:
         return run_prefill(args, rank, world, wl)
     dev = torch.device("cuda")

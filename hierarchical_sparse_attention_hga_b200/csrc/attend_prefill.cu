@@ -277,61 +277,81 @@ attend_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int r = (warp & 3) * 32 + lane;                 // row of the M-tile = TMEM lane
     const int hh = mt * heads_per_tile + r / p.C;         // query head within the group
     const int qi = r % p.C;                               // query within the block
-    const int64_t qpos = static_cast<int64_t>(cur) * p.C + qi;
     const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + mt * 256;
     const float sc = kLog2e * rsqrtf(static_cast<float>(kD));
     float m_used = -CUDART_INF_F, l = 0.f;
-    // key column c of tile t is valid when its unit exists and its token is <= qpos
-    auto col_ok = [&](int t, int c) -> bool {
-      const int u = t * kUnitsPerTile + (c >> 4);
-      return u < n_units && static_cast<int64_t>(s_unit[u] + (c & 15)) <= qpos;
-    };
+    // Units [0, u_cur0) are visible to every row; units [u_cur0, n_units) are
+    // the current chunk (causal: column offset <= qi); slots >= n_units are
+    // padding.  Only tiles reaching u_cur0 need a mask.
+    const int u_cur0 = n_units - p.Ng;
     for (int t = 0; t < n_tiles; ++t) {
       if (!ptx::mbar_wait(&bar_s[mt], t & 1, kWaitLimit)) { timed_out = true; break; }
       ptx::tc_fence_after();
-      float mx = -CUDART_INF_F;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t v[32];
-        ptx::tmem_ld32(trow + ch * 32, v);
+      // Two passes over the row's 128 scores in halves of 64 columns (it keeps
+      // a softmax thread within its register budget): the running max, then
+      // p = 2^(s*sc - m), whose bf16 pairs go back over the S columns read.
+      const bool masked = (t + 1) * kUnitsPerTile > u_cur0;
+      auto load_half = [&](int hf, uint32_t (&v)[2][32]) {
+        ptx::tmem_ld32(trow + hf * 64, v[0]);
+        ptx::tmem_ld32(trow + hf * 64 + 32, v[1]);
         ptx::tmem_wait_ld();
+        if (masked) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (col_ok(t, ch * 32 + j)) mx = fmaxf(mx, __uint_as_float(v[j]) * sc);
+          for (int j = 0; j < 64; ++j) {
+            const int c = hf * 64 + j;
+            const int u = t * kUnitsPerTile + (c >> 4);
+            const bool ok_j = u < u_cur0 || (u < n_units && (u - u_cur0) * kUnit + (c & 15) <= qi);
+            if (!ok_j) v[j >> 5][j & 31] = __float_as_uint(-CUDART_INF_F);
+          }
+        }
+      };
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t v[2][32];
+        load_half(hf, v);
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(v[j >> 5][j & 31]));
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sc;
       if (mx > m_used + kRescaleLog2) {
         if (m_used != -CUDART_INF_F) {  // O holds earlier tiles: rescale it
           const float f = exp2f(m_used - mx);
           l *= f;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
-            uint32_t v[32];
-            ptx::tmem_ld32(trow + 128 + ch * 32, v);
+            uint32_t o[32];
+            ptx::tmem_ld32(trow + 128 + ch * 32, o);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-            ptx::tmem_st32(trow + 128 + ch * 32, v);
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
+            ptx::tmem_st32(trow + 128 + ch * 32, o);
           }
         }
         m_used = mx;
       }
+      // masked scores are -inf and give exactly 0
+      const float nm = m_used == -CUDART_INF_F ? 0.f : -m_used;
+      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t v[32], pk[16];
-        ptx::tmem_ld32(trow + ch * 32, v);
-        ptx::tmem_wait_ld();
-        float pr[32];
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t v[2][32];
+        load_half(hf, v);
+        // pair j of this half lands in v[0][j/2], already consumed
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          pr[j] = col_ok(t, ch * 32 + j) && m_used != -CUDART_INF_F
-                      ? exp2f(__uint_as_float(v[j]) * sc - m_used)
-                      : 0.f;
-          l += pr[j];
+        for (int j = 0; j < 64; j += 2) {
+          const float p0 = exp2f(fmaf(__uint_as_float(v[j >> 5][j & 31]), sc, nm));
+          const float p1 = exp2f(fmaf(__uint_as_float(v[j >> 5][(j & 31) + 1]), sc, nm));
+          l8[(j >> 1) & 7] += p0 + p1;
+          v[0][j >> 1] = ptx::pack_bf16x2(p0, p1);
         }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) pk[j] = ptx::pack_bf16x2(pr[2 * j], pr[2 * j + 1]);
-        ptx::tmem_st16(trow + ch * 16, pk);  // P over the S columns already read
+        ptx::tmem_st32(trow + hf * 32, v[0]);  // P columns 32*hf .. 32*hf+31
       }
+      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bar_p[mt]);

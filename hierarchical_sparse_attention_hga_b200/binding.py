@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_SHAPE", 3: "H
 # Exported symbols of the C ABI, in header order.
 SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device_status",
            "hga_workspace_size", "hga_build_summaries", "hga_route_chunks", "hga_route_groups",
-           "hga_route", "hga_attend", "hga_attend_noalloc")
+           "hga_route", "hga_hot_rows", "hga_gather_host", "hga_attend", "hga_attend_noalloc")
 
 
 class HGAConfig(ctypes.Structure):
@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_route_chunks": (ctypes.c_int, [C, P, I32, P, P, I64, P, P, P]),
         "hga_route_groups": (ctypes.c_int, [C, P, I32, P, P, I64, P, P, P, P]),
         "hga_route": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, P]),
+        "hga_hot_rows": (ctypes.c_int, [C, ctypes.POINTER(I64)]),
+        "hga_gather_host": (ctypes.c_int, [C, P, P, I64, P, P, P, P, I32, P]),
         "hga_attend": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, SZ, P]),
         "hga_attend_noalloc": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P]),
     }
@@ -183,6 +185,22 @@ def hga_route(cfg, q, q_len: int, pos, chunk_sum, group_sum, n_alloc: int, chunk
                                     _ptr(chunk_sum), _ptr(group_sum), n_alloc, _ptr(chunk_idx),
                                     _ptr(chunk_score), _ptr(group_idx), _ptr(group_score),
                                     _stream(stream)), "hga_route")
+
+
+def hga_hot_rows(cfg) -> int:
+    """Rows per (sequence, KV head) of the host tier's device working buffers."""
+    out = ctypes.c_int64(0)
+    _check(load_library().hga_hot_rows(ctypes.byref(_cfg(cfg)), ctypes.byref(out)), "hga_hot_rows")
+    return out.value
+
+
+def hga_gather_host(cfg, k_host, v_host, n_alloc: int, pos, group_idx, k_work, v_work,
+                    refresh_window: bool = False, stream=None) -> None:
+    """Host tier: stage the routed groups (and window rows) from pinned host K/V."""
+    _check(load_library().hga_gather_host(ctypes.byref(_cfg(cfg)), _ptr(k_host), _ptr(v_host),
+                                          n_alloc, _ptr(pos), _ptr(group_idx), _ptr(k_work),
+                                          _ptr(v_work), 1 if refresh_window else 0,
+                                          _stream(stream)), "hga_gather_host")
 
 
 def hga_attend(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=None,

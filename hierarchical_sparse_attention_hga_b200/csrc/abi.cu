@@ -63,7 +63,8 @@ hga_status make_params(const hga_config* cfg, int64_t n_alloc, int32_t q_len, La
   if (c.dtype != HGA_F32 && c.dtype != HGA_BF16) return fail(HGA_ERR_INVALID_ARG, "dtype %d", c.dtype);
   if (c.out_dtype != HGA_F32 && c.out_dtype != HGA_BF16)
     return fail(HGA_ERR_INVALID_ARG, "out_dtype %d", c.out_dtype);
-  if (c.kv_loc != HGA_KV_DEVICE) return fail(HGA_ERR_UNSUPPORTED, "kv_loc %d", c.kv_loc);
+  if (c.kv_loc != HGA_KV_DEVICE && c.kv_loc != HGA_KV_HOST_PINNED)
+    return fail(HGA_ERR_INVALID_ARG, "kv_loc %d", c.kv_loc);
   if (c.heads_q % c.heads_kv) return fail(HGA_ERR_SHAPE, "heads_q %% heads_kv != 0");
   if (c.heads_q / c.heads_kv > 16) return fail(HGA_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
   if (c.head_dim != 64 && c.head_dim != 128) return fail(HGA_ERR_UNSUPPORTED, "head_dim %d", c.head_dim);
@@ -204,6 +205,38 @@ hga_status hga_route(const hga_config* cfg, const void* q, int32_t q_len, const 
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_route");
 }
 
+// The host tier runs bf16, D = 128 decode through the working buffers.
+static hga_status check_host_tier(const hga_config* cfg, const LayerParams& p) {
+  if (cfg->dtype != HGA_BF16 || p.D != 128 || p.g != 16 || p.kg > 1024 || p.q_len != 1)
+    return fail(HGA_ERR_UNSUPPORTED, "the host tier is built for bf16, head_dim 128 decode");
+  return HGA_OK;
+}
+
+hga_status hga_hot_rows(const hga_config* cfg, int64_t* rows) {
+  if (!rows) return fail(HGA_ERR_INVALID_ARG, "rows is NULL");
+  LayerParams p;
+  hga_status st = make_params(cfg, cfg ? cfg->chunk : 0, 1, &p);
+  if (st != HGA_OK) return st;
+  *rows = hot_rows(p);
+  return HGA_OK;
+}
+
+hga_status hga_gather_host(const hga_config* cfg, const void* k_host, const void* v_host,
+                           int64_t n_alloc, const int64_t* pos, const int32_t* group_idx,
+                           void* k_work, void* v_work, int32_t refresh_window, void* stream) {
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+  if (!k_host || !v_host || !pos || !group_idx || !k_work || !v_work)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_gather_host(p, k_host, v_host, pos, group_idx, k_work, v_work,
+                                     refresh_window ? 1 : 0, err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_gather_host");
+}
+
 hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const int64_t* pos,
                       const void* k, const void* v, int64_t n_alloc, const int32_t* group_idx,
                       void* out, float* lse, void* workspace, size_t workspace_bytes,
@@ -212,6 +245,14 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
   hga_status st = make_params(cfg, n_alloc, q_len, &p);
   if (st != HGA_OK) return st;
   if (!q || !pos || !k || !v || !group_idx || !out) return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (cfg->kv_loc == HGA_KV_HOST_PINNED) {
+    if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+    unsigned* err = nullptr;
+    if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+    cudaError_t e = launch_attend_decode_bf16(p, cfg->out_dtype, q, pos, k, v, group_idx, out, lse,
+                                              err, 1, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attend (host tier)");
+  }
   const size_t need = attend_workspace_bytes(p, cfg->dtype);
   if (need && (!workspace || workspace_bytes < need))
     return fail(HGA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);

@@ -326,7 +326,7 @@ cudaError_t launch_attend(const LayerParams& p, int dtype, int out_dtype, const 
                           unsigned* err, cudaStream_t s) {
   using bf = __nv_bfloat16;
   if (use_decode_fast(p, dtype))
-    return launch_attend_decode_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, err, s);
+    return launch_attend_decode_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, err, 0, s);
   if (prefill_tc_path(p, dtype))
     return launch_attend_prefill_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, err, s);
   if (dtype == 0)

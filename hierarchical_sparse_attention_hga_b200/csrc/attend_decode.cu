@@ -32,6 +32,7 @@
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.h"
+#include "topk.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -62,6 +63,8 @@ struct DecodeArgs {
   unsigned* err;
   int units_per_split;
   int nsplit;   // warp-splits per (sequence, KV head) = kWarps * cluster size
+  int hot;      // K/V are the host tier's device working buffers (see host_tier.cu)
+  int64_t rows; // rows per (sequence, KV head) of k / v: n_alloc, or the working-buffer rows
 };
 
 // Address of the 16-byte chunk `chunk` (0..15 over 128 dims) of row `row` in a
@@ -79,6 +82,7 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bars[kWarps][kStages];
   __shared__ int s_gl[1024];
+  __shared__ int s_slot[1024];  // input position of each kept routed group
   __shared__ int s_ng;
   __shared__ float s_ml[kWarps][16][2];   // per-warp (m, l) of each query head
   __shared__ float s_rml[8][16][2];       // rank 0: (m, l) pushed by each CTA of the cluster
@@ -114,12 +118,22 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   const int n_forced = su + lu;
   const int u_lo = split * a.units_per_split;
   const int u_cap = u_lo + a.units_per_split;
-  const int64_t row_base = static_cast<int64_t>(bh) * p.n_alloc;
+  const int64_t row_base = static_cast<int64_t>(bh) * a.rows;
+  // Row of unit u in k / v.  The device cache holds token t at row t.  The host
+  // tier's working buffer holds [sink chunks | ring of local+1 chunks (chunk c
+  // at slot c mod (local+1)) | routed groups in group_idx order].
   auto unit_token = [&](int u) -> int64_t {
     if (u < su) return static_cast<int64_t>(u) * kUnit;
     u -= su;
-    if (u < lu) return static_cast<int64_t>(u_first_local + u) * kUnit;
-    return static_cast<int64_t>(s_gl[u - lu]) * kUnit;
+    if (u < lu) {
+      const int unit = u_first_local + u;
+      if (!a.hot) return static_cast<int64_t>(unit) * kUnit;
+      const int c = unit / ng_per_c, gi = unit % ng_per_c;
+      return static_cast<int64_t>(p.sink + c % (p.local + 1)) * p.C + gi * kUnit;
+    }
+    u -= lu;
+    if (!a.hot) return static_cast<int64_t>(s_gl[u]) * kUnit;
+    return static_cast<int64_t>(p.sink + p.local + 1) * p.C + static_cast<int64_t>(s_slot[u]) * kUnit;
   };
   // Valid tokens in unit u (only the unit holding the query can be partial).
   auto unit_valid = [&](int u) -> int {
@@ -167,35 +181,17 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
 
   pdl_wait();
 
-  // Routed groups kept, in order: warp 0 validates and compacts them.  An id
-  // is kept when it names a group of a candidate chunk and exceeds every id
-  // kept before it (so the list is strictly ascending and has no duplicates).
+  // Routed groups kept, in order: warp 0 validates and compacts them (a group
+  // of a candidate chunk, strictly ascending; anything else is dropped and
+  // flagged).  The host tier's gather applies the same rule.
   if (warp == 0) {
     int n = 0;
     bool bad = false;
     if (ok) {
       const int32_t* gl = a.group_idx + static_cast<size_t>(bh) * p.kg;
-      int run_max = -1;
-      for (int base = 0; base < p.kg; base += 32) {
-        const int i = base + lane;
-        const int gid = i < p.kg ? gl[i] : -1;
-        const int c = gid >= 0 ? gid / p.Ng : -1;
-        const bool in_range = gid >= 0 && c >= p.sink && c < cur - p.local;
-        int incl = in_range ? gid : -1;  // inclusive prefix max over lanes
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int x = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl = max(incl, x);
-        }
-        int excl = __shfl_up_sync(0xffffffffu, incl, 1);
-        excl = max(lane == 0 ? -1 : excl, run_max);
-        const bool keep = in_range && gid > excl;
-        bad |= __any_sync(0xffffffffu, gid >= 0 && !keep);
-        const unsigned km = __ballot_sync(0xffffffffu, keep);
-        if (keep) s_gl[n + __popc(km & ((1u << lane) - 1u))] = gid;
-        n += __popc(km);
-        run_max = max(run_max, __shfl_sync(0xffffffffu, incl, 31));
-      }
+      n = warp_keep_ascending(
+          gl, p.kg, [&](int gid) { return gid / p.Ng >= p.sink && gid / p.Ng < cur - p.local; },
+          s_gl, &bad, s_slot);
     }
     if (lane == 0) {
       s_ng = n;
@@ -430,7 +426,7 @@ int cluster_size(const LayerParams& p) {
 template <typename TO>
 cudaError_t launch_t(const LayerParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                      const void* q, const int64_t* pos, const int32_t* group_idx, void* out,
-                     float* lse, unsigned* err, cudaStream_t s) {
+                     float* lse, unsigned* err, int hot, int64_t rows, cudaStream_t s) {
   const int cl = cluster_size(p);
   DecodeArgs<TO> a;
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -441,6 +437,8 @@ cudaError_t launch_t(const LayerParams& p, const CUtensorMap& tk, const CUtensor
   a.err = err;
   a.nsplit = cl * kWarps;
   a.units_per_split = (max_units(p) + a.nsplit - 1) / a.nsplit;
+  a.hot = hot;
+  a.rows = rows;
   cudaError_t e = ensure_smem<attend_decode_bf16_kernel<TO>>(kSmemBytes);
   if (e != cudaSuccess) return e;
   // A plain (non-programmatic) launch: measured faster here, because CTAs of
@@ -460,15 +458,16 @@ bool decode_fast_path(const LayerParams& p, int dtype) {
 cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const void* q,
                                       const int64_t* pos, const void* k, const void* v,
                                       const int32_t* group_idx, void* out, float* lse,
-                                      unsigned* err, cudaStream_t s) {
+                                      unsigned* err, int hot, cudaStream_t s) {
   CUtensorMap tk, tv;
-  const int64_t rows = static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc;
-  cudaError_t e = make_bf16_map(&tk, k, rows, kUnit);
-  if (e == cudaSuccess) e = make_bf16_map(&tv, v, rows, kUnit);
+  const int64_t rows = hot ? hot_rows(p) : p.n_alloc;
+  const int64_t all_rows = static_cast<int64_t>(p.B) * p.Hkv * rows;
+  cudaError_t e = make_bf16_map(&tk, k, all_rows, kUnit);
+  if (e == cudaSuccess) e = make_bf16_map(&tv, v, all_rows, kUnit);
   if (e != cudaSuccess) return e;
   return out_dtype == 0
-             ? launch_t<float>(p, tk, tv, q, pos, group_idx, out, lse, err, s)
-             : launch_t<__nv_bfloat16>(p, tk, tv, q, pos, group_idx, out, lse, err, s);
+             ? launch_t<float>(p, tk, tv, q, pos, group_idx, out, lse, err, hot, rows, s)
+             : launch_t<__nv_bfloat16>(p, tk, tv, q, pos, group_idx, out, lse, err, hot, rows, s);
 }
 
 }  // namespace hga

@@ -87,10 +87,21 @@ size_t attend_workspace_bytes(const LayerParams& p, int dtype);
 // The bf16, D = 128 decode kernel (TMA + mma.sync, in-cluster merge, no
 // workspace) applies to p.
 bool decode_fast_path(const LayerParams& p, int dtype);
+// hot != 0: k / v are the host tier's device working buffers (hot_rows(p)
+// rows per (sequence, KV head)) instead of the device cache.
 cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const void* q,
                                       const int64_t* pos, const void* k, const void* v,
                                       const int32_t* group_idx, void* out, float* lse,
-                                      unsigned* err, cudaStream_t s);
+                                      unsigned* err, int hot, cudaStream_t s);
+
+// Host tier: rows per (sequence, KV head) of the device working buffers:
+// sink chunks, a ring of local+1 chunks, and kg routed groups.
+__host__ __device__ inline int64_t hot_rows(const LayerParams& p) {
+  return static_cast<int64_t>(p.sink + p.local + 1) * p.C + static_cast<int64_t>(p.kg) * p.g;
+}
+cudaError_t launch_gather_host(const LayerParams& p, const void* k_host, const void* v_host,
+                               const int64_t* pos, const int32_t* group_idx, void* k_work,
+                               void* v_work, int refresh_window, unsigned* err, cudaStream_t s);
 
 // The bf16, D = 128 prefill kernel (64-query blocks on tcgen05 / TMEM) applies to p.
 bool prefill_tc_path(const LayerParams& p, int dtype);

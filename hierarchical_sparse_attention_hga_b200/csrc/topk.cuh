@@ -60,11 +60,12 @@ __device__ __forceinline__ int block_exclusive_scan(int v, TopkSmem& sm, int* to
 // Warp-cooperative compaction of an id list: keeps, in order, every id with
 // in_range(id) true that exceeds every id kept before it (so the output is
 // strictly ascending and free of duplicates).  Called by all 32 lanes of one
-// warp; writes out[0..count) and returns count in every lane; *bad is set when
-// a non-negative id was dropped.
+// warp; writes out[0..count) (and, if given, each kept id's input position to
+// out_slot) and returns count in every lane; *bad is set when a non-negative id
+// was dropped.
 template <typename InRange>
 __device__ int warp_keep_ascending(const int32_t* ids, int n, InRange in_range, int* out,
-                                   bool* bad) {
+                                   bool* bad, int* out_slot = nullptr) {
   const int lane = threadIdx.x & 31;
   int count = 0, run_max = -1;
   bool dropped = false;
@@ -83,7 +84,11 @@ __device__ int warp_keep_ascending(const int32_t* ids, int n, InRange in_range, 
     const bool keep = ok && id > excl;
     dropped |= __any_sync(0xffffffffu, id >= 0 && !keep);
     const unsigned km = __ballot_sync(0xffffffffu, keep);
-    if (keep) out[count + __popc(km & ((1u << lane) - 1u))] = id;
+    if (keep) {
+      const int at = count + __popc(km & ((1u << lane) - 1u));
+      out[at] = id;
+      if (out_slot) out_slot[at] = i;  // position of the kept id in the input list
+    }
     count += __popc(km);
     run_max = max(run_max, __shfl_sync(0xffffffffu, incl, 31));
   }

@@ -204,6 +204,40 @@ hga_status hga_route(const hga_config* cfg, const void* q, int32_t q_len, const 
                      float* group_score, void* stream);
 
 /*
+ * Host tier (HGA technical summary, "Architettura della Memoria": the hot tier
+ * in VRAM holds the chunk summaries and the always-visible windows, the cold
+ * tier in host RAM holds the whole K/V history; "Meccanismo Core", item 4: the
+ * selected groups' original K/V are fetched from host RAM into VRAM for the
+ * exact attention).
+ *
+ * With cfg->kv_loc == HGA_KV_HOST_PINNED the K/V cache [B, Hkv, n_alloc, D]
+ * lives in pinned, device-mapped host memory.  The GPU keeps per (sequence, KV
+ * head) a working buffer of hga_hot_rows() rows of D elements:
+ *   [sink chunks | ring of local+1 chunks, chunk c at slot c mod (local+1) |
+ *    kg routed groups, slot j holding entry j of group_idx]
+ * Built for bf16, head_dim 128 decode.  hga_build_summaries accepts the host
+ * cache as k (it reads it over the host link); hga_route* need no K/V.
+ */
+hga_status hga_hot_rows(const hga_config* cfg, int64_t* rows);
+
+/*
+ * Fills the working buffers for one decode step at pos (host tier): copies from
+ * the pinned host cache the routed groups of group_idx (as hga_route_groups
+ * or hga_route wrote it; the same groups hga_attend keeps) and the current
+ * chunk's rows up to pos; with refresh_window != 0 also the sink and local
+ * chunks (after a prefill, or whenever the window is stale: a decode loop that
+ * calls this at every consecutive position keeps it current; after positions
+ * are skipped, pass refresh_window).  The copy is a
+ * kernel reading host memory directly (zero-copy 16-byte loads over the host
+ * link); nothing is allocated.
+ *   k_host, v_host  pinned host [B, Hkv, n_alloc, 128] bf16
+ *   k_work, v_work  device [B, Hkv, hga_hot_rows(), 128] bf16 (caller-owned)
+ */
+hga_status hga_gather_host(const hga_config* cfg, const void* k_host, const void* v_host,
+                           int64_t n_alloc, const int64_t* pos, const int32_t* group_idx,
+                           void* k_work, void* v_work, int32_t refresh_window, void* stream);
+
+/*
  * Steps 4-5 - gather of the selected tokens' original K/V and exact softmax
  * attention over that bounded set (HGA technical summary, "Metodologia ->
  * Meccanismo Core", item 4 "Attenzione Esatta per Token"; "Contributi Chiave"
@@ -214,7 +248,9 @@ hga_status hga_route(const hga_config* cfg, const void* q, int32_t q_len, const 
  * and the g tokens of every group in its block's group_idx row.  No summary
  * value enters the output.
  *
- *   k, v       device [B, Hkv, n_alloc, D] (cfg->dtype)
+ *   k, v       device [B, Hkv, n_alloc, D] (cfg->dtype); with kv_loc ==
+ *              HGA_KV_HOST_PINNED, the device working buffers filled by
+ *              hga_gather_host (decode only)
  *   group_idx  device int32 [B, Hkv, nblk, kg] from step 3; entries must be
  *              groups of candidate chunks (checked on the device; a bad entry
  *              is skipped and flagged)

@@ -184,6 +184,20 @@ def run_hga(args, rank: int, world: int):
                     dtype=B.HGA_BF16 if wl.dtype == "bf16" else B.HGA_F32, out_dtype=B.HGA_F32)
     bh = wl.batch * wl.heads_kv
     nc, ng = n // wl.chunk, wl.chunk // wl.group
+    # Host tier: the whole K/V cache in pinned host memory; the GPU keeps the
+    # summaries and a working buffer (windows + the step's routed groups).
+    hot = wl.name.startswith("host_tier")
+    if hot:
+        layer.kv_loc = B.HGA_KV_HOST_PINNED
+        k_host, v_host = k.cpu().pin_memory(), v.cpu().pin_memory()
+        del k, v
+        torch.cuda.empty_cache()
+        rows = B.hga_hot_rows(layer)
+        k_work = torch.empty(bh, rows, wl.head_dim, dtype=torch.bfloat16, device=dev)
+        v_work = torch.empty_like(k_work)
+        k_src, v_src = k_host, v_host
+    else:
+        k_src, v_src = k, v
     cs = torch.empty(bh, nc, wl.head_dim, device=dev)
     gs = torch.empty(bh, nc, ng, wl.head_dim, device=dev)
     ci = torch.empty(bh, wl.topk_chunks, dtype=torch.int32, device=dev)
@@ -196,16 +210,24 @@ def run_hga(args, rank: int, world: int):
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
     # prefix summaries (setup, untimed): every row closed before the new token
-    B.hga_build_summaries(layer, k, n, 0, p, cs, gs, stream=sh)
+    B.hga_build_summaries(layer, k_src, n, 0, p, cs, gs, stream=sh)
+    if hot:  # fill the working buffer's windows once
+        B.hga_route(layer, q, 1, pos, cs, gs, n, ci, gi, stream=sh)
+        B.hga_gather_host(layer, k_host, v_host, n, pos, gi, k_work, v_work, refresh_window=True,
+                          stream=sh)
 
     parts = {
-        "summaries": lambda st: B.hga_build_summaries(layer, k, n, p, p + 1, cs, gs, stream=st),
+        "summaries": lambda st: B.hga_build_summaries(layer, k_src, n, p, p + 1, cs, gs, stream=st),
         "route": lambda st: B.hga_route(layer, q, 1, pos, cs, gs, n, ci, gi, stream=st),
-        "attend": lambda st: B.hga_attend(layer, q, 1, pos, k, v, n, gi, out, lse, ws, wsb,
+        "attend": lambda st: B.hga_attend(layer, q, 1, pos, k_work if hot else k_src,
+                                          v_work if hot else v_src, n, gi, out, lse, ws, wsb,
                                           stream=st),
         "route_chunks": lambda st: B.hga_route_chunks(layer, q, 1, pos, cs, n, ci, stream=st),
         "route_groups": lambda st: B.hga_route_groups(layer, q, 1, pos, gs, n, ci, gi, stream=st),
     }
+    if hot:
+        parts["gather"] = lambda st: B.hga_gather_host(layer, k_host, v_host, n, pos, gi, k_work,
+                                                       v_work, stream=st)
 
     side = torch.cuda.Stream()
 
@@ -223,8 +245,12 @@ def run_hga(args, rank: int, world: int):
             main.wait_stream(side)
         return step
 
-    step = make_step(("route", "attend"))
-    step4 = make_step(("route_chunks", "route_groups", "attend"))
+    if hot:
+        step = make_step(("route", "gather", "attend"))
+        step4 = make_step(("route_chunks", "route_groups", "gather", "attend"))
+    else:
+        step = make_step(("route", "attend"))
+        step4 = make_step(("route_chunks", "route_groups", "attend"))
 
     # eager warm-up, then one CUDA graph for the whole step and one per call
     for _ in range(max(1, args.warmup)):
@@ -290,9 +316,9 @@ def run_hga(args, rank: int, world: int):
     # ---- e2e: host (pinned) q and new K/V rows in, output back, every step
     q_host = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).pin_memory() \
         if wl.dtype == "bf16" else torch.from_numpy(x["q"]).pin_memory()
-    kv_new = torch.empty(2, wl.batch, wl.heads_kv, wl.head_dim, dtype=k.dtype).pin_memory()
-    kv_new[0].copy_(k[:, :, p].cpu())
-    kv_new[1].copy_(v[:, :, p].cpu())
+    kv_new = torch.empty(2, wl.batch, wl.heads_kv, wl.head_dim, dtype=torch.bfloat16).pin_memory()
+    kv_new[0].copy_(k_src[:, :, p].cpu())
+    kv_new[1].copy_(v_src[:, :, p].cpu())
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     qv = q.view(torch.int16) if wl.dtype == "bf16" else q
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -301,8 +327,12 @@ def run_hga(args, rank: int, world: int):
         flush.zero_()
         e0.record(stream)
         qv.copy_(q_host, non_blocking=True)
-        k[:, :, p].copy_(kv_new[0], non_blocking=True)
-        v[:, :, p].copy_(kv_new[1], non_blocking=True)
+        if hot:  # the new token's K/V goes into the host cache, a host-side write
+            k_host[:, :, p].copy_(kv_new[0])
+            v_host[:, :, p].copy_(kv_new[1])
+        else:
+            k_src[:, :, p].copy_(kv_new[0], non_blocking=True)
+            v_src[:, :, p].copy_(kv_new[1], non_blocking=True)
         graphs["step"].replay()
         out_host.copy_(out, non_blocking=True)
         e1.record(stream)
@@ -314,7 +344,7 @@ def run_hga(args, rank: int, world: int):
         t = torch.tensor([ms_e2e], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
-    h2d = q_host.numel() * q_host.element_size() + kv_new.numel() * kv_new.element_size()
+    h2d = q_host.numel() * q_host.element_size() + (0 if hot else kv_new.numel() * kv_new.element_size())
     d2h = out_host.numel() * out_host.element_size()
 
     nb = step_bytes(wl)
@@ -324,7 +354,7 @@ def run_hga(args, rank: int, world: int):
     achieved = nb[kern] / (ms[kern] * 1e-3) / 1e9
     total_bytes = nb["summaries"] + nb["route"] + nb["attend"]
     nsplit_combine = 1 if wsb > 0 else 0
-    launches_per_step = 1 + 1 + 1 + nsplit_combine   # summaries, route, attend (+ merge)
+    launches_per_step = 1 + 1 + 1 + nsplit_combine + (1 if hot else 0)  # summaries, route, (gather,) attend
     tokens = wl.batch * world
     line = {
         "metric": METRIC,
@@ -337,7 +367,10 @@ def run_hga(args, rank: int, world: int):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16 K/V, fp32 accumulation" if wl.dtype == "bf16" else "f32",
-        "data": "synthetic (seeded N(0,1) q/k/v; 2 needle chunks per KV head)",
+        "data": "synthetic (seeded N(0,1) q/k/v" +
+                (f"; {wl.needles} needle chunks per KV head" if wl.needles else "") +
+                (f"; log-normal key norms, sigma {wl.lognormal_sigma}" if wl.lognormal_sigma else "") +
+                ("; K/V in pinned host memory" if hot else "") + ")",
         "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": n,
                    "heads_q": wl.heads_q, "heads_kv": wl.heads_kv, "head_dim": wl.head_dim,
                    "chunk": wl.chunk, "group": wl.group, "sink": wl.sink, "local": wl.local,
@@ -356,10 +389,36 @@ def run_hga(args, rank: int, world: int):
         "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "decode tokens/s (one attention layer)",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
+        "host_link": host_link_report(wl, ms, dev) if hot else None,
         "timing": "CUDA graph of the step replayed per timed step; CUDA events on the launch stream",
         "clocks": clk.report(),
     }
     return line, wl, seed, x
+
+
+def host_link_report(wl: S.Workload, ms: dict, dev) -> dict:
+    """Host-tier traffic over the host link per step, against a pinned H2D copy probe."""
+    import torch
+    cur = (wl.context - 1) // wl.chunk
+    cur_rows = wl.context - 1 - cur * wl.chunk + 1
+    row = wl.head_dim * 2 * 2  # K and V, bf16
+    units = wl.batch * wl.heads_kv
+    routed = units * wl.topk_groups * wl.group * row
+    window = units * cur_rows * row
+    src = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = 0.0
+    for _ in range(5):
+        e0.record()
+        dst.copy_(src, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        best = max(best, src.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    gbs = (routed + window) / (ms["gather"] * 1e-3) / 1e9
+    return {"bytes_per_step": routed + window, "routed_bytes": routed, "window_bytes": window,
+            "gather_us": ms["gather"] * 1e3, "achieved_gbs": gbs, "h2d_copy_probe_gbs": best,
+            "frac_of_probe": gbs / best}
 
 
 # ------------------------------------------------------------------ prefill

@@ -50,6 +50,35 @@ def parse():
     return ap.parse_args()
 
 
+def profile_traffic(kernel: str, wl: S.Workload):
+    """DRAM bytes per launch of `kernel` from a committed ncu capture (profiles/*.md).
+
+    The capture may be of a smaller case of the same workload; its bytes are
+    scaled by the units processed (the line's `scale`: batch, or batch*context).
+    Returns None when no capture covers the kernel or when its source file has
+    changed since the counters were taken.
+    """
+    import glob
+    import hashlib
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(path):
+            if not line.startswith("traffic:"):
+                continue
+            kv = dict(x.split("=", 1) for x in line.split()[1:])
+            if kv.get("kernel") != kernel or kv.get("workload") != wl.name:
+                continue
+            src = os.path.join(ROOT, kv["source"])
+            if not os.path.exists(src):
+                return None
+            if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != kv["sha256_16"]:
+                return None  # the kernel changed since the counters were taken
+            ratio = wl.batch / int(kv["batch"])
+            if kv.get("scale") == "batch*context":
+                ratio *= wl.context / int(kv["context"])
+            return int(float(kv["dram_bytes"]) * ratio)
+    return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -385,7 +414,9 @@ def run_hga(args, rank: int, world: int):
         "step_hbm_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
         "roofline": {"kernel": kern, "bound": "hbm", "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": None, "algorithmic_bytes": nb[kern]},
+                     "traffic": profile_traffic("route_chunks_kernel" if kern == "route" else
+                                                "attend_decode_bf16_kernel", wl),
+                     "algorithmic_bytes": nb[kern]},
         "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "decode tokens/s (one attention layer)",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -568,7 +599,8 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
         "attend_flops": flops,
         "roofline": {"kernel": "attend", "bound": "tensor", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": None, "algorithmic_flops": flops},
+                     "traffic": profile_traffic("attend_prefill_kernel", wl),
+                     "algorithmic_flops": flops},
         "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "prefill tokens/s (one attention layer)",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": q_host.numel() * 2,
                 "d2h_bytes_per_step": out_host.numel() * 2},

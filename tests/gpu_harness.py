@@ -41,8 +41,9 @@ def to_device(x: np.ndarray, dtype: str):
 
 
 def run_gpu(wl: S.Workload, x: dict, q_len: int | None = None, out_dtype: int = B.HGA_F32,
-            pos=None, summaries_range=None, check_status: bool = True) -> dict:
-    """Runs build_summaries -> route_chunks -> route_groups -> attend; returns numpy results."""
+            pos=None, summaries_range=None, check_status: bool = True, fused: bool = False) -> dict:
+    """Runs build_summaries -> route (two calls, or hga_route when fused) -> attend;
+    returns numpy results."""
     import torch
     q_len = x["q"].shape[2] if q_len is None else q_len
     layer = layer_of(wl, out_dtype)
@@ -68,8 +69,12 @@ def run_gpu(wl: S.Workload, x: dict, q_len: int | None = None, out_dtype: int = 
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     t0, t1 = (0, n) if summaries_range is None else summaries_range
     B.hga_build_summaries(layer, k, n, t0, t1, chunk_sum, group_sum)
-    B.hga_route_chunks(layer, q, q_len, pos_t, chunk_sum, n, chunk_idx, chunk_score)
-    B.hga_route_groups(layer, q, q_len, pos_t, group_sum, n, chunk_idx, group_idx, group_score)
+    if fused:
+        B.hga_route(layer, q, q_len, pos_t, chunk_sum, group_sum, n, chunk_idx, group_idx,
+                    chunk_score, group_score)
+    else:
+        B.hga_route_chunks(layer, q, q_len, pos_t, chunk_sum, n, chunk_idx, chunk_score)
+        B.hga_route_groups(layer, q, q_len, pos_t, group_sum, n, chunk_idx, group_idx, group_score)
     B.hga_attend(layer, q, q_len, pos_t, k, v, n, group_idx, out, lse, ws, ws_bytes)
     torch.cuda.synchronize()
     status = B.hga_device_status()
@@ -216,3 +221,21 @@ def compare_prefill_blocks(wl: S.Workload, x: dict, res: dict, b: int, h: int, b
                 err = float(np.max(np.abs(got - o)))
                 assert err <= tol, f"prefill out b{b} h{h} blk{blk} row{i} head{hh}: {err:.3e}"
                 assert abs(res["lse"][b, h * g + hh, r0 + i] - lse) <= max(tol, 1e-4)
+
+
+def check_properties(wl: S.Workload, res: dict):
+    """Size-independent properties of every (b, h, block): selections ascending,
+    unique, -1 padded, inside the candidate ranges, groups inside selected chunks,
+    outputs finite."""
+    ng = wl.chunk // wl.group
+    ci, gi = res["chunk_idx"], res["group_idx"]
+    assert np.isfinite(res["out"]).all() and np.isfinite(res["lse"]).all()
+    for idx in np.ndindex(ci.shape[:3]):
+        c = ci[idx]
+        valid = c[c >= 0]
+        assert (np.diff(valid) > 0).all() and (c[len(valid):] == -1).all()
+        assert (valid >= wl.sink).all()
+        g = gi[idx]
+        gv = g[g >= 0]
+        assert (np.diff(gv) > 0).all() and (g[len(gv):] == -1).all()
+        assert set((gv // ng).tolist()) <= set(valid.tolist())

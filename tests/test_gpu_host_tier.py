@@ -113,3 +113,17 @@ def test_host_tier_rejects_unsupported_shapes():
     with pytest.raises(B.HGAError) as e:
         B.hga_gather_host(lay, 16, 16, 1024, 16, 16, 16, 16)
     assert e.value.status == 3
+
+
+def test_host_tier_decode_128k_batch8_full_size():
+    """The host-tier workload at full size: 131072 tokens, batch 8, K/V pinned on the host."""
+    wl = S.workload("host_tier_decode_128k")
+    x = S.make_inputs(wl, S.seed_for(3))
+    r = Runner(wl, x)
+    r.summaries(0, wl.context, host=True)
+    out, lse, gi = r.step(x["pos"], host=True, refresh=True)
+    res = dict(chunk_idx=r.ci.cpu().numpy().reshape(8, 8, 1, -1), group_idx=gi.reshape(8, 8, 1, -1),
+               out=out, lse=lse)
+    assert np.isfinite(out).all()
+    for b, h in ((0, 0), (5, 4), (7, 7)):
+        compare_head(wl, x, res, b, h)

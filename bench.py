@@ -177,6 +177,60 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+# ------------------------------------------------------------ ranks (N > 1)
+
+class Ranks:
+    """Cross-rank plumbing of the timed region (one process per GPU).
+
+    Every rank takes the same steps in the same order: a barrier before and
+    after the timed steps, and a MAX reduction of each time it reports.  With
+    one rank every call is a no-op.  The data path itself has no collective:
+    the ranks decode independent sequences (weak scaling).
+    """
+
+    def __init__(self, world: int, device):
+        self.world = world
+        self.device = device
+        self.dist = None
+        if world > 1:
+            import torch.distributed as dist
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist:
+            self.dist.barrier()
+
+    def max(self, value: float) -> float:
+        if not self.dist:
+            return value
+        import torch
+        t = torch.tensor([value], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def init_ranks(backend: str) -> tuple[int, int]:
+    """Joins the process group torchrun describes in the environment."""
+    import datetime
+
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if world > 1:
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Input seed of one rank: each rank's sequences are distinct."""
+    return S.seed_for(list(S.WORKLOADS).index(workload)) + 7919 * rank
+
+
+def job_rate(units_per_rank: float, world: int, ms_step: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the max-over-ranks time."""
+    return units_per_rank * world / (ms_step * 1e-3)
+
+
 # ------------------------------------------------------------------ CUDA arm
 
 def run_hga(args, rank: int, world: int):
@@ -195,7 +249,7 @@ def run_hga(args, rank: int, world: int):
     if wl.prefill:
         return run_prefill(args, rank, world, wl)
     dev = torch.device("cuda")
-    seed = S.seed_for(list(S.WORKLOADS).index(args.workload)) + 7919 * rank
+    seed = rank_seed(args.workload, rank)
     x = S.make_inputs(wl, seed)
     n = wl.context
     p = n - 1
@@ -307,25 +361,20 @@ def run_hga(args, rank: int, world: int):
     for _ in range(args.warmup):
         flush.zero_()
         graphs["step"].replay()
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    ranks = Ranks(world, dev)
+    torch.cuda.synchronize()
+    ranks.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         starts, ends = timed(graphs["step"], args.steps)
         torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
+    ranks.barrier()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     ms_step = sum(step_ms) / len(step_ms)
     a4, b4 = timed(graphs["step4"], min(args.steps, 200))
     torch.cuda.synchronize()
     ms_step4 = sum(x.elapsed_time(y) for x, y in zip(a4, b4)) / len(a4)
-    if dist:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = ranks.max(ms_step)
     assert B.hga_device_status(sh) == 0
     # timing floor: an empty graph-sized launch measured the same way
     g_floor = torch.cuda.CUDAGraph()
@@ -369,10 +418,7 @@ def run_hga(args, rank: int, world: int):
         if i >= args.warmup:
             e2e.append(e0.elapsed_time(e1))
     ms_e2e = sum(e2e) / len(e2e)
-    if dist:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = ranks.max(ms_e2e)
     h2d = q_host.numel() * q_host.element_size() + (0 if hot else kv_new.numel() * kv_new.element_size())
     d2h = out_host.numel() * out_host.element_size()
 
@@ -384,10 +430,10 @@ def run_hga(args, rank: int, world: int):
     total_bytes = nb["summaries"] + nb["route"] + nb["attend"]
     nsplit_combine = 1 if wsb > 0 else 0
     launches_per_step = 1 + 1 + 1 + nsplit_combine + (1 if hot else 0)  # summaries, route, (gather,) attend
-    tokens = wl.batch * world
+    tokens = wl.batch  # per rank
     line = {
         "metric": METRIC,
-        "value": tokens / (ms_step * 1e-3),
+        "value": job_rate(tokens, world, ms_step),
         "unit": "decode tokens/s (one attention layer)",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step,
@@ -417,7 +463,7 @@ def run_hga(args, rank: int, world: int):
                      "traffic": profile_traffic("route_chunks_kernel" if kern == "route" else
                                                 "attend_decode_bf16_kernel", wl),
                      "algorithmic_bytes": nb[kern]},
-        "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "decode tokens/s (one attention layer)",
+        "e2e": {"value": job_rate(tokens, world, ms_e2e), "unit": "decode tokens/s (one attention layer)",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "host_link": host_link_report(wl, ms, dev) if hot else None,
@@ -488,7 +534,7 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
     from hierarchical_sparse_attention_hga_b200 import binding as B
 
     dev = torch.device("cuda")
-    seed = S.seed_for(list(S.WORKLOADS).index(args.workload)) + 7919 * rank
+    seed = rank_seed(args.workload, rank)
     x = S.make_inputs(wl, seed)
     n = wl.context
     nblk = n // wl.chunk
@@ -546,16 +592,13 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
         torch.cuda.synchronize()
         return sum(a_.elapsed_time(b_) for a_, b_ in ev) / iters
 
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    ranks = Ranks(world, dev)
+    ranks.barrier()
+    torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         ms_step = timed(graphs["step"], args.steps)
-    if dist:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ranks.barrier()
+    ms_step = ranks.max(ms_step)
     ms = {name: timed(graphs[name], max(3, min(args.steps, 20))) for name in parts}
     assert B.hga_device_status() == 0
 
@@ -574,15 +617,15 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
         e1.synchronize()
         if i:
             e2e.append(e0.elapsed_time(e1))
-    ms_e2e = sum(e2e) / len(e2e)
+    ms_e2e = ranks.max(sum(e2e) / len(e2e))
 
     flops = prefill_flops(wl)
     peak, peak_kind = tensor_peak()
     achieved = flops / (ms["attend"] * 1e-3) / 1e12
-    tokens = wl.batch * n * world
+    tokens = wl.batch * n  # per rank
     line = {
         "metric": METRIC + " (prefill)",
-        "value": tokens / (ms_step * 1e-3),
+        "value": job_rate(tokens, world, ms_step),
         "unit": "prefill tokens/s (one attention layer)",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "attn_us_per_layer": ms_step * 1e3,
@@ -601,7 +644,7 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
                      "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": profile_traffic("attend_prefill_kernel", wl),
                      "algorithmic_flops": flops},
-        "e2e": {"value": tokens / (ms_e2e * 1e-3), "unit": "prefill tokens/s (one attention layer)",
+        "e2e": {"value": job_rate(tokens, world, ms_e2e), "unit": "prefill tokens/s (one attention layer)",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": q_host.numel() * 2,
                 "d2h_bytes_per_step": out_host.numel() * 2},
         "gpu_launches": 3 * args.steps,
@@ -717,25 +760,36 @@ def oracle_decode_rate(wl: S.Workload, seed: int, budget_s: float, x=None):
 
 
 def run_reference(args, rank: int):
+    """The oracle arm: the float64 CPU oracle timed on the host cores, rank 0 only.
+
+    Each step is a bounded sample of the same workload (sized so the whole
+    run stays within a few minutes), extrapolated to the arm's unit.
+    """
     if rank != 0:
         return None
     wl = S.workload(args.workload)
     if args.batch:
         wl = wl.with_(batch=args.batch)
-    seed = S.seed_for(list(S.WORKLOADS).index(args.workload))
+    if args.context:
+        wl = wl.with_(context=args.context)
+    seed = rank_seed(args.workload, 0)
+    rate_fn = oracle_prefill_rate if wl.prefill else oracle_decode_rate
     rates = []
-    # each step is a bounded sample sized so that the whole run stays within ~3 minutes
     budget = max(0.02, min(args.cpu_seconds / 10, 150.0 / (args.warmup + args.steps)))
     for i in range(args.warmup + args.steps):
-        r, sample, cores = oracle_decode_rate(wl, seed, budget_s=budget)
+        r, sample, cores = rate_fn(wl, seed, budget_s=budget)
         if i >= args.warmup:
             rates.append(r)
     value = statistics.median(rates)
-    unit = "decode tokens/s (one attention layer)"
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+    kind = "prefill" if wl.prefill else "decode"
+    unit = f"{kind} tokens/s (one attention layer)"
+    tokens_per_step = wl.batch * (wl.context if wl.prefill else 1)
+    return {"impl": "reference", "metric": METRIC + (" (prefill)" if wl.prefill else ""),
+            "value": value, "unit": unit,
             "n_gpus": args.gpus, "steps": len(rates), "warmup": args.warmup,
-            "ms_per_step": wl.batch / value * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, same generator)",
+            "ms_per_step": tokens_per_step / value * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, same generator)",
             "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": wl.context},
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                              "sample": sample},
@@ -752,12 +806,9 @@ def main():
             print(json.dumps(line))
         return
     if world > 1:
-        import datetime
-
         import torch
-        import torch.distributed as dist
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        rank, world = init_ranks("nccl")
     line, wl, seed, x = run_hga(args, rank, world)
     if rank == 0:
         if not args.no_cpu_baseline:

@@ -81,6 +81,15 @@ cudaError_t launch_route(const LayerParams& p, int dtype, const void* q, const i
                          float* chunk_score, int32_t* group_idx, float* group_score,
                          unsigned* err, cudaStream_t s);
 
+// Prefill routing, several consecutive query blocks per CTA (level 1, level 2
+// from chunk_idx, or both in one launch); applies to p when prefill_route_path.
+bool prefill_route_path(const LayerParams& p, int dtype);
+cudaError_t launch_route_prefill(const LayerParams& p, int dtype, bool level1, bool level2,
+                                 const void* q, const int64_t* pos, const float* chunk_sum,
+                                 const float* group_sum, int32_t* chunk_idx, float* chunk_score,
+                                 int32_t* group_idx, float* group_score, unsigned* err,
+                                 cudaStream_t s);
+
 // Workspace bytes of launch_attend for p (0 when the launch needs none).
 size_t attend_workspace_bytes(const LayerParams& p, int dtype);
 

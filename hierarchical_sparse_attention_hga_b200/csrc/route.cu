@@ -119,13 +119,6 @@ __host__ __device__ inline RouteSmem route_smem(const LayerParams& p, int cl, bo
 }
 
 // One cluster of `cl` CTAs per (sequence, KV head, block): CTA r scores the
-// r-th slice of the candidates into its own shared memory; after a cluster
-// barrier, CTA 0 gathers every slice through distributed shared memory and
-// runs the top-k.  With cl == 1 this is a plain single-CTA scan.
-// With FUSE, CTA rank 0 continues into level 2 (the work of route_groups_kernel)
-// with the selected chunks still in shared memory; results are identical to the
-// two separate launches.
-// One cluster of `cl` CTAs per (sequence, KV head, block): CTA r scores the
 // r-th slice of the candidates and selects that slice's top-kc, then pushes
 // those (score, index) pairs into CTA 0's shared memory (distributed shared
 // memory stores).  CTA 0 takes the top-kc of the pushed pairs: the global
@@ -366,6 +359,9 @@ cudaError_t launch_route_chunks(const LayerParams& p, int dtype, const void* q, 
                                 const float* chunk_sum, int32_t* chunk_idx, float* chunk_score,
                                 unsigned* err, cudaStream_t s) {
   using bf = __nv_bfloat16;
+  if (prefill_route_path(p, dtype))
+    return launch_route_prefill(p, dtype, true, false, q, pos, chunk_sum, nullptr, chunk_idx,
+                                chunk_score, nullptr, nullptr, err, s);
   if (dtype == 0)
     return p.D == 64 ? launch_route_chunks_t<float, 64, false>(p, q, pos, chunk_sum, nullptr, chunk_idx, chunk_score, nullptr, nullptr, err, s)
                      : launch_route_chunks_t<float, 128, false>(p, q, pos, chunk_sum, nullptr, chunk_idx, chunk_score, nullptr, nullptr, err, s);
@@ -378,6 +374,9 @@ cudaError_t launch_route(const LayerParams& p, int dtype, const void* q, const i
                          float* chunk_score, int32_t* group_idx, float* group_score,
                          unsigned* err, cudaStream_t s) {
   using bf = __nv_bfloat16;
+  if (prefill_route_path(p, dtype))
+    return launch_route_prefill(p, dtype, true, true, q, pos, chunk_sum, group_sum, chunk_idx,
+                                chunk_score, group_idx, group_score, err, s);
   if (dtype == 0)
     return p.D == 64 ? launch_route_chunks_t<float, 64, true>(p, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx, group_score, err, s)
                      : launch_route_chunks_t<float, 128, true>(p, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx, group_score, err, s);
@@ -389,6 +388,10 @@ cudaError_t launch_route_groups(const LayerParams& p, int dtype, const void* q, 
                                 const float* group_sum, const int32_t* chunk_idx,
                                 int32_t* group_idx, float* group_score, unsigned* err,
                                 cudaStream_t s) {
+  if (prefill_route_path(p, dtype))
+    return launch_route_prefill(p, dtype, false, true, q, pos, nullptr, group_sum,
+                                const_cast<int32_t*>(chunk_idx), nullptr, group_idx, group_score,
+                                err, s);
   if (dtype == 0)
     return p.D == 64 ? launch_route_groups_t<float, 64>(p, q, pos, group_sum, chunk_idx, group_idx, group_score, err, s)
                      : launch_route_groups_t<float, 128>(p, q, pos, group_sum, chunk_idx, group_idx, group_score, err, s);

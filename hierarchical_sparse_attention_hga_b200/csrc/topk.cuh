@@ -224,3 +224,106 @@ __device__ int block_topk(const float* sc, int n, int k, int* sel, TopkSmem& sm)
 }
 
 }  // namespace hga
+
+namespace hga {
+
+// Per-warp scratch of warp_topk: up to kWarpTopkList (key, index) survivors.
+constexpr int kWarpTopkList = 64;
+
+// Warp-collective top-k of sc[0..n) (larger score first, equal scores to the
+// lower index); writes the chosen indices in ascending order to out[0..) and
+// returns their count, min(n, k), in every lane.  lst_key / lst_idx are this
+// warp's kWarpTopkList-entry scratch.
+//
+// For k <= 32 the k-th largest of the 32 lanes' maxima is a lower bound on the
+// k-th largest score (those k maxima come from k different scores), so only
+// scores at or above it can be chosen; they are usually few and get exact
+// ranks by pairwise comparison.  Otherwise (or if too many survive) a
+// most-significant-bit-first bisection finds the k-th largest key exactly.
+__device__ __forceinline__ int warp_topk(const float* sc, int n, int k, int* out,
+                                         unsigned* lst_key, int* lst_idx) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  if (k <= 0) return 0;
+  if (n <= k) {
+    for (int i = lane; i < n; i += 32) out[i] = i;
+    __syncwarp();
+    return max(n, 0);
+  }
+  unsigned thr = 0;
+  if (k <= 32) {
+    unsigned m = 0;
+    for (int i = lane; i < n; i += 32) m = max(m, order_key(sc[i]));
+    // bitonic sort of the lane maxima, descending across lanes
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const unsigned o = __shfl_xor_sync(0xffffffffu, m, stride);
+        const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+        m = keep_max ? max(m, o) : min(m, o);
+      }
+    }
+    thr = __shfl_sync(0xffffffffu, m, k - 1);
+  }
+  // survivors (key >= thr), compacted in index order
+  int cnt = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const unsigned key = i < n ? order_key(sc[i]) : 0u;
+    const bool s = i < n && key >= thr;
+    const unsigned bal = __ballot_sync(0xffffffffu, s);
+    const int at = cnt + __popc(bal & lt);
+    if (s && at < kWarpTopkList) {
+      lst_key[at] = key;
+      lst_idx[at] = i;
+    }
+    cnt += __popc(bal);
+  }
+  __syncwarp();
+  if (cnt <= kWarpTopkList) {
+    const bool h0 = lane < cnt, h1 = lane + 32 < cnt;
+    const unsigned k0 = h0 ? lst_key[lane] : 0u, k1 = h1 ? lst_key[lane + 32] : 0u;
+    const int i0 = h0 ? lst_idx[lane] : 0, i1 = h1 ? lst_idx[lane + 32] : 0;
+    int r0 = 0, r1 = 0;  // how many survivors come before this one
+    for (int j = 0; j < cnt; ++j) {
+      const unsigned kj = lst_key[j];
+      const int ij = lst_idx[j];
+      r0 += (kj > k0 || (kj == k0 && ij < i0)) ? 1 : 0;
+      r1 += (kj > k1 || (kj == k1 && ij < i1)) ? 1 : 0;
+    }
+    const bool s0 = h0 && r0 < k, s1 = h1 && r1 < k;
+    const unsigned b0 = __ballot_sync(0xffffffffu, s0), b1 = __ballot_sync(0xffffffffu, s1);
+    if (s0) out[__popc(b0 & lt)] = i0;
+    if (s1) out[__popc(b0) + __popc(b1 & lt)] = i1;
+    __syncwarp();
+    return __popc(b0) + __popc(b1);
+  }
+  // exact k-th largest key t: the largest t with #(key >= t) >= k
+  unsigned t = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const unsigned cand = t | (1u << bit);
+    unsigned c = 0;
+    for (int i = lane; i < n; i += 32) c += order_key(sc[i]) >= cand ? 1u : 0u;
+    if (__reduce_add_sync(0xffffffffu, c) >= static_cast<unsigned>(k)) t = cand;
+  }
+  unsigned gt = 0;
+  for (int i = lane; i < n; i += 32) gt += order_key(sc[i]) > t ? 1u : 0u;
+  const int ties = k - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+  int w = 0, seen = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const unsigned key = i < n ? order_key(sc[i]) : 0u;
+    const bool eq = i < n && key == t;
+    const unsigned beq = __ballot_sync(0xffffffffu, eq);
+    const bool s = (i < n && key > t) || (eq && seen + __popc(beq & lt) < ties);
+    const unsigned bs = __ballot_sync(0xffffffffu, s);
+    if (s) out[w + __popc(bs & lt)] = i;
+    w += __popc(bs);
+    seen += __popc(beq);
+  }
+  __syncwarp();
+  return k;
+}
+
+}  // namespace hga

@@ -266,6 +266,20 @@ def test_prefill_tensor_core_path_small(heads_q, heads_kv, out_dtype):
         compare_head(wl, x, res, 0, h)
 
 
+def test_prefill_suffix_with_ragged_block_count_and_positions():
+    """A 13-block prompt continuing a cache (queries start mid-cache), two sequences
+    at different positions: the router's blocks-per-CTA grouping has a ragged tail."""
+    wl = S.workload("llama3_8b_prefill_64k", batch=2, context=4096, heads_q=8, heads_kv=2,
+                    topk_chunks=8, topk_groups=16)
+    q_len = 13 * wl.chunk
+    x = S.make_inputs(wl, 25, q_len=q_len)
+    x["pos"] = np.array([4095, 1535], dtype=np.int64)
+    res = run_gpu(wl, x, q_len=q_len)
+    for b in range(2):
+        for h in range(2):
+            compare_prefill_blocks(wl, x, res, b, h, blocks=range(13), rows=(0, 17, 63))
+
+
 def test_prefill_tensor_core_path_8k_sampled_blocks():
     """Llama-3-8B-shaped prefill at 8K context: many KV tiles per block, all workload k values."""
     wl = S.workload("llama3_8b_prefill_64k", context=8192)

@@ -62,6 +62,20 @@ cudaError_t ensure_smem(size_t bytes) {
   return e;
 }
 
+// SMs of the current device (cached per device; 148 if the query fails).
+inline int device_sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = cache[dev].load();
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev].store(n);
+  }
+  return n;
+}
+
 // dtype: 0 = float32, 1 = bfloat16 (hga_dtype values).
 cudaError_t launch_summaries(const LayerParams& p, int dtype, const void* k, int64_t t_begin,
                              int64_t t_end, float* chunk_sum, float* group_sum, cudaStream_t s);
@@ -89,6 +103,14 @@ cudaError_t launch_route_prefill(const LayerParams& p, int dtype, bool level1, b
                                  const float* group_sum, int32_t* chunk_idx, float* chunk_score,
                                  int32_t* group_idx, float* group_score, unsigned* err,
                                  cudaStream_t s);
+
+// Decode routing, one cluster of small CTAs per (sequence, KV head); same modes.
+bool decode_route_path(const LayerParams& p);
+cudaError_t launch_route_decode(const LayerParams& p, int dtype, bool level1, bool level2,
+                                const void* q, const int64_t* pos, const float* chunk_sum,
+                                const float* group_sum, int32_t* chunk_idx, float* chunk_score,
+                                int32_t* group_idx, float* group_score, unsigned* err,
+                                cudaStream_t s);
 
 // Workspace bytes of launch_attend for p (0 when the launch needs none).
 size_t attend_workspace_bytes(const LayerParams& p, int dtype);

@@ -362,6 +362,9 @@ cudaError_t launch_route_chunks(const LayerParams& p, int dtype, const void* q, 
   if (prefill_route_path(p, dtype))
     return launch_route_prefill(p, dtype, true, false, q, pos, chunk_sum, nullptr, chunk_idx,
                                 chunk_score, nullptr, nullptr, err, s);
+  if (decode_route_path(p))
+    return launch_route_decode(p, dtype, true, false, q, pos, chunk_sum, nullptr, chunk_idx,
+                               chunk_score, nullptr, nullptr, err, s);
   if (dtype == 0)
     return p.D == 64 ? launch_route_chunks_t<float, 64, false>(p, q, pos, chunk_sum, nullptr, chunk_idx, chunk_score, nullptr, nullptr, err, s)
                      : launch_route_chunks_t<float, 128, false>(p, q, pos, chunk_sum, nullptr, chunk_idx, chunk_score, nullptr, nullptr, err, s);
@@ -377,6 +380,9 @@ cudaError_t launch_route(const LayerParams& p, int dtype, const void* q, const i
   if (prefill_route_path(p, dtype))
     return launch_route_prefill(p, dtype, true, true, q, pos, chunk_sum, group_sum, chunk_idx,
                                 chunk_score, group_idx, group_score, err, s);
+  if (decode_route_path(p))
+    return launch_route_decode(p, dtype, true, true, q, pos, chunk_sum, group_sum, chunk_idx,
+                               chunk_score, group_idx, group_score, err, s);
   if (dtype == 0)
     return p.D == 64 ? launch_route_chunks_t<float, 64, true>(p, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx, group_score, err, s)
                      : launch_route_chunks_t<float, 128, true>(p, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx, group_score, err, s);
@@ -392,6 +398,10 @@ cudaError_t launch_route_groups(const LayerParams& p, int dtype, const void* q, 
     return launch_route_prefill(p, dtype, false, true, q, pos, nullptr, group_sum,
                                 const_cast<int32_t*>(chunk_idx), nullptr, group_idx, group_score,
                                 err, s);
+  if (decode_route_path(p))
+    return launch_route_decode(p, dtype, false, true, q, pos, nullptr, group_sum,
+                               const_cast<int32_t*>(chunk_idx), nullptr, group_idx, group_score,
+                               err, s);
   if (dtype == 0)
     return p.D == 64 ? launch_route_groups_t<float, 64>(p, q, pos, group_sum, chunk_idx, group_idx, group_score, err, s)
                      : launch_route_groups_t<float, 128>(p, q, pos, group_sum, chunk_idx, group_idx, group_score, err, s);

@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_SHAPE", 3: "H
 # Exported symbols of the C ABI, in header order.
 SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device_status",
            "hga_workspace_size", "hga_build_summaries", "hga_route_chunks", "hga_route_groups",
-           "hga_route", "hga_hot_rows", "hga_gather_host", "hga_attend", "hga_attend_noalloc")
+           "hga_route", "hga_hot_rows", "hga_gather_host", "hga_attend", "hga_decode_step",
+           "hga_attend_noalloc")
 
 
 class HGAConfig(ctypes.Structure):
@@ -73,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_hot_rows": (ctypes.c_int, [C, ctypes.POINTER(I64)]),
         "hga_gather_host": (ctypes.c_int, [C, P, P, I64, P, P, P, P, I32, P]),
         "hga_attend": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, SZ, P]),
+        "hga_decode_step": (ctypes.c_int, [C, P, P, P, P, I64, P, P, P, P, P, P, P, P, P]),
         "hga_attend_noalloc": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -209,6 +211,16 @@ def hga_attend(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=
                                      _ptr(v), n_alloc, _ptr(group_idx), _ptr(out), _ptr(lse),
                                      _ptr(workspace), workspace_bytes, _stream(stream)),
            "hga_attend")
+
+
+def hga_decode_step(cfg, q, pos, chunk_sum, group_sum, n_alloc: int, k, v, chunk_idx, group_idx,
+                    out, lse=None, chunk_score=None, group_score=None, stream=None) -> None:
+    """Routing and attention of one decode step in one launch (hga_route + hga_attend)."""
+    _check(load_library().hga_decode_step(ctypes.byref(_cfg(cfg)), _ptr(q), _ptr(pos),
+                                          _ptr(chunk_sum), _ptr(group_sum), n_alloc, _ptr(k),
+                                          _ptr(v), _ptr(chunk_idx), _ptr(chunk_score),
+                                          _ptr(group_idx), _ptr(group_score), _ptr(out),
+                                          _ptr(lse), _stream(stream)), "hga_decode_step")
 
 
 def hga_attend_noalloc(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=None,

@@ -263,4 +263,26 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attend");
 }
 
+hga_status hga_decode_step(const hga_config* cfg, const void* q, const int64_t* pos,
+                           const float* chunk_sum, const float* group_sum, int64_t n_alloc,
+                           const void* k, const void* v, int32_t* chunk_idx, float* chunk_score,
+                           int32_t* group_idx, float* group_score, void* out, float* lse,
+                           void* stream) {
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if (!q || !pos || !chunk_sum || !group_sum || !k || !v || !chunk_idx || !group_idx || !out)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (cfg->kv_loc != HGA_KV_DEVICE || !decode_step_path(p, cfg->dtype))
+    return fail(HGA_ERR_UNSUPPORTED,
+                "hga_decode_step is built for bf16, head_dim 128, group 16 decode with K/V in "
+                "device memory; use hga_route + hga_attend");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_decode_step(p, cfg->out_dtype, q, pos, chunk_sum, group_sum, k, v,
+                                     chunk_idx, chunk_score, group_idx, group_score, out, lse, err,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_decode_step");
+}
+
 }  // extern "C"

@@ -112,6 +112,15 @@ cudaError_t launch_route_decode(const LayerParams& p, int dtype, bool level1, bo
                                 int32_t* group_idx, float* group_score, unsigned* err,
                                 cudaStream_t s);
 
+// One decode step (routing + attention) in one launch; applies when
+// decode_step_path (bf16, D = 128 decode, device-resident K/V).
+bool decode_step_path(const LayerParams& p, int dtype);
+cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* q,
+                               const int64_t* pos, const float* chunk_sum, const float* group_sum,
+                               const void* k, const void* v, int32_t* chunk_idx,
+                               float* chunk_score, int32_t* group_idx, float* group_score,
+                               void* out, float* lse, unsigned* err, cudaStream_t s);
+
 // Workspace bytes of launch_attend for p (0 when the launch needs none).
 size_t attend_workspace_bytes(const LayerParams& p, int dtype);
 

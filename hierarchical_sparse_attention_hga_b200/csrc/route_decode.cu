@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "route_common.cuh"
 #include "topk.cuh"
 
 namespace cg = cooperative_groups;
@@ -31,14 +32,14 @@ namespace cg = cooperative_groups;
 namespace hga {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kWarps = kThreads / 32;
+using route::kThreads;
+using route::kWarps;
+using route::round4;
+using route::score_rows8;
+using route::cta_topk;
 constexpr int kMaxCluster = 8;
-constexpr int kRankTopkMax = 128;  // rank-count top-k up to this many candidates
 
 enum { kL1 = 1, kL2 = 2 };
-
-__host__ __device__ constexpr int round4(int n) { return (n + 3) & ~3; }
 
 // Dynamic shared memory, in 4-byte words (each part a multiple of 4 words):
 //   qbar [D] | slice scores [per] | warp top-k scratch keys, ids [2 x kWarps x 64] |
@@ -110,58 +111,6 @@ int max_active_clusters(int cl, size_t smem) {
   return n;
 }
 
-// Scores n summary rows, row(i) a float4 pointer to D floats, against qv (this
-// lane's float4 columns s8, s8 + 8, ... of the query) into sc[0..n).
-template <int D, typename RowFn>
-__device__ __forceinline__ void score_rows8(int n, const float4 (&qv)[D / 32], float* sc, RowFn row) {
-  constexpr int F4 = D / 32;
-  constexpr int UNR = 8 / F4;  // eight float4 loads in flight per lane
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane >> 3, s8 = lane & 7;
-  for (int r0 = warp * 4 * UNR; r0 < n; r0 += kWarps * 4 * UNR) {
-    float4 x[UNR][F4];
-#pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const float4* src = row(min(r0 + u * 4 + sub, n - 1));
-#pragma unroll
-      for (int k = 0; k < F4; ++k) x[u][k] = __ldg(src + s8 + 8 * k);
-    }
-#pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      float a = 0.f;
-#pragma unroll
-      for (int k = 0; k < F4; ++k) {
-        a = fmaf(x[u][k].x, qv[k].x, a);
-        a = fmaf(x[u][k].y, qv[k].y, a);
-        a = fmaf(x[u][k].z, qv[k].z, a);
-        a = fmaf(x[u][k].w, qv[k].w, a);
-      }
-      a += __shfl_xor_sync(0xffffffffu, a, 4);  // the same sum in all eight lanes
-      a += __shfl_xor_sync(0xffffffffu, a, 2);
-      a += __shfl_xor_sync(0xffffffffu, a, 1);
-      const int i = r0 + u * 4 + sub;
-      if (s8 == 0 && i < n) sc[i] = a;
-    }
-  }
-}
-
-// Top-k of sc[0..n) (ties to the lower index) into out[0..), ascending; block-
-// collective, out complete on return.  Small candidate sets (every decode set of
-// the usual shapes) take the rank count over all 128 threads; larger ones one
-// warp's top-k.
-__device__ __forceinline__ int cta_topk(const float* sc, int n, int k, int* out, TopkSmem& tsm,
-                                        unsigned* lkey, int* lidx, int* s_n) {
-  if (n <= kRankTopkMax) return block_topk_rank<kThreads>(sc, n, k, out, tsm);
-  if ((threadIdx.x >> 5) == 0) {
-    const int r = warp_topk(sc, n, k, out, lkey, lidx);
-    if ((threadIdx.x & 31) == 0) *s_n = r;
-  }
-  __syncthreads();
-  const int r = *s_n;
-  __syncthreads();
-  return r;
-}
-
 template <typename T, int D, int MODE>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 route_decode_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
@@ -174,7 +123,7 @@ route_decode_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
   constexpr int F4 = D / 32;
   extern __shared__ __align__(16) float dyn[];
   __shared__ int s_n;
-  __shared__ TopkSmem tsm;
+  __shared__ int s_cnt[kWarps];
   cg::cluster_group cluster = cg::this_cluster();
   const int cl = kLevel1 ? static_cast<int>(cluster.num_blocks()) : 1;
   const int rank = kLevel1 ? static_cast<int>(cluster.block_rank()) : 0;
@@ -202,12 +151,7 @@ route_decode_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
   const int cur = ok ? static_cast<int>(pb / p.C) : 0;
 
   // routing query: mean of the G heads' query rows (q is never written by this library)
-  for (int d = threadIdx.x; d < D; d += kThreads) {
-    float s = 0.f;
-    for (int hh = 0; hh < p.G; ++hh)
-      s += to_f32(q[(static_cast<size_t>(b) * p.Hq + h * p.G + hh) * D + d]);
-    qbar[d] = s / static_cast<float>(p.G);
-  }
+  route::decode_query_mean<T, D>(q, p, b, h, qbar);
   pdl_wait();  // the summaries may come from the kernel just before
   __syncthreads();
   float4 qv[F4];
@@ -221,11 +165,11 @@ route_decode_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
     const int slice = (n_cand + cl - 1) / cl;
     const int lo = min(n_cand, rank * slice), hi = min(n_cand, lo + slice);
     const float* rows = chunk_sum + (static_cast<size_t>(item) * p.n_chunks + p.sink + lo) * D;
-    score_rows8<D>(hi - lo, qv, sc, [&](int i) {
+    score_rows8<D, 8 / (D / 32)>(hi - lo, qv, sc, [&](int i) {
       return reinterpret_cast<const float4*>(rows + static_cast<size_t>(i) * D);
     });
     __syncthreads();
-    const int nl = cta_topk(sc, hi - lo, p.kc, pick, tsm, lkey, lidx, &s_n);
+    const int nl = cta_topk(sc, hi - lo, p.kc, pick, lkey, lidx, s_cnt);
     cluster.barrier_wait();  // every CTA of the cluster is running
     {
       float* dsc = cluster.map_shared_rank(psc, 0);
@@ -249,7 +193,7 @@ route_decode_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
       n_m += c;
     }
     __syncthreads();
-    ns = cta_topk(msc, n_m, p.kc, pick, tsm, lkey, lidx, &s_n);
+    ns = cta_topk(msc, n_m, p.kc, pick, lkey, lidx, s_cnt);
     for (int i = threadIdx.x; i < p.kc; i += kThreads) {
       const int c = i < ns ? midx[pick[i]] + p.sink : -1;
       if (i < ns) chunks[i] = c;
@@ -278,12 +222,12 @@ route_decode_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
     // ---- level 2: the groups of the selected chunks (ascending chunk ids)
     const int n_g = ns * p.Ng;
     const float* gbase = group_sum + static_cast<size_t>(item) * p.n_chunks * p.Ng * D;
-    score_rows8<D>(n_g, qv, gsc, [&](int i) {
+    score_rows8<D, 8 / (D / 32)>(n_g, qv, gsc, [&](int i) {
       return reinterpret_cast<const float4*>(
           gbase + (static_cast<size_t>(chunks[i / p.Ng]) * p.Ng + i % p.Ng) * D);
     });
     __syncthreads();
-    const int ng = cta_topk(gsc, n_g, p.kg, gsel, tsm, lkey, lidx, &s_n);
+    const int ng = cta_topk(gsc, n_g, p.kg, gsel, lkey, lidx, s_cnt);
     for (int i = threadIdx.x; i < p.kg; i += kThreads) {
       const bool have = i < ng;
       const int sg = have ? gsel[i] : 0;

@@ -54,6 +54,28 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   __shared__ float s_gsum[8][D];             // raw group sums of one chunk
   __shared__ double s_omega[P];
   const int n_lo = P - p.n_high;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const T* kb = k + static_cast<size_t>(bh) * p.n_alloc * D;
+  // The first chunk's key rows are loaded before the tables are built (k is
+  // never written by this library), so their latency overlaps the table setup.
+  float x0[kGroup][PPL], y0[kGroup][PPL];
+  bool pre = static_cast<int>(blockIdx.x) < c_count && warp < p.Ng;
+  if (pre) {  // only rows the chunk or this warp's group finishes are read
+    const int64_t c0 = static_cast<int64_t>(c_first + blockIdx.x) * p.C;
+    const int64_t g0 = c0 + static_cast<int64_t>(warp) * kGroup;
+    pre = (c0 + p.C - 1 >= t_begin && c0 + p.C - 1 < t_end) ||
+          (g0 + kGroup - 1 >= t_begin && g0 + kGroup - 1 < t_end);
+  }
+  if (pre) {
+    const int64_t g0 = static_cast<int64_t>(c_first + blockIdx.x) * p.C + static_cast<int64_t>(warp) * kGroup;
+#pragma unroll
+    for (int o = 0; o < kGroup; ++o) {
+      const T* row = kb + (g0 + o) * D + lane * PPL;
+      PairLoad<T, PPL>::run(row, x0[o]);
+      PairLoad<T, PPL>::run(row + P, y0[o]);
+    }
+  }
   for (int i = threadIdx.x; i < n_lo; i += blockDim.x)
     s_omega[i] = pow(p.theta, -2.0 * (p.n_high + i) / D);
   __syncthreads();
@@ -74,10 +96,6 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   __syncthreads();
   pdl_wait();
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const T* kb = k + static_cast<size_t>(bh) * p.n_alloc * D;
-
   for (int ci = blockIdx.x; ci < c_count; ci += gridDim.x) {
     const int c = c_first + ci;
     const int64_t c0 = static_cast<int64_t>(c) * p.C;
@@ -91,11 +109,21 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
 #pragma unroll
         for (int u = 0; u < PPL; ++u) gx[u] = gy[u] = 0.f;
         float x[kGroup][PPL], y[kGroup][PPL];
+        if (ci == static_cast<int>(blockIdx.x)) {
 #pragma unroll
-        for (int o = 0; o < kGroup; ++o) {
-          const T* row = kb + (g0 + o) * D + lane * PPL;
-          PairLoad<T, PPL>::run(row, x[o]);
-          PairLoad<T, PPL>::run(row + P, y[o]);
+          for (int o = 0; o < kGroup; ++o)
+#pragma unroll
+            for (int u = 0; u < PPL; ++u) {
+              x[o][u] = x0[o][u];
+              y[o][u] = y0[o][u];
+            }
+        } else {
+#pragma unroll
+          for (int o = 0; o < kGroup; ++o) {
+            const T* row = kb + (g0 + o) * D + lane * PPL;
+            PairLoad<T, PPL>::run(row, x[o]);
+            PairLoad<T, PPL>::run(row + P, y[o]);
+          }
         }
 #pragma unroll
         for (int o = 0; o < kGroup; ++o) {

@@ -266,6 +266,29 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
                       void* stream);
 
 /*
+ * Steps 2-5 of one decode step in one launch: level-1 and level-2 routing
+ * (HGA technical summary, "Metodologia -> Meccanismo Core", item 2), then the
+ * gather and exact attention of the chosen tokens (item 4).  It writes what
+ * hga_route followed by hga_attend writes: chunk_idx, group_idx and the
+ * scores bit for bit, out and lse up to the order in which the kernel merges
+ * softmax partials (well inside the bf16 output's rounding).
+ *
+ * The sink, local and current chunks do not depend on routing, so their K/V
+ * loads and attention overlap the routing inside the launch, and no second
+ * launch waits on the first.  Decode only (q_len is 1): bf16 K/V in device
+ * memory (kv_loc HGA_KV_DEVICE), head_dim 128, group 16, at most 16 query
+ * heads per KV head, topk_groups <= 1024; other shapes return
+ * HGA_ERR_UNSUPPORTED (use hga_route + hga_attend).  Arguments and layouts are
+ * those of hga_route and hga_attend; chunk_score, group_score and lse may be
+ * NULL.  No workspace.
+ */
+hga_status hga_decode_step(const hga_config* cfg, const void* q, const int64_t* pos,
+                           const float* chunk_sum, const float* group_sum, int64_t n_alloc,
+                           const void* k, const void* v, int32_t* chunk_idx, float* chunk_score,
+                           int32_t* group_idx, float* group_score, void* out, float* lse,
+                           void* stream);
+
+/*
  * hga_attend for callers that cannot allocate device memory.  The paper has no
  * counterpart: this is a deployment convenience of this library.
  *

@@ -114,3 +114,23 @@ def test_workspace_size_is_zero_for_prefill_and_grows_with_batch(lib):
     # bf16, D = 128 decode merges its split-K partials inside a CTA cluster
     assert B.hga_workspace_size(B.Layer(batch=16, heads_q=32, heads_kv=8, head_dim=128), 32768,
                                 1) == 0
+
+
+def test_decode_step_rejects_what_it_does_not_fuse(lib):
+    """hga_decode_step: null pointers, fp32 K/V, D = 64 and host-tier K/V are refused on the
+    host (no CUDA call is made)."""
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    layer = B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128)
+    with pytest.raises(B.HGAError) as e:
+        B.hga_decode_step(layer, None, 16, 16, 16, 4096, 16, 16, 16, 16, 16, stream=0)
+    assert e.value.status == 1
+    for kw in (dict(dtype=B.HGA_F32), dict(head_dim=64, n_high_pairs=16)):
+        other = B.Layer(batch=1, heads_q=32, heads_kv=8, **{"head_dim": 128, **kw})
+        with pytest.raises(B.HGAError) as e:
+            B.hga_decode_step(other, 16, 16, 16, 16, 4096, 16, 16, 16, 16, 16, stream=0)
+        assert e.value.status == 3
+    host = B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128)
+    host.kv_loc = B.HGA_KV_HOST_PINNED
+    with pytest.raises(B.HGAError) as e:
+        B.hga_decode_step(host, 16, 16, 16, 16, 4096, 16, 16, 16, 16, 16, stream=0)
+    assert e.value.status == 3

@@ -87,8 +87,9 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
   }
   __syncthreads();
 
-  // Everything up to pdl_wait() reads only pos, k and v (never written by this
-  // library), so it overlaps the routing kernel still running ahead of us.
+  // Everything up to pdl_wait() reads only pos, q and the device K/V cache (never
+  // written by this library), so it overlaps the routing kernel still running
+  // ahead of us.
   const int64_t pb = a.pos[b];
   const bool ok = valid_position(pb, p, threadIdx.x == 0 && rank == 0 ? a.err : nullptr);
   const int cur = ok ? static_cast<int>(pb / p.C) : 0;
@@ -131,9 +132,11 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
       issue_unit(&tm_k, &tm_v, wsm + stage * kStageBytes, &wbar[stage],
                  static_cast<int32_t>(row_base + unit_token(u)));
   };
-  // Forced units (sink, local, current) do not depend on routing: start them now.
-  const int pre0 = u_lo < n_forced ? 1 : 0;
-  const int pre1 = u_lo + 1 < n_forced && u_lo + 1 < u_cap ? 1 : 0;
+  // Forced units (sink, local, current) do not depend on routing: start them now
+  // from the device cache.  The host tier's working buffers are written by the
+  // gather kernel just before, so there they wait for it.
+  const int pre0 = !a.hot && u_lo < n_forced ? 1 : 0;
+  const int pre1 = !a.hot && u_lo + 1 < n_forced && u_lo + 1 < u_cap ? 1 : 0;
   if (pre0) issue(u_lo, 0);
   if (pre1) issue(u_lo + 1, 1);
 
@@ -241,11 +244,13 @@ cudaError_t launch_t(const LayerParams& p, const CUtensorMap& tk, const CUtensor
   a.rows = rows;
   cudaError_t e = ensure_smem<attend_decode_bf16_kernel<TO>>(kSmemBytes);
   if (e != cudaSuccess) return e;
-  // A plain (non-programmatic) launch: measured faster here, because CTAs of
-  // this kernel launched early would hold SM slots while the routing kernel
-  // before it finishes.  pdl_wait() inside is then a no-op.
+  // Programmatic launch (the prologue and the forced units' loads overlap the
+  // routing kernel's tail) while the grid is small; a grid of more than two
+  // CTAs per SM launched early holds slots that the kernels before it (and the
+  // summary append beside it) still need, and measured slower.
+  const bool early = static_cast<int64_t>(cl) * p.B * p.Hkv <= 2 * device_sm_count();
   return launch_pdl(attend_decode_bf16_kernel<TO>, dim3(cl, p.B * p.Hkv), dim3(kWarps * 32),
-                    kSmemBytes, s, cl | kNoPdl, tk, tv, a, p);
+                    kSmemBytes, s, cl | (early ? 0 : kNoPdl), tk, tv, a, p);
 }
 
 }  // namespace

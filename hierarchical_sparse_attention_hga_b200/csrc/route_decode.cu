@@ -181,6 +181,10 @@ route_decode_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
       if (threadIdx.x == 0) cluster.map_shared_rank(pcnt, 0)[rank] = nl;
     }
     cluster.sync();  // the pushes are visible to CTA 0
+    // The next kernel may launch now: its prologue (which reads no output of
+    // this kernel) overlaps the merge and level 2 below; it still waits for
+    // this grid to complete before reading group_idx.
+    pdl_trigger();
     if (rank != 0) return;
     // ---- merge: the slices' picks in rank order (= ascending candidate index)
     int n_m = 0;

@@ -43,7 +43,7 @@ template <> struct PairLoad<__nv_bfloat16, 1> {
 
 constexpr int kGroup = 16;
 
-template <typename T, int D>
+template <typename T, int D, bool PRELOAD>
 __global__ void __launch_bounds__(256)
 summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_t t_end,
                  int c_first, int c_count, float* __restrict__ chunk_sum,
@@ -57,10 +57,11 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const T* kb = k + static_cast<size_t>(bh) * p.n_alloc * D;
-  // The first chunk's key rows are loaded before the tables are built (k is
-  // never written by this library), so their latency overlaps the table setup.
+  // With PRELOAD (each CTA finishes one chunk: a decode append), the chunk's key
+  // rows are loaded before the tables are built (k is never written by this
+  // library), so their latency overlaps the table setup.
   float x0[kGroup][PPL], y0[kGroup][PPL];
-  bool pre = static_cast<int>(blockIdx.x) < c_count && warp < p.Ng;
+  bool pre = PRELOAD && static_cast<int>(blockIdx.x) < c_count && warp < p.Ng;
   if (pre) {  // only rows the chunk or this warp's group finishes are read
     const int64_t c0 = static_cast<int64_t>(c_first + blockIdx.x) * p.C;
     const int64_t g0 = c0 + static_cast<int64_t>(warp) * kGroup;
@@ -109,7 +110,7 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
 #pragma unroll
         for (int u = 0; u < PPL; ++u) gx[u] = gy[u] = 0.f;
         float x[kGroup][PPL], y[kGroup][PPL];
-        if (ci == static_cast<int>(blockIdx.x)) {
+        if (PRELOAD && ci == static_cast<int>(blockIdx.x)) {
 #pragma unroll
           for (int o = 0; o < kGroup; ++o)
 #pragma unroll
@@ -197,7 +198,11 @@ cudaError_t launch_summaries_t(const LayerParams& p, const void* k, int64_t t_be
   dim3 grid(gx, bh);
   const int n_lo = D / 2 - p.n_high;
   const size_t smem = static_cast<size_t>(kGroup + p.Ng) * n_lo * sizeof(float2);
-  return launch_pdl(summaries_kernel<T, D>, grid, dim3(32 * p.Ng), smem, stream, 1,
+  if (c_count <= gx)  // one chunk per CTA
+    return launch_pdl(summaries_kernel<T, D, true>, grid, dim3(32 * p.Ng), smem, stream, 1,
+                      static_cast<const T*>(k), p, t_begin, t_end, c_first, c_count, chunk_sum,
+                      group_sum);
+  return launch_pdl(summaries_kernel<T, D, false>, grid, dim3(32 * p.Ng), smem, stream, 1,
                     static_cast<const T*>(k), p, t_begin, t_end, c_first, c_count, chunk_sum,
                     group_sum);
 }

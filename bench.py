@@ -337,14 +337,13 @@ def run_hga(args, rank: int, world: int):
         step = make_step(("route", "gather", "attend"))
         step2 = step
         step4 = make_step(("route_chunks", "route_groups", "gather", "attend"))
-        step1 = None
     else:
-        # The timed step: the summary append beside hga_route -> hga_attend (measured
-        # faster on B200 than the one-launch hga_decode_step, reported as one_launch_step_us).
+        # The timed step: the summary append beside hga_decode_step (one launch when the
+        # batch has about one (sequence, KV head) item per SM, else the routing and
+        # attention kernels); the two-call and four-call steps are reported beside it.
         step2 = make_step(("route", "attend"))
-        step = step2
+        step = make_step(("decode_step",)) if fused else step2
         step4 = make_step(("route_chunks", "route_groups", "attend"))
-        step1 = make_step(("decode_step",)) if fused else None
 
     # eager warm-up, then one CUDA graph for the whole step and one per call
     for _ in range(max(1, args.warmup)):
@@ -352,7 +351,7 @@ def run_hga(args, rank: int, world: int):
     torch.cuda.synchronize()
     assert B.hga_device_status(sh) == 0
     graphs = {}
-    steps = [("step", step), ("step2", step2), ("step4", step4)] + ([("step1", step1)] if step1 else [])
+    steps = [("step", step), ("step2", step2), ("step4", step4)]
     for name, fn in list(parts.items()) + steps:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
@@ -389,11 +388,6 @@ def run_hga(args, rank: int, world: int):
     a2, b2 = timed(graphs["step2"], min(args.steps, 200))
     torch.cuda.synchronize()
     ms_step2 = sum(x.elapsed_time(y) for x, y in zip(a2, b2)) / len(a2)
-    ms_step1 = None
-    if step1:
-        a1, b1 = timed(graphs["step1"], min(args.steps, 200))
-        torch.cuda.synchronize()
-        ms_step1 = sum(x.elapsed_time(y) for x, y in zip(a1, b1)) / len(a1)
     ms_step = ranks.max(ms_step)
     assert B.hga_device_status(sh) == 0
     # timing floor: an empty graph-sized launch measured the same way
@@ -447,14 +441,23 @@ def run_hga(args, rank: int, world: int):
     # one launch reads the query rows once
     nb["decode_step"] = nb["route"] + nb["attend"] - 2 * wl.batch * wl.heads_kv * wl.gqa * wl.head_dim * (
         2 if wl.dtype == "bf16" else 4)
-    kern = max(("route", "attend"), key=lambda kk: ms[kk])
+    # hga_decode_step is one launch when the batch has between half an item and one
+    # item per SM (the library's rule), else the routing and attention kernels
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    items = wl.batch * wl.heads_kv
+    one_launch = fused and sms <= 2 * items <= 2 * sms and \
+        wl.topk_chunks * (wl.chunk // wl.group) <= 128
+    kern = "decode_step" if one_launch else max(("route", "attend"), key=lambda kk: ms[kk])
     kernel_name = {"decode_step": "decode_step_kernel", "route": "route_decode_kernel",
                    "attend": "attend_decode_bf16_kernel"}[kern]
     hbm, peak_kind = peaks()
     achieved = nb[kern] / (ms[kern] * 1e-3) / 1e9
     total_bytes = nb["summaries"] + nb["route"] + nb["attend"]
-    # summaries, route, (gather,) attend (+ the split-K combine when a workspace is used)
-    launches_per_step = 3 + (1 if wsb > 0 else 0) + (1 if hot else 0)
+    if one_launch:
+        launches_per_step = 2  # summary append, decode step
+    else:
+        # summaries, route, (gather,) attend (+ the split-K combine when a workspace is used)
+        launches_per_step = 3 + (1 if wsb > 0 else 0) + (1 if hot else 0)
     tokens = wl.batch  # per rank
     line = {
         "metric": METRIC,
@@ -479,7 +482,7 @@ def run_hga(args, rank: int, world: int):
                    "l2": "flushed (256 MB write) before every timed step",
                    "parallelism": f"replicas x{world} (independent sequences per GPU)"},
         "per_kernel_us": {kk: ms[kk] * 1e3 for kk in parts},
-        "one_launch_step_us": ms_step1 * 1e3 if ms_step1 else None,
+        "two_call_step_us": ms_step2 * 1e3,
         "four_call_step_us": ms_step4 * 1e3,
         "timing_floor_us": floor_us,
         "step_hbm_bytes": total_bytes,

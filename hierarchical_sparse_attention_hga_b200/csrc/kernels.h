@@ -112,8 +112,11 @@ cudaError_t launch_route_decode(const LayerParams& p, int dtype, bool level1, bo
                                 int32_t* group_idx, float* group_score, unsigned* err,
                                 cudaStream_t s);
 
-// One decode step (routing + attention) in one launch; applies when
-// decode_step_path (bf16, D = 128 decode, device-resident K/V).
+// One decode step (routing + attention): one launch of decode_step_kernel when
+// decode_item_path (about one (sequence, KV head) item per SM), else the routing
+// and the attention kernels; applies when decode_step_path (bf16, D = 128
+// decode, device-resident K/V).
+bool decode_item_path(const LayerParams& p);
 bool decode_step_path(const LayerParams& p, int dtype);
 cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* q,
                                const int64_t* pos, const float* chunk_sum, const float* group_sum,

@@ -227,6 +227,42 @@ __device__ int block_topk(const float* sc, int n, int k, int* sel, TopkSmem& sm)
 
 namespace hga {
 
+// Top-k of sc[0..n), n <= NT, by rank counting with one candidate per thread
+// (j beats i if s_j > s_i, or s_j == s_i and j < i; i is taken when fewer than k
+// beat it), compacted in index order.  Block-collective (blockDim == NT); sc is
+// 16-byte aligned shared memory; s_cnt holds NT / 32 ints.  Writes out[0..),
+// returns min(n, k).
+template <int NT>
+__device__ int block_rank_topk(const float* sc, int n, int k, int* out, int* s_cnt) {
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  bool take = false;
+  if (t < n) {
+    const float si = sc[t];
+    int beats = 0;
+    int j = 0;
+#pragma unroll 4
+    for (; j + 4 <= n; j += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(sc + j);
+      beats += (x.x > si || (x.x == si && j < t)) + (x.y > si || (x.y == si && j + 1 < t)) +
+               (x.z > si || (x.z == si && j + 2 < t)) + (x.w > si || (x.w == si && j + 3 < t));
+    }
+    for (; j < n; ++j) beats += sc[j] > si || (sc[j] == si && j < t);
+    take = beats < k;
+  }
+  const unsigned bal = __ballot_sync(0xffffffffu, take);
+  if (lane == 0) s_cnt[w] = __popc(bal);
+  __syncthreads();
+  int at = __popc(bal & ((1u << lane) - 1u)), total = 0;
+#pragma unroll
+  for (int x = 0; x < NT / 32; ++x) {
+    if (x < w) at += s_cnt[x];
+    total += s_cnt[x];
+  }
+  if (take) out[at] = t;
+  __syncthreads();
+  return total;
+}
+
 // Per-warp scratch of warp_topk: up to kWarpTopkList (key, index) survivors.
 constexpr int kWarpTopkList = 64;
 

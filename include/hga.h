@@ -266,18 +266,21 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
                       void* stream);
 
 /*
- * Steps 2-5 of one decode step in one launch: level-1 and level-2 routing
- * (HGA technical summary, "Metodologia -> Meccanismo Core", item 2), then the
- * gather and exact attention of the chosen tokens (item 4).  It writes what
- * hga_route followed by hga_attend writes: chunk_idx, group_idx and the
- * scores bit for bit, out and lse up to the order in which the kernel merges
- * softmax partials (well inside the bf16 output's rounding).
+ * Steps 2-5 of one decode step: level-1 and level-2 routing (HGA technical
+ * summary, "Metodologia -> Meccanismo Core", item 2), then the gather and exact
+ * attention of the chosen tokens (item 4).  It writes what hga_route followed by
+ * hga_attend writes: chunk_idx, group_idx and the scores bit for bit, out and lse
+ * up to the bf16 rounding of the softmax weights (the units are attended in
+ * another grouping).
  *
- * The sink, local and current chunks do not depend on routing, so their K/V
- * loads and attention overlap the routing inside the launch, and no second
- * launch waits on the first.  Decode only (q_len is 1): bf16 K/V in device
- * memory (kv_loc HGA_KV_DEVICE), head_dim 128, group 16, at most 16 query
- * heads per KV head, topk_groups <= 1024; other shapes return
+ * When the batch holds about one (sequence, KV head) item per SM (B * Hkv
+ * between half the SM count and the SM count), the step is one launch: one CTA
+ * per item streams its chunk summaries with bulk copies, attends the sink,
+ * local and current chunks while the chosen chunks' group summaries load, then
+ * routes level 2 and attends the routed groups.  Other batches get hga_route's
+ * and hga_attend's kernels, launched by this call.  Decode only (q_len is 1):
+ * bf16 K/V in device memory (kv_loc HGA_KV_DEVICE), head_dim 128, group 16, at
+ * most 16 query heads per KV head, topk_groups <= 1024; other shapes return
  * HGA_ERR_UNSUPPORTED (use hga_route + hga_attend).  Arguments and layouts are
  * those of hga_route and hga_attend; chunk_score, group_score and lse may be
  * NULL.  No workspace.

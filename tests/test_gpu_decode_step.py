@@ -1,7 +1,9 @@
-"""One-launch decode step (hga_decode_step) against hga_route + hga_attend and the oracle.
+"""hga_decode_step against hga_route + hga_attend and the oracle.
 
-The fused kernel runs the same routing code as hga_route, so the routed indices and
-scores must be bit-identical.  Its warps attend the units in another grouping, so
+Batches with about one (sequence, KV head) item per SM run the one-launch kernel
+(one CTA per item); smaller and larger batches run the routing and attention
+kernels through the same call.  The one-launch kernel scores with the routing
+kernel's arithmetic, so the routed indices and scores must be bit-identical.  Its warps attend the units in another grouping, so
 the running maxima against which P is rounded to bf16 differ and the outputs agree
 to that rounding (well inside the 2e-2 output tolerance).  Every case is also
 checked against the float64 oracle.
@@ -125,3 +127,23 @@ def test_decode_step_llama3_8b_32k_batch16_full_size():
     for b in range(wl.batch):
         for h in range(wl.heads_kv):
             assert set(S.needle_chunks(wl, S.seed_for(1), b, h)) <= set(fus["chunk_idx"][b, h, 0])
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("llama3_8b_decode_32k", dict(batch=12, context=4096, needles=0)),
+    ("wide_head_decode_64k", dict(batch=10, context=8192, chunk=128, topk_chunks=8,
+                                  topk_groups=16)),
+])
+def test_decode_step_one_cta_per_item(name, kw):
+    """Batches with about one (sequence, KV head) item per SM take the one-CTA-per-item
+    variant; ragged positions, down to a sequence with no candidate chunk."""
+    wl = S.workload(name, **kw)
+    x = S.make_inputs(wl, 33)
+    rng = np.random.default_rng(5)
+    pos = rng.integers(wl.chunk, wl.context, size=wl.batch)
+    pos[0], pos[1], pos[2] = wl.context - 1, 5, 2 * wl.chunk + 3
+    x["pos"] = pos.astype(np.int64)
+    sep, fus = run_both(wl, x)
+    check_same_routing_close_output(sep, fus, 1e-2)
+    for b in (0, 1, 2, wl.batch - 1):
+        compare_head(wl, x, fus, b, 0)

@@ -7,7 +7,12 @@
 // sink, local and current chunks are always visible, so they are not
 // candidates: content routing covers the intermediate context only.
 //
-// One CTA per (sequence, KV head, query block).  The routing query is the mean
+// This file holds the general routing kernels and the entry points' dispatch:
+// decode goes to route_decode.cu and prefill to route_prefill.cu whenever their
+// shared-memory layouts fit (every shape up to millions of tokens); the kernels
+// below serve the rest.
+//
+// One cluster per (sequence, KV head, query block).  The routing query is the mean
 // of the block's post-RoPE query rows over the G heads sharing the KV head,
 // summed in a fixed order (deterministic).  Summary rows are streamed with
 // 16-byte loads, one row per D/4 lanes, eight rows in flight per lane; scores

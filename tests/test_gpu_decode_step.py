@@ -3,10 +3,10 @@
 Batches with about one (sequence, KV head) item per SM run the one-launch kernel
 (one CTA per item); smaller and larger batches run the routing and attention
 kernels through the same call.  The one-launch kernel scores with the routing
-kernel's arithmetic, so the routed indices and scores must be bit-identical.  Its warps attend the units in another grouping, so
-the running maxima against which P is rounded to bf16 differ and the outputs agree
-to that rounding (well inside the 2e-2 output tolerance).  Every case is also
-checked against the float64 oracle.
+kernel's arithmetic, so the routed indices and scores must be bit-identical.  Its
+warps attend the units in another grouping, so the running maxima against which P
+is rounded to bf16 differ and the outputs agree to that rounding (well inside the
+2e-2 output tolerance).  Every case is also checked against the float64 oracle.
 """
 
 import numpy as np

@@ -35,10 +35,6 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162flo
 __device__ __forceinline__ void store_out(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store_out(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
-template <typename T> struct Vec4;  // four consecutive elements
-template <> struct Vec4<float> { using type = float4; };
-template <> struct Vec4<__nv_bfloat16> { using type = uint2; };
-
 // Load 4 consecutive elements starting at p (16 B aligned for float, 8 B for bf16).
 __device__ __forceinline__ void load4(const float* p, float (&o)[4]) {
   float4 v = __ldg(reinterpret_cast<const float4*>(p));

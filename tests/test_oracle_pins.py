@@ -142,6 +142,56 @@ def test_summary_score_is_shift_invariant():
         assert score(delta) == pytest.approx(base, rel=1e-9, abs=1e-9)
 
 
+@pytest.mark.parametrize("n_high", [0, 2, 5, 8])
+@pytest.mark.parametrize("chunk,group", [(16, 4), (32, 8)])
+def test_build_summaries_table_rows_sit_at_their_span_centres(n_high, chunk, group):
+    """Every row of the chunk and group tables against the closed form of a constant raw key.
+
+    Chunk c holds the keys k_t = R(t) a_c: one raw key a_c (different for every
+    chunk) rotated to each token's own position.  Then the row of chunk c is
+    R(r) (D_C(omega) a_c) on high pairs and R(r) a_c on low pairs with
+    r = c*C + (C-1)/2, and the row of group w of chunk c is the same with
+    r = c*C + w*g + (g-1)/2 and the Dirichlet factor D_g.  A row computed at
+    another position (the chunk start, the group's chunk start, a shifted
+    centre), from another chunk's tokens, or missing its normalisation fails.
+    """
+    d, theta, nc = 16, 50.0, 6
+    prm = _params(chunk=chunk, group=group, n_high_pairs=n_high, rope_theta=theta)
+    rng = np.random.default_rng(31 + n_high)
+    a = rng.standard_normal((nc, d))
+    pos = np.arange(nc * chunk)
+    k_rot = O.rope_apply(np.repeat(a, chunk, axis=0), pos, theta)
+    cs, gs = O.build_summaries(k_rot, prm)
+    omega = O.rope_inv_freq(d, theta)
+
+    def closed_form(raw, length, centre):
+        f = np.array([_dirichlet(length, w) if i < n_high else 1.0 for i, w in enumerate(omega)])
+        return O.rope_apply((raw * np.concatenate([f, f]))[None], [centre], theta)[0]
+
+    ng = chunk // group
+    assert cs.shape == (nc, d) and gs.shape == (nc, ng, d)
+    for c in range(nc):
+        np.testing.assert_allclose(cs[c], closed_form(a[c], chunk, c * chunk + (chunk - 1) / 2),
+                                   atol=1e-11)
+        for w in range(ng):
+            centre = c * chunk + w * group + (group - 1) / 2
+            np.testing.assert_allclose(gs[c, w], closed_form(a[c], group, centre), atol=1e-11)
+
+
+def test_span_summary_start_position_cancels():
+    """The summary of given keys does not depend on the start position passed with them.
+
+    Un-rotating token m at t0 + m and re-rotating the mean at t0 + (L-1)/2 is
+    one rotation by (L-1)/2 - m: the absolute start cancels, which is why a
+    summary can be formed with one offset table for every span.
+    """
+    rng = np.random.default_rng(17)
+    k_rot = rng.standard_normal((16, 32))
+    base = O.span_summary(k_rot, 0, 5, 1e4)
+    for t0 in (1, 48, 1000, 65536):
+        np.testing.assert_allclose(O.span_summary(k_rot, t0, 5, 1e4), base, atol=1e-9)
+
+
 def test_build_summaries_leaves_incomplete_rows_undefined():
     prm = _params()
     k = np.random.default_rng(7).standard_normal((64, 16))

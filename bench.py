@@ -313,9 +313,10 @@ def run_hga(args, rank: int, world: int):
                                                        v_work, stream=st)
     # routing and attention in one launch (bf16, D = 128, K/V in device memory)
     fused = not hot and wl.dtype == "bf16" and wl.head_dim == 128 and wl.group == 16 and wl.gqa <= 16
-    if fused:
+    if fused:  # the whole step: summary append, routing and attention
         parts["decode_step"] = lambda st: B.hga_decode_step(layer, q, pos, cs, gs, n, k_src, v_src,
-                                                            ci, gi, out, lse, stream=st)
+                                                            ci, gi, out, lse, append=True,
+                                                            stream=st)
 
     side = torch.cuda.Stream()
 
@@ -338,11 +339,12 @@ def run_hga(args, rank: int, world: int):
         step2 = step
         step4 = make_step(("route_chunks", "route_groups", "gather", "attend"))
     else:
-        # The timed step: the summary append beside hga_decode_step (one launch when the
-        # batch has about one (sequence, KV head) item per SM, else the routing and
-        # attention kernels); the two-call and four-call steps are reported beside it.
+        # The timed step: hga_decode_step with the summary append (one launch when the
+        # batch has at least half a (sequence, KV head) item per SM, else the append,
+        # routing and attention kernels); the two-call and four-call steps (append on a
+        # side stream) are reported beside it.
         step2 = make_step(("route", "attend"))
-        step = make_step(("decode_step",)) if fused else step2
+        step = parts["decode_step"] if fused else step2
         step4 = make_step(("route_chunks", "route_groups", "attend"))
 
     # eager warm-up, then one CUDA graph for the whole step and one per call
@@ -439,22 +441,35 @@ def run_hga(args, rank: int, world: int):
     nb = step_bytes(wl)
     nb["route"] = nb["route_chunks"] + nb["route_groups"]
     # one launch reads the query rows once
-    nb["decode_step"] = nb["route"] + nb["attend"] - 2 * wl.batch * wl.heads_kv * wl.gqa * wl.head_dim * (
-        2 if wl.dtype == "bf16" else 4)
-    # hga_decode_step is one launch when the batch has between half an item and one
-    # item per SM (the library's rule), else the routing and attention kernels
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    items = wl.batch * wl.heads_kv
-    one_launch = fused and sms <= 2 * items <= 2 * sms and \
-        wl.topk_chunks * (wl.chunk // wl.group) <= 128
+    nb["decode_step"] = nb["summaries"] + nb["route"] + nb["attend"] - \
+        2 * wl.batch * wl.heads_kv * wl.gqa * wl.head_dim * (2 if wl.dtype == "bf16" else 4)
+    # the library says whether hga_decode_step is its one-launch kernel for this shape
+    one_launch = fused and B.hga_decode_step_launches(layer, n) == 1
     kern = "decode_step" if one_launch else max(("route", "attend"), key=lambda kk: ms[kk])
     kernel_name = {"decode_step": "decode_step_kernel", "route": "route_decode_kernel",
                    "attend": "attend_decode_bf16_kernel"}[kern]
+    # The roofline kernel's duration: CUDA events on the launch stream around a direct
+    # launch queued behind the L2 flush (the host enqueues the call while the flush
+    # runs, so the events bracket the GPU work, without the graph launch latency
+    # that the per-call graph replays above include).
+    n_direct = min(args.steps, 200)
+    ds = [torch.cuda.Event(enable_timing=True) for _ in range(n_direct)]
+    de = [torch.cuda.Event(enable_timing=True) for _ in range(n_direct)]
+    for i in range(n_direct):
+        flush.zero_()
+        ds[i].record(stream)
+        parts[kern](sh)
+        de[i].record(stream)
+    torch.cuda.synchronize()
+    kern_ms = ranks.max(sum(x.elapsed_time(y) for x, y in zip(ds, de)) / n_direct)
+    assert B.hga_device_status(sh) == 0
     hbm, peak_kind = peaks()
-    achieved = nb[kern] / (ms[kern] * 1e-3) / 1e9
+    achieved = nb[kern] / (kern_ms * 1e-3) / 1e9
     total_bytes = nb["summaries"] + nb["route"] + nb["attend"]
     if one_launch:
-        launches_per_step = 2  # summary append, decode step
+        launches_per_step = 1  # the decode step, summary append included
+    elif fused:
+        launches_per_step = 3  # summary append, routing, attention
     else:
         # summaries, route, (gather,) attend (+ the split-K combine when a workspace is used)
         launches_per_step = 3 + (1 if wsb > 0 else 0) + (1 if hot else 0)
@@ -490,9 +505,11 @@ def run_hga(args, rank: int, world: int):
         "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": profile_traffic(kernel_name, wl),
-                     "algorithmic_bytes": nb[kern],
-                     "duration": "the kernel's one-launch CUDA graph replayed after an L2 flush "
-                                 "(includes the graph launch latency)"},
+                     "algorithmic_bytes": nb[kern], "kernel_us": kern_ms * 1e3,
+                     "graph_replay_us": ms[kern] * 1e3,
+                     "duration": "CUDA events on the launch stream around a direct launch of the "
+                                 "call, queued behind the L2 flush (mean of the timed launches); "
+                                 "graph_replay_us is the call's CUDA graph replayed the same way"},
         "e2e": {"value": job_rate(tokens, world, ms_e2e), "unit": "decode tokens/s (one attention layer)",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,

@@ -23,9 +23,10 @@ STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_SHAPE", 3: "H
 
 # Exported symbols of the C ABI, in header order.
 SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device_status",
+           "hga_debug_inject",
            "hga_workspace_size", "hga_build_summaries", "hga_route_chunks", "hga_route_groups",
            "hga_route", "hga_hot_rows", "hga_gather_host", "hga_attend", "hga_decode_step",
-           "hga_attend_noalloc")
+           "hga_decode_step_launches", "hga_attend_noalloc")
 
 
 class HGAConfig(ctypes.Structure):
@@ -74,7 +75,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_hot_rows": (ctypes.c_int, [C, ctypes.POINTER(I64)]),
         "hga_gather_host": (ctypes.c_int, [C, P, P, I64, P, P, P, P, I32, P]),
         "hga_attend": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, SZ, P]),
-        "hga_decode_step": (ctypes.c_int, [C, P, P, P, P, I64, P, P, P, P, P, P, P, P, P]),
+        "hga_decode_step": (ctypes.c_int, [C, P, P, P, P, I64, P, P, P, P, P, P, P, P, I32, P]),
+        "hga_debug_inject": (I32, [I32]),
+        "hga_decode_step_launches": (ctypes.c_int, [C, I64, ctypes.POINTER(I32)]),
         "hga_attend_noalloc": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -196,6 +199,14 @@ def hga_hot_rows(cfg) -> int:
     return out.value
 
 
+def hga_decode_step_launches(cfg, n_alloc: int) -> int:
+    """1 when hga_decode_step runs as one kernel for this shape, 2 when it launches two."""
+    out = ctypes.c_int32(0)
+    _check(load_library().hga_decode_step_launches(ctypes.byref(_cfg(cfg)), n_alloc,
+                                                    ctypes.byref(out)), "hga_decode_step_launches")
+    return out.value
+
+
 def hga_gather_host(cfg, k_host, v_host, n_alloc: int, pos, group_idx, k_work, v_work,
                     refresh_window: bool = False, stream=None) -> None:
     """Host tier: stage the routed groups (and window rows) from pinned host K/V."""
@@ -214,13 +225,20 @@ def hga_attend(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=
 
 
 def hga_decode_step(cfg, q, pos, chunk_sum, group_sum, n_alloc: int, k, v, chunk_idx, group_idx,
-                    out, lse=None, chunk_score=None, group_score=None, stream=None) -> None:
-    """Routing and attention of one decode step in one launch (hga_route + hga_attend)."""
+                    out, lse=None, chunk_score=None, group_score=None, append: bool = False,
+                    stream=None) -> None:
+    """One decode step: the summary append (if asked), routing and attention."""
     _check(load_library().hga_decode_step(ctypes.byref(_cfg(cfg)), _ptr(q), _ptr(pos),
                                           _ptr(chunk_sum), _ptr(group_sum), n_alloc, _ptr(k),
                                           _ptr(v), _ptr(chunk_idx), _ptr(chunk_score),
                                           _ptr(group_idx), _ptr(group_score), _ptr(out),
-                                          _ptr(lse), _stream(stream)), "hga_decode_step")
+                                          _ptr(lse), 1 if append else 0, _stream(stream)),
+           "hga_decode_step")
+
+
+def hga_debug_inject(flags: int) -> int:
+    """Test hook: sets the library's debug flags for later launches; returns the old flags."""
+    return load_library().hga_debug_inject(flags)
 
 
 def hga_attend_noalloc(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=None,

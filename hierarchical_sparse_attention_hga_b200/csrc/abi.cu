@@ -3,6 +3,9 @@
 // aborts; see include/hga.h for the contract of each call.
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -14,6 +17,15 @@ namespace hga {
 namespace {
 
 thread_local char g_msg[512] = "";
+
+// Test hooks (kDebug* bits) copied into every launch's parameters.
+std::atomic<unsigned> g_debug{0};
+
+// NVTX range around an entry point (a no-op unless a profiler is attached).
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+};
 
 hga_status fail(hga_status st, const char* fmt, ...) {
   va_list ap;
@@ -89,6 +101,7 @@ hga_status make_params(const hga_config* cfg, int64_t n_alloc, int32_t q_len, La
   p->q_len = q_len; p->nblk = q_len == 1 ? 1 : q_len / c.chunk;
   p->n_alloc = n_alloc; p->n_chunks = static_cast<int>(n_alloc / c.chunk);
   p->theta = c.rope_theta;
+  p->debug = g_debug.load();
   return HGA_OK;
 }
 
@@ -132,8 +145,14 @@ hga_status hga_device_status(void* stream) {
   if (e == cudaSuccess) e = cudaMemsetAsync(err, 0, sizeof(unsigned), s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "hga_device_status");
+  if (host & kErrTimeout)
+    return fail(HGA_ERR_TIMEOUT, "a bounded device wait gave up, bits 0x%x", host);
   if (host) return fail(HGA_ERR_DEVICE_CHECK, "device check failed, bits 0x%x", host);
   return HGA_OK;
+}
+
+int32_t hga_debug_inject(int32_t flags) {
+  return static_cast<int32_t>(g_debug.exchange(static_cast<unsigned>(flags)));
 }
 
 hga_status hga_workspace_size(const hga_config* cfg, int64_t n_alloc, int32_t q_len, size_t* bytes) {
@@ -148,6 +167,7 @@ hga_status hga_workspace_size(const hga_config* cfg, int64_t n_alloc, int32_t q_
 hga_status hga_build_summaries(const hga_config* cfg, const void* k, int64_t n_alloc,
                                int64_t t_begin, int64_t t_end, float* chunk_sum,
                                float* group_sum, void* stream) {
+  Range nvtx_range("hga_build_summaries");
   LayerParams p;
   hga_status st = make_params(cfg, n_alloc, 1, &p);
   if (st != HGA_OK) return st;
@@ -162,6 +182,7 @@ hga_status hga_build_summaries(const hga_config* cfg, const void* k, int64_t n_a
 hga_status hga_route_chunks(const hga_config* cfg, const void* q, int32_t q_len,
                             const int64_t* pos, const float* chunk_sum, int64_t n_alloc,
                             int32_t* chunk_idx, float* chunk_score, void* stream) {
+  Range nvtx_range("hga_route_chunks");
   LayerParams p;
   hga_status st = make_params(cfg, n_alloc, q_len, &p);
   if (st != HGA_OK) return st;
@@ -177,6 +198,7 @@ hga_status hga_route_groups(const hga_config* cfg, const void* q, int32_t q_len,
                             const int64_t* pos, const float* group_sum, int64_t n_alloc,
                             const int32_t* chunk_idx, int32_t* group_idx, float* group_score,
                             void* stream) {
+  Range nvtx_range("hga_route_groups");
   LayerParams p;
   hga_status st = make_params(cfg, n_alloc, q_len, &p);
   if (st != HGA_OK) return st;
@@ -193,6 +215,7 @@ hga_status hga_route(const hga_config* cfg, const void* q, int32_t q_len, const 
                      const float* chunk_sum, const float* group_sum, int64_t n_alloc,
                      int32_t* chunk_idx, float* chunk_score, int32_t* group_idx,
                      float* group_score, void* stream) {
+  Range nvtx_range("hga_route");
   LayerParams p;
   hga_status st = make_params(cfg, n_alloc, q_len, &p);
   if (st != HGA_OK) return st;
@@ -224,6 +247,7 @@ hga_status hga_hot_rows(const hga_config* cfg, int64_t* rows) {
 hga_status hga_gather_host(const hga_config* cfg, const void* k_host, const void* v_host,
                            int64_t n_alloc, const int64_t* pos, const int32_t* group_idx,
                            void* k_work, void* v_work, int32_t refresh_window, void* stream) {
+  Range nvtx_range("hga_gather_host");
   LayerParams p;
   hga_status st = make_params(cfg, n_alloc, 1, &p);
   if (st != HGA_OK) return st;
@@ -241,6 +265,7 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
                       const void* k, const void* v, int64_t n_alloc, const int32_t* group_idx,
                       void* out, float* lse, void* workspace, size_t workspace_bytes,
                       void* stream) {
+  Range nvtx_range("hga_attend");
   LayerParams p;
   hga_status st = make_params(cfg, n_alloc, q_len, &p);
   if (st != HGA_OK) return st;
@@ -264,10 +289,11 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
 }
 
 hga_status hga_decode_step(const hga_config* cfg, const void* q, const int64_t* pos,
-                           const float* chunk_sum, const float* group_sum, int64_t n_alloc,
-                           const void* k, const void* v, int32_t* chunk_idx, float* chunk_score,
+                           float* chunk_sum, float* group_sum, int64_t n_alloc, const void* k,
+                           const void* v, int32_t* chunk_idx, float* chunk_score,
                            int32_t* group_idx, float* group_score, void* out, float* lse,
-                           void* stream) {
+                           int32_t append, void* stream) {
+  Range nvtx_range("hga_decode_step");
   LayerParams p;
   hga_status st = make_params(cfg, n_alloc, 1, &p);
   if (st != HGA_OK) return st;
@@ -280,9 +306,20 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q, const int64_t* 
   unsigned* err = nullptr;
   if ((st = device_error_ptr(&err)) != HGA_OK) return st;
   cudaError_t e = launch_decode_step(p, cfg->out_dtype, q, pos, chunk_sum, group_sum, k, v,
-                                     chunk_idx, chunk_score, group_idx, group_score, out, lse, err,
-                                     static_cast<cudaStream_t>(stream));
+                                     chunk_idx, chunk_score, group_idx, group_score, out, lse,
+                                     append != 0, err, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_decode_step");
+}
+
+hga_status hga_decode_step_launches(const hga_config* cfg, int64_t n_alloc, int32_t* launches) {
+  if (!launches) return fail(HGA_ERR_INVALID_ARG, "launches is NULL");
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if (cfg->kv_loc != HGA_KV_DEVICE || !decode_step_path(p, cfg->dtype))
+    return fail(HGA_ERR_UNSUPPORTED, "hga_decode_step does not take this shape");
+  *launches = decode_item_path(p) ? 1 : 2;
+  return HGA_OK;
 }
 
 }  // extern "C"

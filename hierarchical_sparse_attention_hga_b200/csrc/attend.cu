@@ -64,7 +64,7 @@ int choose_split_tokens(const LayerParams& p, int* nsplit) {
     return static_cast<int>(tmax);
   }
   const int64_t items = static_cast<int64_t>(p.B) * p.Hkv;
-  const int64_t want = 148 * 4;  // CTAs for a few waves on 148 SMs
+  const int64_t want = static_cast<int64_t>(device_sm_count()) * 4;  // a few waves
   int64_t per = (tmax * items + want - 1) / want;
   per = ((per + kTile - 1) / kTile) * kTile;
   per = per < 64 ? 64 : (per > 512 ? 512 : per);

@@ -218,8 +218,9 @@ int max_units(const LayerParams& p) {
 // in a single wave.
 int cluster_size(const LayerParams& p) {
   const int64_t bh = static_cast<int64_t>(p.B) * p.Hkv;
-  const int64_t want = (148 * 12 + bh * kWarps - 1) / (bh * kWarps);
-  const int64_t fit = (148 * 3) / bh;
+  const int64_t sms = device_sm_count();
+  const int64_t want = (sms * 12 + bh * kWarps - 1) / (bh * kWarps);
+  const int64_t fit = (sms * 3) / bh;
   const int64_t useful = (max_units(p) + kWarps - 1) / kWarps;
   int64_t cl = want < fit ? want : fit;
   cl = cl < useful ? cl : useful;

@@ -39,17 +39,25 @@ void* g_scratch_ptr[kMaxDevices] = {};
 // per device with that device current (cudaGetSymbolAddress) and cached.
 hga_status scratch_ptr(void** out) {
   int dev = 0;
+  char msg[256];
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    hga::set_last_error("hga_attend_noalloc: no usable current device");
+  if (e != cudaSuccess) {
+    snprintf(msg, sizeof(msg), "hga_attend_noalloc: cudaGetDevice failed: %s",
+             cudaGetErrorString(e));
+    hga::set_last_error(msg);
     return HGA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    snprintf(msg, sizeof(msg), "hga_attend_noalloc: device ordinal %d (at most %d devices)", dev,
+             kMaxDevices);
+    hga::set_last_error(msg);
+    return HGA_ERR_UNSUPPORTED;
   }
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) {
-      char msg[256];
       snprintf(msg, sizeof(msg), "hga_attend_noalloc: cudaGetSymbolAddress failed: %s",
                cudaGetErrorString(e));
       hga::set_last_error(msg);

@@ -27,7 +27,14 @@ struct LayerParams {
   int64_t n_alloc;            // cache rows per (b, h)
   int n_chunks;               // n_alloc / C
   double theta;
+  unsigned debug;             // test hooks (kDebug* bits); 0 in normal use
 };
+
+// Test hook of the one-launch decode step: warp 0 skips its first group-summary
+// copy of the first item of each CTA but still waits for it, so that bounded wait
+// runs out (nothing is in flight into that stage) and the kernel reports
+// HGA_ERR_TIMEOUT through the device error word.
+constexpr unsigned kDebugSkipRouteArrive = 1u;
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

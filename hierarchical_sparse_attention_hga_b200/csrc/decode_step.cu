@@ -1,25 +1,46 @@
-// One decode step (steps 2-5) in one launch, for batches with about one
-// (sequence, KV head) item per SM: one CTA of eight warps per item, no cluster.
-// bf16 K/V, D = 128.  Other batches take the routing and attention kernels.
+// One decode step of the HGA hot path in one launch: the summary append
+// (step 1), chunk routing (2), group routing (3), and the gather and exact
+// attention of the chosen tokens (4, 5), for every (sequence, KV head) item of
+// the batch.  bf16 K/V, D = 128; batches of at least half an item per SM (the
+// routing and attention kernels serve smaller ones).
 //
 // HGA technical summary ("Hierarchical Global Attention (HGA)", gist.science
-// 2606.30709), "Metodologia -> Meccanismo Core": item 2 (level 1 over the
-// chunk summaries, level 2 over the group summaries of the chosen chunks,
-// sink / local / current chunks always visible) and item 4 (the original K/V
-// of the chosen tokens, attended exactly with a standard softmax).
+// 2606.30709), "Metodologia -> Meccanismo Core": item 3 (RoPE-aware summaries
+// of each complete group and chunk), item 2 (level 1 over the chunk summaries,
+// level 2 over the group summaries of the chosen chunks, sink / local /
+// current chunks always visible) and item 4 (the original K/V of the chosen
+// tokens, attended exactly with a standard softmax).
 //
-// Per item, in one CTA:
-//   1. the warps start the TMA loads of their first forced units, and one
-//      thread streams the item's candidate chunk summaries (contiguous fp32
-//      rows) through a two-stage shared-memory ring with bulk copies, so the
-//      scan runs at the SM's share of the HBM bandwidth; the warps score each
-//      64-row tile from shared memory with the routing kernel's arithmetic;
-//   2. top-kc of the scores; the chosen chunks' group summaries are
-//      bulk-loaded while the warps attend the forced units;
-//   3. level 2 (top-kg), then the routed groups; the eight warps' partials are
-//      merged by log-sum-exp in shared memory.
-// Routing is bit-identical to hga_route; the output matches hga_attend up to
-// the bf16 rounding of P.
+// One CTA works on one item at a time (persistent over the items), with W
+// streaming warps and one append warp (W = 7, one CTA per SM; or W = 3, two
+// CTAs per SM when the batch has more items than SMs: eight warps per SM
+// either way, two per SM sub-partition, so each thread may hold 255 registers).  Every streaming warp owns a ring of
+// three 8 KB stages and walks its own list of 8 KB units, each one bulk or TMA
+// copy group: 16 candidate chunk-summary rows (fp32), or 16 tokens of K and V
+// (bf16, 128B-swizzled boxes).  So the whole item is a stream of equal units
+// spread over the warps, with up to 3 W units in flight.
+//
+//   scan:    candidate summary units, round-robin over all warps; each warp
+//            scores its rows with the routing kernel's arithmetic and keeps a
+//            running top-kc list in registers (a bitonic network over 64-bit
+//            keys: score order, then the lower chunk index), then publishes it;
+//   forced:  the sink, local and current chunks' K/V units, round-robin over
+//            warps 1..W-1, queued right behind their scan units (so their
+//            loads fill the gap while the routing finishes);
+//   route:   warp 0 merges the W lists (top-kc), streams the chosen chunks'
+//            group summaries through its ring and keeps a running top-kg list
+//            the same way, then publishes the routed group list;
+//   routed:  the routed groups' K/V units, round-robin over all warps;
+//   merge:   the warps' (o, m, l) partials, by log-sum-exp in shared memory.
+//
+// The append warp meanwhile finalises the summary rows that the item's new
+// token closes (a group, and the chunk when the token ends it), with the batch
+// builder's arithmetic (summary_math.cuh), so the rows are bit-identical to
+// hga_build_summaries.  Those rows belong to the current chunk, which this
+// step never routes.
+//
+// Routing is bit-identical to hga_route (same scores, same tie rule); the
+// output matches hga_attend up to the bf16 rounding of P.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -27,6 +48,7 @@
 #include "kernels.h"
 #include "ptx.cuh"
 #include "route_common.cuh"
+#include "summary_math.cuh"
 #include "tmap.h"
 #include "topk.cuh"
 
@@ -34,48 +56,193 @@ namespace hga {
 namespace {
 
 using namespace decode;
-using route::round4;
 
-constexpr int kIW = 8;                            // warps
-constexpr int kIT = kIW * 32;                     // threads
-constexpr int kTileRows = 64;                     // summary rows per scan tile
-constexpr int kRowBytes = kD * 4;                 // one fp32 summary row
-constexpr int kScanTileBytes = kTileRows * kRowBytes;  // 32 KB
-constexpr int kScanStages = 2;
-constexpr int kRingsBytes = kIW * kWarpBytes;     // 128 KB of per-warp K/V rings
+constexpr int kS = 3;                        // ring stages per streaming warp
+constexpr int kRows = 16;                    // summary rows per unit
+constexpr int kRowBytes = kD * 4;            // one fp32 summary row
+static_assert(kRows * kRowBytes == kStageBytes, "a summary unit fills one stage");
+constexpr int kKcMax = 64;                   // top-kc held as 32 * R1 keys per warp
+constexpr int kKgMax = 128;                  // routed groups per item
+constexpr unsigned kBarStream = 1;           // named barrier of the streaming warps
 
-// Words after the rings and the scan ring:
-//   qbar [D] | scores [per] | picks [kc] | chunks [kc] | group scores [kc x Ng] |
-//   chosen group positions [kg] | group list [kg]
-struct ItemSmem {
-  int per, kc, ng, kg;
-  __host__ __device__ int o_sc() const { return kD; }
-  __host__ __device__ int o_pick() const { return o_sc() + per; }
-  __host__ __device__ int o_chunks() const { return o_pick() + round4(kc); }
-  __host__ __device__ int o_gsc() const { return o_chunks() + round4(kc); }
-  __host__ __device__ int o_gsel() const { return o_gsc() + round4(ng); }
-  __host__ __device__ int o_glist() const { return o_gsel() + round4(kg); }
-  __host__ __device__ int words() const { return o_glist() + round4(kg); }
+// Barrier `id` over `n` threads, in a form that lets different warps reach it at
+// different instructions (the append warp and the streaming warps end apart).
+__device__ __forceinline__ void named_sync(unsigned id, unsigned n) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cta_sync() { asm volatile("barrier.sync 0;" ::: "memory"); }
+
+// ---------------------------------------------------------------- 64-bit keys
+// Larger key = better: the score's order key, then the lower index.
+
+__device__ __forceinline__ uint64_t make_key(float s, int id) {
+  return (static_cast<uint64_t>(order_key(s)) << 32) | static_cast<uint32_t>(~id);
+}
+__device__ __forceinline__ int key_id(uint64_t k) { return static_cast<int>(~static_cast<uint32_t>(k)); }
+__device__ __forceinline__ float key_score(uint64_t k) {
+  const uint32_t u = static_cast<uint32_t>(k >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+// One compare-exchange layer of a bitonic network over the warp's 32 R
+// elements, element e = r * 32 + lane held in a[r].  Blocks of `size` are
+// ordered descending when (e & size) == 0 == DESC. 
+template <int R, bool DESC>
+__device__ __forceinline__ void bitonic_layer(uint64_t (&a)[R], int size, int j) {
+  const int lane = threadIdx.x & 31;
+  uint64_t b[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (j >= 32) {  // partner in register r ^ (j / 32) of the same lane
+      uint64_t t = a[0];
+#pragma unroll
+      for (int q = 1; q < R; ++q)
+        if (q == (r ^ (j >> 5))) t = a[q];
+      b[r] = t;
+    } else {
+      b[r] = __shfl_xor_sync(0xffffffffu, a[r], j);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = r * 32 + lane;
+    const bool desc = ((e & size) == 0) == DESC;
+    const bool keep_max = ((e & j) == 0) == desc;
+    a[r] = keep_max ? (a[r] > b[r] ? a[r] : b[r]) : (a[r] < b[r] ? a[r] : b[r]);
+  }
+}
+
+template <int R, bool DESC>
+__device__ __forceinline__ void bitonic_sort(uint64_t (&a)[R]) {
+#pragma unroll
+  for (int size = 2; size <= 32 * R; size <<= 1)
+#pragma unroll
+    for (int j = size >> 1; j > 0; j >>= 1) bitonic_layer<R, DESC>(a, size, j);
+}
+
+// L and N sorted descending; L becomes the 32 R largest of both, descending.
+template <int R>
+__device__ __forceinline__ void merge_desc(uint64_t (&L)[R], const uint64_t (&N)[R]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const uint64_t n = __shfl_sync(0xffffffffu, N[R - 1 - r], 31 - lane);  // N reversed
+    L[r] = L[r] > n ? L[r] : n;
+  }
+#pragma unroll
+  for (int j = 16 * R; j > 0; j >>= 1) bitonic_layer<R, true>(L, 32 * R, j);
+}
+
+// Element e of a warp-distributed array.
+template <int R>
+__device__ __forceinline__ uint64_t element(const uint64_t (&a)[R], int e) {
+  uint64_t v = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (r == (e >> 5)) v = a[r];
+  return __shfl_sync(0xffffffffu, v, e & 31);
+}
+
+// Inserts key x (the same in every lane) into the sorted list L (descending,
+// 32 R entries, element e = r * 32 + lane): entries below x move down one place
+// and the last one drops out.
+template <int R>
+__device__ __forceinline__ void insert_key(uint64_t (&L)[R], uint64_t x) {
+  const int lane = threadIdx.x & 31;
+  int pos = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) pos += __popc(__ballot_sync(0xffffffffu, L[r] > x));
+  uint64_t prev[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const uint64_t up = __shfl_up_sync(0xffffffffu, L[r], 1);
+    const uint64_t last = r > 0 ? __shfl_sync(0xffffffffu, L[r > 0 ? r - 1 : 0], 31) : 0ull;
+    prev[r] = lane == 0 ? last : up;  // element e - 1
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = r * 32 + lane;
+    L[r] = e < pos ? L[r] : (e == pos ? x : prev[r]);
+  }
+}
+
+// Adds the 16 new keys of lanes 0..15 (0 = none) to the running list L
+// (descending; the first k entries are the k best so far).  The keys that beat
+// the k-th entry are inserted one at a time (usually a few); a batch with many
+// winners (the first units) is sorted and merged instead.
+template <int R>
+__device__ __forceinline__ void offer16(uint64_t (&L)[R], uint64_t nk, int k) {
+  unsigned m = __ballot_sync(0xffffffffu, nk > element<R>(L, k - 1));
+  if (__popc(m) > 6) {
+    uint64_t n[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) n[r] = r == 0 ? nk : 0ull;
+    bitonic_sort<R, true>(n);
+    merge_desc<R>(L, n);
+    return;
+  }
+  while (m) {
+    const int src = __ffs(m) - 1;
+    m &= m - 1;
+    insert_key<R>(L, __shfl_sync(0xffffffffu, nk, src));
+  }
+}
+
+// Scores of 16 fp32 summary rows in shared memory against the routing query
+// (qv: this lane's float4 columns s8, s8 + 8, ... with s8 = lane % 8), with the
+// routing kernel's arithmetic (eight lanes per row, the same sum order).  Lane
+// L < 16 returns the score of row L.
+__device__ __forceinline__ float score16(const float* rows, const float4 (&qv)[kD / 32]) {
+  const int lane = threadIdx.x & 31, sub = lane >> 3, s8 = lane & 7;
+  float mine = 0.f;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const float4* src = reinterpret_cast<const float4*>(rows + (it * 4 + sub) * kD);
+    float a = 0.f;
+#pragma unroll
+    for (int k = 0; k < kD / 32; ++k) {
+      const float4 x = src[s8 + 8 * k];
+      a = fmaf(x.x, qv[k].x, a);
+      a = fmaf(x.y, qv[k].y, a);
+      a = fmaf(x.z, qv[k].z, a);
+      a = fmaf(x.w, qv[k].w, a);
+    }
+    a += __shfl_xor_sync(0xffffffffu, a, 4);  // the same sum in all eight lanes
+    a += __shfl_xor_sync(0xffffffffu, a, 2);
+    a += __shfl_xor_sync(0xffffffffu, a, 1);
+    const float v = __shfl_sync(0xffffffffu, a, (lane & 3) * 8);
+    if ((lane >> 2) == it) mine = v;
+  }
+  return mine;
+}
+
+// ------------------------------------------------------------ shared memory
+
+constexpr int kL2Max = kKcMax * 8;  // level-2 candidates: chosen chunks x groups per chunk
+
+struct StepSmem {  // byte offsets into the dynamic shared memory (after alignment)
+  int W, n_tab;
+  __host__ __device__ size_t rings() const { return static_cast<size_t>(W) * kS * kStageBytes; }
+  __host__ __device__ size_t o_union() const { return rings(); }                    // u64 [W][kKcMax]
+  __host__ __device__ size_t o_ckey() const { return o_union() + static_cast<size_t>(W) * kKcMax * 8; }
+  __host__ __device__ size_t o_gkey() const { return o_ckey() + kKcMax * 8; }       // u64 [kL2Max]
+  __host__ __device__ size_t o_gsc() const { return o_gkey() + kL2Max * 8; }        // float [kKgMax]
+  __host__ __device__ size_t o_qbar() const { return o_gsc() + kKgMax * 4; }        // float [kD]
+  __host__ __device__ size_t o_chunks() const { return o_qbar() + kD * 4; }         // int [kKcMax]
+  __host__ __device__ size_t o_glist() const { return o_chunks() + kKcMax * 4; }    // int [kKgMax]
+  __host__ __device__ size_t o_gsum() const { return o_glist() + kKgMax * 4; }      // float [8][kD]
+  __host__ __device__ size_t o_tab() const { return o_gsum() + 8 * kD * 4; }        // float2 [n_tab]
+  __host__ __device__ size_t bytes() const { return 1024 + o_tab() + static_cast<size_t>(n_tab) * 8; }
 };
-__host__ __device__ inline ItemSmem item_smem(const LayerParams& p) {
-  ItemSmem L;
-  L.per = round4(p.n_chunks);
-  L.kc = p.kc;
-  L.ng = p.kc * p.Ng;
-  L.kg = p.kg;
-  return L;
-}
-__host__ __device__ inline size_t item_smem_bytes(const LayerParams& p) {
-  return 1024 + kRingsBytes + kScanStages * kScanTileBytes +
-         static_cast<size_t>(item_smem(p).words()) * 4;
-}
 
 template <typename TO>
-struct ItemArgs {
+struct StepArgs {
   const __nv_bfloat16* q;
   const int64_t* pos;
-  const float* chunk_sum;
-  const float* group_sum;
+  const __nv_bfloat16* k;   // the cache (the append warp's reads; address warming)
+  const __nv_bfloat16* v;
+  float* chunk_sum;
+  float* group_sum;
   int32_t* chunk_idx;
   float* chunk_score;
   int32_t* group_idx;
@@ -83,286 +250,467 @@ struct ItemArgs {
   TO* out;
   float* lse;
   unsigned* err;
+  int append;
+  int n_items;
 };
 
-// Scores rows [0, n) held in shared memory at `rows` (kD floats each) against
-// qv into sc[0..n): eight lanes per row, the routing kernel's arithmetic.
-__device__ __forceinline__ void score_smem_rows(const float* rows, int n, const float4 (&qv)[kD / 32],
-                                                float* sc) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane >> 3, s8 = lane & 7;
-  for (int r0 = warp * 8; r0 < n; r0 += kIW * 8) {
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i = r0 + u * 4 + sub;
-      const float4* src = reinterpret_cast<const float4*>(rows + static_cast<size_t>(min(i, n - 1)) * kD);
-      float a = 0.f;
-#pragma unroll
-      for (int k = 0; k < kD / 32; ++k) {
-        const float4 x = src[s8 + 8 * k];
-        a = fmaf(x.x, qv[k].x, a);
-        a = fmaf(x.y, qv[k].y, a);
-        a = fmaf(x.z, qv[k].z, a);
-        a = fmaf(x.w, qv[k].w, a);
-      }
-      a += __shfl_xor_sync(0xffffffffu, a, 4);  // the same sum in all eight lanes
-      a += __shfl_xor_sync(0xffffffffu, a, 2);
-      a += __shfl_xor_sync(0xffffffffu, a, 1);
-      if (s8 == 0 && i < n) sc[i] = a;
-    }
+// 2 MB pages of each of the item's group-summary, K and V regions whose address
+// translation is warmed at the start of an item (covers 16 MB, a 64K context).
+constexpr int kTlbPages = 8;
+
+// Place of `key` among the n keys at `keys` (shared memory): the number above it.
+__device__ __forceinline__ int rank_among(const uint64_t* keys, int n, uint64_t key) {
+  int r0 = 0, r1 = 0, i = 0;
+#pragma unroll 4
+  for (; i + 2 <= n; i += 2) {
+    r0 += keys[i] > key;
+    r1 += keys[i + 1] > key;
   }
+  if (i < n) r0 += keys[i] > key;
+  return r0 + r1;
 }
 
-// Top-k of sc[0..n) into out[0..), ascending (block-collective, kIT threads).
-__device__ __forceinline__ int item_topk(const float* sc, int n, int k, int* out, int* s_cnt,
-                                         TopkSmem& tsm) {
-  if (n <= kIT) return block_rank_topk<kIT>(sc, n, k, out, s_cnt);
-  return block_topk<kIT>(sc, n, k, out, tsm);
-}
+// ------------------------------------------------------------------ kernel
+//
+// Per item, every streaming warp walks one stream of units through its ring:
+//
+//   [scan units] | B1 top-kc by rank B2 | [group-summary units of its chosen
+//   chunks] [window units] | B3 top-kg by rank B4 | [routed units]
+//
+// where B1..B4 are barriers of the streaming warps.  The group-summary fetch is
+// the critical path after the scan, so each warp queues its window (sink, local,
+// current) loads right behind its own group-summary copies; they land while the
+// level-2 selection runs.
 
-template <typename TO>
-__global__ void __launch_bounds__(kIT, 1)
+template <int W, int R1, typename TO>
+__global__ void __launch_bounds__((W + 1) * 32, W == 7 ? 1 : 2)
 decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, ItemArgs<TO> a, LayerParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, StepArgs<TO> a, LayerParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bars[kIW][kStages];
-  __shared__ uint64_t bar_scan[kScanStages], bar_l2;
-  __shared__ float s_ml[kIW][16][2];
-  __shared__ int s_cnt[kIW];
-  __shared__ TopkSmem tsm;
+  __shared__ uint64_t bars[W][kS];
+  __shared__ float s_ml[W][16][2];
+  __shared__ int s_abort;
 
-  const int item = blockIdx.x;  // (sequence, KV head) = b * Hkv + h
-  const int b = item / p.Hkv, h = item % p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  uint8_t* ring0 = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* scan = ring0 + kRingsBytes;
-  float* rw = reinterpret_cast<float*>(scan + kScanStages * kScanTileBytes);
-  const ItemSmem L = item_smem(p);
-  float* qbar = rw;
-  float* sc = rw + L.o_sc();
-  int* pick = reinterpret_cast<int*>(rw + L.o_pick());
-  int* chunks = reinterpret_cast<int*>(rw + L.o_chunks());
-  float* gsc = rw + L.o_gsc();
-  int* gsel = reinterpret_cast<int*>(rw + L.o_gsel());
-  int* glist = reinterpret_cast<int*>(rw + L.o_glist());
+  const int tid = threadIdx.x;  // streaming threads: 0 .. W * 32 - 1
+  uint8_t* base = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
+  StepSmem L{W, summ::table_entries(p, kD)};
+  uint64_t* s_union = reinterpret_cast<uint64_t*>(base + L.o_union());
+  uint64_t* ckey = reinterpret_cast<uint64_t*>(base + L.o_ckey());  // chosen chunks' keys, rank order
+  uint64_t* gkey = reinterpret_cast<uint64_t*>(base + L.o_gkey());
+  float* gsc = reinterpret_cast<float*>(base + L.o_gsc());
+  float* qbar = reinterpret_cast<float*>(base + L.o_qbar());
+  int* chunks = reinterpret_cast<int*>(base + L.o_chunks());  // chosen chunks, rank order
+  int* glist = reinterpret_cast<int*>(base + L.o_glist());    // routed groups, rank order
+  float(*gsum)[kD] = reinterpret_cast<float(*)[kD]>(base + L.o_gsum());
+  float2* tab = reinterpret_cast<float2*>(base + L.o_tab());
 
   if (threadIdx.x == 0) {
     ptx::prefetch_tensormap(&tm_k);
     ptx::prefetch_tensormap(&tm_v);
-    for (int w = 0; w < kIW; ++w)
-      for (int s = 0; s < kStages; ++s) ptx::mbar_init(&bars[w][s], 1);
-    for (int s = 0; s < kScanStages; ++s) ptx::mbar_init(&bar_scan[s], 1);
-    ptx::mbar_init(&bar_l2, 1);
+    for (int w = 0; w < W; ++w)
+      for (int s = 0; s < kS; ++s) ptx::mbar_init(&bars[w][s], 1);
+    s_abort = 0;
     ptx::fence_barrier_init();
   }
   __syncthreads();
 
-  const int64_t pb = a.pos[b];  // pos, q, k and v are never written by this library
-  const bool ok = valid_position(pb, p, threadIdx.x == 0 ? a.err : nullptr);
-  const int cur = ok ? static_cast<int>(pb / p.C) : 0;
-  const int b0 = max(0, cur - p.local);
-  // forced units: sink [0, su), then local + current up to the query [su, n_forced)
-  const int ng_per_c = p.C / kUnit;
-  const int su = ok ? min(p.sink, b0) * ng_per_c : 0;
-  const int u_first_local = b0 * ng_per_c;
-  const int n_forced = ok ? su + static_cast<int>(pb / kUnit) - u_first_local + 1 : 0;
-  auto forced_token = [&](int u) -> int64_t {
-    return static_cast<int64_t>(u < su ? u : u_first_local + (u - su)) * kUnit;
-  };
-  const int fpw = (n_forced + kIW - 1) / kIW;
-  const int f_lo = min(n_forced, warp * fpw), f_hi = min(n_forced, f_lo + fpw);
-
-  uint8_t* wsm = ring0 + warp * kWarpBytes;
-  const uint32_t wsm_u32 = ptx::smem_u32(wsm);
-  uint64_t* wbar = bars[warp];
-  const int64_t row_base = static_cast<int64_t>(item) * p.n_alloc;
-  int issued = 0, done = 0;
-  auto issue_token = [&](int64_t tok) {
-    if (lane == 0)
-      issue_unit(&tm_k, &tm_v, wsm + (issued & 1) * kStageBytes, &wbar[issued & 1],
-                 static_cast<int32_t>(row_base + tok));
-    ++issued;
-  };
-  int f_next = f_lo;
-  while (f_next < f_hi && issued < kStages) issue_token(forced_token(f_next++));
-
-  route::decode_query_mean<__nv_bfloat16, kD>(a.q, p, b, h, qbar);  // threads < D
-  pdl_wait();  // the summaries may come from the kernel just before
-
-  // ---- 1. level 1: stream the candidate chunk summaries through the scan ring
-  const int n_cand = ok ? max(0, cur - p.local - p.sink) : 0;
-  const int n_tiles = (n_cand + kTileRows - 1) / kTileRows;
-  const float* cbase = a.chunk_sum + (static_cast<size_t>(item) * p.n_chunks + p.sink) * kD;
-  auto issue_tile = [&](int t) {  // one thread
-    const int nr = min(kTileRows, n_cand - t * kTileRows);
-    uint64_t* bar = &bar_scan[t % kScanStages];
-    ptx::mbar_expect_tx(bar, static_cast<uint32_t>(nr) * kRowBytes);
-    ptx::bulk_load(scan + (t % kScanStages) * kScanTileBytes,
-                   cbase + static_cast<size_t>(t) * kTileRows * kD,
-                   static_cast<uint32_t>(nr) * kRowBytes, bar);
-  };
-  if (threadIdx.x == 0)
-    for (int t = 0; t < min(n_tiles, kScanStages); ++t) issue_tile(t);
-  __syncthreads();  // qbar
-  float4 qv[kD / 32];
-#pragma unroll
-  for (int k = 0; k < kD / 32; ++k) qv[k] = reinterpret_cast<const float4*>(qbar)[(lane & 7) + 8 * k];
-
-  bool timed_out = false;
-  for (int t = 0; t < n_tiles; ++t) {
-    const bool landed = ptx::mbar_wait(&bar_scan[t % kScanStages], (t / kScanStages) & 1, kWaitLimit);
-    if (!landed) timed_out = true;
-    const int nr = min(kTileRows, n_cand - t * kTileRows);
-    if (landed)
-      score_smem_rows(reinterpret_cast<const float*>(scan + (t % kScanStages) * kScanTileBytes), nr,
-                      qv, sc + t * kTileRows);
-    __syncthreads();  // the stage is free again
-    if (threadIdx.x == 0 && t + kScanStages < n_tiles) issue_tile(t + kScanStages);
-  }
-  const bool scan_ok = !__syncthreads_or(timed_out);
-  if (!scan_ok && threadIdx.x == 0)  // every tile was issued: wait (bounded) for the last ones
-    for (int t = max(0, n_tiles - kScanStages); t < n_tiles; ++t)
-      ptx::mbar_wait(&bar_scan[t % kScanStages], (t / kScanStages) & 1, kWaitLimit);
-  const int ns = scan_ok ? item_topk(sc, n_cand, p.kc, pick, s_cnt, tsm) : 0;
-  for (int i = threadIdx.x; i < p.kc; i += kIT) {
-    const int c = i < ns ? pick[i] + p.sink : -1;
-    if (i < ns) chunks[i] = c;
-    a.chunk_idx[static_cast<size_t>(item) * p.kc + i] = c;
-    if (a.chunk_score)
-      a.chunk_score[static_cast<size_t>(item) * p.kc + i] = i < ns ? sc[pick[i]] : CUDART_NAN_F;
-  }
-  __syncthreads();
-  // the chosen chunks' group summaries (Ng contiguous rows each) into the scan ring
-  const int n_g = ns * p.Ng;
-  const float* gbase = a.group_sum + static_cast<size_t>(item) * p.n_chunks * p.Ng * kD;
-  if (threadIdx.x == 0 && n_g > 0) {
-    ptx::mbar_expect_tx(&bar_l2, static_cast<uint32_t>(n_g) * kRowBytes);
-    for (int i = 0; i < ns; ++i)
-      ptx::bulk_load(scan + static_cast<size_t>(i) * p.Ng * kRowBytes,
-                     gbase + static_cast<size_t>(chunks[i]) * p.Ng * kD,
-                     static_cast<uint32_t>(p.Ng) * kRowBytes, &bar_l2);
-  }
-
-  // ---- 2. the forced units, while the group summaries load
-  uint32_t qa[8][4];
-  load_q_frags(a.q, p, b, h, qa);
-  const float scale = kLog2e * rsqrtf(static_cast<float>(kD));
-  WarpState w;
-  w.init();
-  auto consume = [&](int valid) -> bool {
-    const int st = done & 1;
-    if (!ptx::mbar_wait(&wbar[st], (done >> 1) & 1, kWaitLimit)) return false;
-    const uint32_t kt = wsm_u32 + st * kStageBytes;
-    attend_unit(kt, kt + kTileBytes, valid, qa, scale, w);
-    ++done;
-    return true;
-  };
-  for (int u = f_lo; u < f_hi && !timed_out; ++u) {
-    if (!consume(u == n_forced - 1 ? static_cast<int>(pb % kUnit) + 1 : kUnit)) {
-      timed_out = true;
-      break;
-    }
-    if (f_next < f_hi) issue_token(forced_token(f_next++));
-  }
-
-  // ---- 3. level 2, then the routed groups
-  bool l2_ok = true;
-  if (n_g > 0) {
-    l2_ok = ptx::mbar_wait(&bar_l2, 0, kWaitLimit);
-    if (l2_ok) score_smem_rows(reinterpret_cast<const float*>(scan), n_g, qv, gsc);
-  }
-  l2_ok = !__syncthreads_or(!l2_ok);
-  if (!l2_ok) timed_out = true;
-  const int ng = l2_ok ? item_topk(gsc, n_g, p.kg, gsel, s_cnt, tsm) : 0;
-  for (int i = threadIdx.x; i < p.kg; i += kIT) {
-    const bool have = i < ng;
-    const int sg = have ? gsel[i] : 0;
-    const int gid = have ? chunks[sg / p.Ng] * p.Ng + sg % p.Ng : -1;
-    a.group_idx[static_cast<size_t>(item) * p.kg + i] = gid;
-    if (a.group_score)
-      a.group_score[static_cast<size_t>(item) * p.kg + i] = have ? gsc[sg] : CUDART_NAN_F;
-    if (have) glist[i] = gid;
-  }
-  __syncthreads();
-  const int rpw = (ng + kIW - 1) / kIW;
-  const int r_lo = min(ng, warp * rpw), r_hi = min(ng, r_lo + rpw);
-  int r_next = r_lo;
-  if (!timed_out)
-    while (r_next < r_hi && issued - done < kStages)
-      issue_token(static_cast<int64_t>(glist[r_next++]) * kUnit);
-  for (int u = r_lo; u < r_hi && !timed_out; ++u) {
-    if (!consume(kUnit)) {
-      timed_out = true;
-      break;
-    }
-    if (r_next < r_hi) issue_token(static_cast<int64_t>(glist[r_next++]) * kUnit);
-  }
-  if (timed_out) {
-    // A wait gave up: the partial is dropped (the output is wrong and flagged),
-    // the copies still in flight are waited for once more (bounded), and every
-    // barrier below is still reached.
-    if (lane == 0) flag_error(a.err, kErrTimeout);
-    for (; done < issued; ++done) ptx::mbar_wait(&wbar[done & 1], (done >> 1) & 1, kWaitLimit);
-    w.m0 = w.m1 = -CUDART_INF_F;
-    w.l0 = w.l1 = 0.f;
-  }
-
-  // ---- merge the warps' partials (each in its own ring, whose copies all landed)
-  const int g = lane >> 2, t4 = lane & 3;
-  w.l0 += __shfl_xor_sync(0xffffffffu, w.l0, 1);
-  w.l0 += __shfl_xor_sync(0xffffffffu, w.l0, 2);
-  w.l1 += __shfl_xor_sync(0xffffffffu, w.l1, 1);
-  w.l1 += __shfl_xor_sync(0xffffffffu, w.l1, 2);
-  float* wo = reinterpret_cast<float*>(wsm);  // [16 heads][128]
-  if (done == 0) {
-    w.m0 = w.m1 = -CUDART_INF_F;
-    w.l0 = w.l1 = 0.f;
-  } else {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      *reinterpret_cast<float2*>(wo + g * kD + j * 8 + 2 * t4) = make_float2(w.o[j][0], w.o[j][1]);
-      *reinterpret_cast<float2*>(wo + (g + 8) * kD + j * 8 + 2 * t4) =
-          make_float2(w.o[j][2], w.o[j][3]);
-    }
-  }
-  if (t4 == 0) {
-    s_ml[warp][g][0] = w.m0;
-    s_ml[warp][g][1] = w.l0;
-    s_ml[warp][g + 8][0] = w.m1;
-    s_ml[warp][g + 8][1] = w.l1;
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < p.G * kD; idx += kIT) {
-    const int hh = idx / kD, d = idx % kD;
-    float mm = -CUDART_INF_F;
-#pragma unroll
-    for (int v = 0; v < kIW; ++v) mm = fmaxf(mm, s_ml[v][hh][0]);
-    float ll = 0.f, oo = 0.f;
-    if (mm != -CUDART_INF_F) {
-#pragma unroll
-      for (int v = 0; v < kIW; ++v) {
-        const float mv = s_ml[v][hh][0];
-        if (mv == -CUDART_INF_F) continue;
-        const float f = exp2f(mv - mm);
-        ll += s_ml[v][hh][1] * f;
-        oo += reinterpret_cast<const float*>(ring0 + v * kWarpBytes)[hh * kD + d] * f;
+  // ------------------------------------------------------------ append warp
+  if (warp == W) {
+    if (a.append) {
+      for (int i = lane; i < L.n_tab; i += 32) tab[i] = summ::table_entry(p, kD, i);
+      __syncwarp();
+      pdl_wait();  // the rows read and written may belong to the kernel just before
+      for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+        const int64_t pb = a.pos[item / p.Hkv];
+        if (pb < 0 || pb >= p.n_alloc) continue;
+        summ::append_closed_rows<__nv_bfloat16, kD>(
+            a.k + static_cast<size_t>(item) * p.n_alloc * kD,
+            a.chunk_sum + static_cast<size_t>(item) * p.n_chunks * kD,
+            a.group_sum + static_cast<size_t>(item) * p.n_chunks * p.Ng * kD, p, pb, tab, gsum);
       }
     }
-    const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + hh;
-    store_out(a.out + row * kD + d, ll > 0.f ? oo / ll : 0.f);
-    if (a.lse && d == 0) a.lse[row] = ll > 0.f ? (mm + log2f(ll)) * kLn2 : -CUDART_INF_F;
+    cta_sync();
+    pdl_trigger();
+    return;
   }
+
+  // ------------------------------------------------------- streaming warps
+  const float scale = kLog2e * rsqrtf(static_cast<float>(kD));
+  uint8_t* ring = base + static_cast<size_t>(warp) * kS * kStageBytes;
+  uint64_t* wbar = bars[warp];
+  int issued = 0, done = 0;  // this warp's ring counters, continued over items
+  int item_no = 0;           // items this CTA has started
+  auto stage = [&](int i) { return ring + (i % kS) * kStageBytes; };
+  // a debug run that withholds a copy gives up after 2 ms instead of 50 ms
+  const uint64_t limit_ns = (p.debug & kDebugSkipRouteArrive) ? 2000000ull : 50000000ull;
+  auto wait_stage = [&](int i) { return ptx::mbar_wait_ns(&wbar[i % kS], (i / kS) & 1, kWaitLimit, limit_ns); };
+  // candidate summary rows that exist past the sink chunks (whatever the position)
+  const int rows_max = max(0, p.n_chunks - p.sink);
+  const int n_su_max = (rows_max + kRows - 1) / kRows;
+  const int cpu = kRows / p.Ng;  // chosen chunks per group-summary unit
+
+  pdl_wait();  // summaries may come from the kernel just before
+  for (int item = blockIdx.x; item < a.n_items; item += gridDim.x, ++item_no) {
+    const int b = item / p.Hkv, h = item % p.Hkv;
+    if (s_abort) {  // an earlier item of this CTA timed out: write the empty result, no waits
+      if (warp == 0) {
+        for (int i = lane; i < p.kc; i += 32) a.chunk_idx[static_cast<size_t>(item) * p.kc + i] = -1;
+        for (int i = lane; i < p.kg; i += 32) a.group_idx[static_cast<size_t>(item) * p.kg + i] = -1;
+      }
+      for (int idx = tid; idx < p.G * kD; idx += W * 32) {
+        const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + idx / kD;
+        store_out(a.out + row * kD + idx % kD, 0.f);
+        if (a.lse && idx % kD == 0) a.lse[row] = -CUDART_INF_F;
+      }
+      continue;
+    }
+    const float* cbase = a.chunk_sum + (static_cast<size_t>(item) * p.n_chunks + p.sink) * kD;
+    const float* gbase = a.group_sum + static_cast<size_t>(item) * p.n_chunks * p.Ng * kD;
+    const int64_t row_base = static_cast<int64_t>(item) * p.n_alloc;
+
+    // 1. position, routing query and Q fragments: independent loads, issued first so
+    //    that they do not queue behind the bulk copies below
+    const int64_t pb = a.pos[b];
+    constexpr int kQD = (kD + W * 32 - 1) / (W * 32);  // routing-query dims per thread
+    unsigned short v[kQD][16];  // bf16 bits; converted after the bulk copies are issued
+    const unsigned short* qraw = reinterpret_cast<const unsigned short*>(a.q);
+#pragma unroll
+    for (int j = 0; j < kQD; ++j) {
+      const int d = min(kD - 1, tid + j * W * 32);
+#pragma unroll
+      for (int hh = 0; hh < 16; ++hh)
+        v[j][hh] = hh < p.G ? __ldg(qraw + (static_cast<size_t>(b) * p.Hq + h * p.G + hh) * kD + d) : 0;
+    }
+    uint32_t qa[8][4];
+    load_q_frags(a.q, p, b, h, qa);
+    // warm the address translation of the item's group-summary and K/V regions
+    // (read later at scattered places) while the scan runs
+    if (warp == 0 && lane < 3 * kTlbPages) {
+      const int which = lane / kTlbPages, page = lane % kTlbPages;
+      const size_t span = which == 0 ? static_cast<size_t>(p.n_chunks) * p.Ng * kD * 4
+                                     : static_cast<size_t>(p.n_alloc) * kD * 2;
+      const uint8_t* region = which == 0 ? reinterpret_cast<const uint8_t*>(gbase)
+                              : which == 1 ? reinterpret_cast<const uint8_t*>(a.k + row_base * kD)
+                                           : reinterpret_cast<const uint8_t*>(a.v + row_base * kD);
+      const size_t off = static_cast<size_t>(page) << 21;
+      if (off < span) asm volatile("prefetch.global.L2 [%0];" ::"l"(region + off));
+    }
+
+    // 2. the warp's first scan units before the position is known: the rows that
+    //    exist past the sink (the units beyond this item's candidates are dropped)
+    const int n_spec = min(kS, n_su_max > warp ? (n_su_max - warp + W - 1) / W : 0);
+    for (int i = 0; i < n_spec; ++i) {
+      const int su = warp + i * W;
+      if (lane == 0) {
+        const int nr = min(kRows, rows_max - su * kRows);
+        ptx::mbar_expect_tx(&wbar[issued % kS], static_cast<uint32_t>(nr) * kRowBytes);
+        ptx::bulk_load(stage(issued), cbase + static_cast<size_t>(su) * kRows * kD,
+                       static_cast<uint32_t>(nr) * kRowBytes, &wbar[issued % kS]);
+      }
+      ++issued;
+    }
+#pragma unroll
+    for (int j = 0; j < kQD; ++j) {
+      const int d = tid + j * W * 32;
+      float s = 0.f;
+#pragma unroll
+      for (int hh = 0; hh < 16; ++hh)
+        if (hh < p.G) s += __uint_as_float(static_cast<unsigned>(v[j][hh]) << 16);
+      if (d < kD) qbar[d] = s / static_cast<float>(p.G);
+    }
+
+    // 3. this item's stream: [scan | group summaries | window | routed]
+    const bool ok = valid_position(pb, p, (warp == 0 && lane == 0) ? a.err : nullptr);
+    const int cur = ok ? static_cast<int>(pb / p.C) : 0;
+    const int b0 = max(0, cur - p.local);
+    const int n_cand = ok ? max(0, cur - p.local - p.sink) : 0;
+    const int n_su = (n_cand + kRows - 1) / kRows;
+    const int upc = p.C / kUnit;  // K/V units per chunk
+    const int su_sink = ok ? min(p.sink, b0) * upc : 0;
+    const int u_first_local = b0 * upc;
+    const int n_forced = ok ? su_sink + static_cast<int>(pb / kUnit) - u_first_local + 1 : 0;
+    const int ns = min(p.kc, n_cand);       // chosen chunks
+    const int n_l2 = ns * p.Ng;             // level-2 candidates
+    const int ng = min(p.kg, n_l2);         // routed groups
+    auto count = [&](int n) { return n > warp ? (n - warp + W - 1) / W : 0; };  // i = warp + k W < n
+    const int n_head = max(count(n_su), n_spec);  // scan units (those past n_su are dropped)
+    const int n_mine = count(ns);                 // chosen chunks warp, warp + W, ...
+    const int n_fw = count(n_forced);             // window units warp, warp + W, ...
+    const int n_l2u = (n_mine + cpu - 1) / cpu;
+    const int n_rw = count(ng);
+    // stream index -> unit: [0, e_l2) scan; [e_l2, e_fw) group summaries; [e_fw, e_rt)
+    // window; [e_rt, e_all) routed
+    const int e_l2 = n_head, e_fw = e_l2 + n_l2u, e_rt = e_fw + n_fw, e_all = e_rt + n_rw;
+    auto forced_token = [&](int f) -> int64_t {
+      return static_cast<int64_t>(f < su_sink ? f : u_first_local + (f - su_sink)) * kUnit;
+    };
+    int next = n_spec;  // next stream unit to issue
+    bool timed_out = false;
+    auto issue_upto = [&](int limit) {
+      while (next < limit && issued - done < kS) {
+        const int i = next++;
+        uint8_t* st = stage(issued);
+        uint64_t* bar = &wbar[issued % kS];
+        if (lane == 0) {
+          if (i < e_l2) {
+            const int su = warp + i * W;
+            const int nr = min(kRows, n_cand - su * kRows);
+            ptx::mbar_expect_tx(bar, static_cast<uint32_t>(nr) * kRowBytes);
+            ptx::bulk_load(st, cbase + static_cast<size_t>(su) * kRows * kD,
+                           static_cast<uint32_t>(nr) * kRowBytes, bar);
+          } else if (i < e_fw) {
+            // a debug run withholds warp 0's first group-summary copy: its bounded wait
+            // on that stage then runs out with nothing in flight
+            const bool skip = (p.debug & kDebugSkipRouteArrive) && warp == 0 && item_no == 0 && i == e_l2;
+            const int k0 = (i - e_l2) * cpu, k1 = min(n_mine, k0 + cpu);
+            if (!skip) {
+              ptx::mbar_expect_tx(bar, static_cast<uint32_t>((k1 - k0) * p.Ng) * kRowBytes);
+              for (int kk = k0; kk < k1; ++kk)
+                ptx::bulk_load(st + static_cast<size_t>(kk - k0) * p.Ng * kRowBytes,
+                               gbase + static_cast<size_t>(chunks[warp + kk * W]) * p.Ng * kD,
+                               static_cast<uint32_t>(p.Ng) * kRowBytes, bar);
+            }
+          } else if (i < e_rt) {
+            issue_unit(&tm_k, &tm_v, st, bar,
+                       static_cast<int32_t>(row_base + forced_token(warp + (i - e_fw) * W)));
+          } else {
+            issue_unit(&tm_k, &tm_v, st, bar,
+                       static_cast<int32_t>(row_base + static_cast<int64_t>(glist[warp + (i - e_rt) * W]) * kUnit));
+          }
+        }
+        ++issued;
+      }
+    };
+    // consumes stream units [from, to) with `fn`, topping the ring up to `limit`
+    auto consume = [&](int from, int to, int limit, auto&& fn) {
+      for (int i = from; i < to && !timed_out; ++i) {
+        if (!wait_stage(done)) {
+          timed_out = true;
+          break;
+        }
+        fn(i, stage(done));
+        ++done;
+        __syncwarp();
+        issue_upto(limit);
+      }
+    };
+    issue_upto(e_l2);
+
+    named_sync(kBarStream, W * 32);  // qbar
+    float4 qv[kD / 32];
+#pragma unroll
+    for (int k = 0; k < kD / 32; ++k) qv[k] = reinterpret_cast<const float4*>(qbar)[(lane & 7) + 8 * k];
+
+    // ---- scan: score the warp's candidate units into a running top-kc list
+    uint64_t l1[R1];
+#pragma unroll
+    for (int r = 0; r < R1; ++r) l1[r] = 0ull;
+    consume(0, e_l2, e_l2, [&](int i, uint8_t* st) {
+      if (i * W + warp < n_su) {
+        const int su = warp + i * W;
+        const float sc = score16(reinterpret_cast<const float*>(st), qv);
+        const int r = su * kRows + lane;
+        offer16<R1>(l1, lane < kRows && r < n_cand ? make_key(sc, p.sink + r) : 0ull, p.kc);
+      }
+    });
+#pragma unroll
+    for (int r = 0; r < R1; ++r)
+      if (r * 32 + lane < p.kc) s_union[warp * p.kc + r * 32 + lane] = l1[r];
+    named_sync(kBarStream, W * 32);  // B1
+
+    // ---- level 1: the kc best of the W lists, by rank, into chunks (rank order)
+    for (int c = tid; c < W * p.kc; c += W * 32) {
+      const uint64_t key = s_union[c];
+      if (key == 0ull) continue;
+      const int rank = rank_among(s_union, W * p.kc, key);
+      if (rank < ns) {
+        chunks[rank] = key_id(key);
+        ckey[rank] = key;
+      }
+    }
+    named_sync(kBarStream, W * 32);  // B2
+
+    // ---- level 2: this warp's chosen chunks' group rows (then its window units
+    // queue behind them and land while the selection runs)
+    issue_upto(e_rt);
+    consume(e_l2, e_fw, e_rt, [&](int i, uint8_t* st) {
+      const float sc = score16(reinterpret_cast<const float*>(st), qv);
+      const int k0 = (i - e_l2) * cpu;
+      const int rows = (min(n_mine, k0 + cpu) - k0) * p.Ng;
+      if (lane < rows) {
+        const int e = warp + (k0 + lane / p.Ng) * W;  // chosen chunk (rank order)
+        const int g = lane % p.Ng;
+        gkey[e * p.Ng + g] = make_key(sc, chunks[e] * p.Ng + g);
+      }
+    });
+    named_sync(kBarStream, W * 32);  // B3
+    // the kg best group keys, by rank, into glist (rank order)
+    for (int j = tid; j < n_l2; j += W * 32) {
+      const uint64_t key = gkey[j];
+      const int rank = rank_among(gkey, n_l2, key);
+      if (rank < ng) {
+        glist[rank] = key_id(key);
+        gsc[rank] = key_score(key);
+      }
+    }
+    named_sync(kBarStream, W * 32);  // B4
+
+    // ---- window and routed units
+    WarpState ws;
+    ws.init();
+    int attended = 0;
+    issue_upto(e_all);
+    if (warp == 0) {  // outputs, ascending ids, while the units load
+      int32_t* cidx = a.chunk_idx + static_cast<size_t>(item) * p.kc;
+      float* cscore = a.chunk_score ? a.chunk_score + static_cast<size_t>(item) * p.kc : nullptr;
+      for (int e = lane; e < p.kc; e += 32) {
+        if (e < ns) {
+          const int id = chunks[e];
+          int at = 0;
+          for (int f = 0; f < ns; ++f) at += chunks[f] < id;
+          cidx[at] = id;
+          if (cscore) cscore[at] = key_score(ckey[e]);
+        } else {
+          cidx[e] = -1;
+          if (cscore) cscore[e] = CUDART_NAN_F;
+        }
+      }
+      int32_t* gidx = a.group_idx + static_cast<size_t>(item) * p.kg;
+      float* gscore = a.group_score ? a.group_score + static_cast<size_t>(item) * p.kg : nullptr;
+      for (int e = lane; e < p.kg; e += 32) {
+        if (e < ng) {
+          const int id = glist[e];
+          int at = 0;
+          for (int f = 0; f < ng; ++f) at += glist[f] < id;
+          gidx[at] = id;
+          if (gscore) gscore[at] = gsc[e];
+        } else {
+          gidx[e] = -1;
+          if (gscore) gscore[e] = CUDART_NAN_F;
+        }
+      }
+    }
+    consume(e_fw, e_all, e_all, [&](int i, uint8_t* st) {
+      const uint32_t kt = ptx::smem_u32(st);
+      int valid = kUnit;
+      if (i < e_rt && warp + (i - e_fw) * W == n_forced - 1) valid = static_cast<int>(pb % kUnit) + 1;
+      attend_unit(kt, kt + kTileBytes, valid, qa, scale, ws);
+      ++attended;
+    });
+    bool drained = true;
+    if (timed_out) {
+      // A wait gave up: the partial is dropped (the output is wrong and flagged),
+      // the copies still in flight are waited for once more (bounded), and every
+      // barrier below is still reached.  Later items of this CTA are skipped.
+      if (lane == 0) {
+        flag_error(a.err, kErrTimeout);
+        s_abort = 1;
+      }
+      for (; done < issued; ++done) drained &= wait_stage(done);
+      ws.m0 = ws.m1 = -CUDART_INF_F;
+      ws.l0 = ws.l1 = 0.f;
+    }
+
+    // ---- merge the warps' partials through shared memory (each warp's stage 0)
+    const int g = lane >> 2, t4 = lane & 3;
+    ws.l0 += __shfl_xor_sync(0xffffffffu, ws.l0, 1);
+    ws.l0 += __shfl_xor_sync(0xffffffffu, ws.l0, 2);
+    ws.l1 += __shfl_xor_sync(0xffffffffu, ws.l1, 1);
+    ws.l1 += __shfl_xor_sync(0xffffffffu, ws.l1, 2);
+    float* wo = reinterpret_cast<float*>(ring);  // [16 heads][128]
+    const bool write_o = drained && attended > 0;
+    if (!write_o) {
+      ws.m0 = ws.m1 = -CUDART_INF_F;
+      ws.l0 = ws.l1 = 0.f;
+    } else {
+      // row hh, column c at hh * 128 + (c ^ ((hh & 7) << 3)): the eight rows a
+      // store touches land in different banks
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int c = (j * 8 + 2 * t4) ^ (g << 3);
+        *reinterpret_cast<float2*>(wo + g * kD + c) = make_float2(ws.o[j][0], ws.o[j][1]);
+        *reinterpret_cast<float2*>(wo + (g + 8) * kD + c) = make_float2(ws.o[j][2], ws.o[j][3]);
+      }
+    }
+    if (t4 == 0) {
+      s_ml[warp][g][0] = ws.m0;
+      s_ml[warp][g][1] = ws.l0;
+      s_ml[warp][g + 8][0] = ws.m1;
+      s_ml[warp][g + 8][1] = ws.l1;
+    }
+    named_sync(kBarStream, W * 32);
+    for (int idx = tid; idx < p.G * kD; idx += W * 32) {
+      const int hh = idx / kD, d = idx % kD;
+      float mm = -CUDART_INF_F;
+#pragma unroll
+      for (int v = 0; v < W; ++v) mm = fmaxf(mm, s_ml[v][hh][0]);
+      float ll = 0.f, oo = 0.f;
+      if (mm != -CUDART_INF_F) {
+#pragma unroll
+        for (int v = 0; v < W; ++v) {
+          const float mv = s_ml[v][hh][0];
+          if (mv == -CUDART_INF_F) continue;
+          const float f = exp2f(mv - mm);
+          ll += s_ml[v][hh][1] * f;
+          oo += reinterpret_cast<const float*>(base + static_cast<size_t>(v) * kS * kStageBytes)
+                    [hh * kD + (d ^ ((hh & 7) << 3))] * f;
+        }
+      }
+      const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + hh;
+      store_out(a.out + row * kD + d, ll > 0.f ? oo / ll : 0.f);
+      if (a.lse && d == 0) a.lse[row] = ll > 0.f ? (mm + log2f(ll)) * kLn2 : -CUDART_INF_F;
+    }
+    // the rings and the lists are reused by the next item (its copies are
+    // ordered after this item's shared-memory writes)
+    ptx::fence_proxy_async();
+    named_sync(kBarStream, W * 32);
+  }
+  cta_sync();
   pdl_trigger();
 }
 
-template <typename TO>
-cudaError_t launch_t(const LayerParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                     const ItemArgs<TO>& a, cudaStream_t s) {
-  const size_t smem = item_smem_bytes(p);
-  cudaError_t e = ensure_smem<decode_step_kernel<TO>>(smem);
+// ------------------------------------------------------------------ launch
+
+struct StepShape {
+  int W;           // streaming warps per CTA (7: one CTA per SM; 3: two per SM), plus one append warp
+  int R1;          // key registers per lane of the level-1 lists (top-kc <= 32 R1)
+  int grid;
+};
+
+StepShape step_shape(const LayerParams& p) {
+  const int64_t items = static_cast<int64_t>(p.B) * p.Hkv;
+  const int sms = device_sm_count();
+  StepShape s;
+  s.W = items <= sms ? 7 : 3;
+  s.R1 = p.kc <= 32 ? 1 : 2;
+  const int64_t slots = static_cast<int64_t>(sms) * (s.W == 7 ? 1 : 2);
+  s.grid = static_cast<int>(items < slots ? items : slots);
+  return s;
+}
+
+size_t step_smem_bytes(const LayerParams& p, int W) {
+  return StepSmem{W, summ::table_entries(p, kD)}.bytes();
+}
+
+template <int W, int R1, typename TO>
+cudaError_t launch_t(const LayerParams& p, int grid, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const StepArgs<TO>& a, cudaStream_t s) {
+  const size_t smem = step_smem_bytes(p, W);
+  cudaError_t e = ensure_smem<decode_step_kernel<W, R1, TO>>(smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_step_kernel<TO>, dim3(p.B * p.Hkv), dim3(kIT), smem, s, 1, tk, tv, a, p);
+  return launch_pdl(decode_step_kernel<W, R1, TO>, dim3(grid), dim3((W + 1) * 32), smem, s, 1,
+                    tk, tv, a, p);
+}
+
+template <typename TO>
+cudaError_t dispatch(const LayerParams& p, const StepShape& sh, const CUtensorMap& tk,
+                     const CUtensorMap& tv, const StepArgs<TO>& a, cudaStream_t s) {
+  if (sh.W == 7)
+    return sh.R1 == 1 ? launch_t<7, 1, TO>(p, sh.grid, tk, tv, a, s)
+                      : launch_t<7, 2, TO>(p, sh.grid, tk, tv, a, s);
+  return sh.R1 == 1 ? launch_t<3, 1, TO>(p, sh.grid, tk, tv, a, s)
+                    : launch_t<3, 2, TO>(p, sh.grid, tk, tv, a, s);
 }
 
 }  // namespace
@@ -370,8 +718,11 @@ cudaError_t launch_t(const LayerParams& p, const CUtensorMap& tk, const CUtensor
 bool decode_item_path(const LayerParams& p) {
   const int64_t items = static_cast<int64_t>(p.B) * p.Hkv;
   const int sms = device_sm_count();
-  return items * 2 >= sms && items <= sms && item_smem_bytes(p) <= 220 * 1024 &&
-         p.kc * p.Ng <= kScanStages * kTileRows;
+  const StepShape sh = step_shape(p);
+  // dynamic shared memory: one CTA per SM may take 225 KB, two per SM 112 KB each
+  const size_t limit = sh.W == 7 ? 225 * 1024 : 112 * 1024;
+  return items * 2 >= sms && p.kc <= kKcMax && p.kg <= kKgMax && p.Ng <= 8 &&
+         kRows % p.Ng == 0 && step_smem_bytes(p, sh.W) <= limit;
 }
 
 bool decode_step_path(const LayerParams& p, int dtype) {
@@ -380,13 +731,16 @@ bool decode_step_path(const LayerParams& p, int dtype) {
 }
 
 cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* q,
-                               const int64_t* pos, const float* chunk_sum, const float* group_sum,
+                               const int64_t* pos, float* chunk_sum, float* group_sum,
                                const void* k, const void* v, int32_t* chunk_idx,
                                float* chunk_score, int32_t* group_idx, float* group_score,
-                               void* out, float* lse, unsigned* err, cudaStream_t s) {
-  if (!decode_item_path(p)) {  // the routing kernel, then the attention kernel
-    cudaError_t e = launch_route(p, 1, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score,
-                                 group_idx, group_score, err, s);
+                               void* out, float* lse, int append, unsigned* err, cudaStream_t s) {
+  if (!decode_item_path(p)) {  // the summary append, the routing kernel, then the attention kernel
+    cudaError_t e = cudaSuccess;
+    if (append) e = launch_append_per_sequence(p, 1, k, pos, chunk_sum, group_sum, s);
+    if (e == cudaSuccess)
+      e = launch_route(p, 1, q, pos, chunk_sum, group_sum, chunk_idx, chunk_score, group_idx,
+                       group_score, err, s);
     if (e != cudaSuccess) return e;
     return launch_attend_decode_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, err, 0, s);
   }
@@ -395,15 +749,19 @@ cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* 
   cudaError_t e = make_bf16_map(&tk, k, all_rows, kUnit);
   if (e == cudaSuccess) e = make_bf16_map(&tv, v, all_rows, kUnit);
   if (e != cudaSuccess) return e;
+  const StepShape sh = step_shape(p);
+  const int n_items = p.B * p.Hkv;
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
   if (out_dtype == 0) {
-    ItemArgs<float> a{static_cast<const __nv_bfloat16*>(q), pos, chunk_sum, group_sum, chunk_idx,
-                      chunk_score, group_idx, group_score, static_cast<float*>(out), lse, err};
-    return launch_t<float>(p, tk, tv, a, s);
+    StepArgs<float> a{qb, pos, kb, static_cast<const __nv_bfloat16*>(v), chunk_sum, group_sum, chunk_idx, chunk_score, group_idx,
+                      group_score, static_cast<float*>(out), lse, err, append, n_items};
+    return dispatch<float>(p, sh, tk, tv, a, s);
   }
-  ItemArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(q), pos, chunk_sum, group_sum,
-                            chunk_idx, chunk_score, group_idx, group_score,
-                            static_cast<__nv_bfloat16*>(out), lse, err};
-  return launch_t<__nv_bfloat16>(p, tk, tv, a, s);
+  StepArgs<__nv_bfloat16> a{qb, pos, kb, static_cast<const __nv_bfloat16*>(v), chunk_sum, group_sum, chunk_idx, chunk_score, group_idx,
+                            group_score, static_cast<__nv_bfloat16*>(out), lse, err, append,
+                            n_items};
+  return dispatch<__nv_bfloat16>(p, sh, tk, tv, a, s);
 }
 
 }  // namespace hga

@@ -112,17 +112,23 @@ cudaError_t launch_route_decode(const LayerParams& p, int dtype, bool level1, bo
                                 int32_t* group_idx, float* group_score, unsigned* err,
                                 cudaStream_t s);
 
-// One decode step (routing + attention): one launch of decode_step_kernel when
-// decode_item_path (about one (sequence, KV head) item per SM), else the routing
-// and the attention kernels; applies when decode_step_path (bf16, D = 128
-// decode, device-resident K/V).
+// One decode step (optional summary append + routing + attention): one launch of
+// decode_step_kernel when decode_item_path (at least half a (sequence, KV head)
+// item per SM), else the append, routing and attention kernels; applies when
+// decode_step_path (bf16, D = 128 decode, device-resident K/V).
 bool decode_item_path(const LayerParams& p);
 bool decode_step_path(const LayerParams& p, int dtype);
 cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* q,
-                               const int64_t* pos, const float* chunk_sum, const float* group_sum,
+                               const int64_t* pos, float* chunk_sum, float* group_sum,
                                const void* k, const void* v, int32_t* chunk_idx,
                                float* chunk_score, int32_t* group_idx, float* group_score,
-                               void* out, float* lse, unsigned* err, cudaStream_t s);
+                               void* out, float* lse, int append, unsigned* err, cudaStream_t s);
+
+// The summary rows each sequence's token pos[b] closes (one warp per (sequence,
+// KV head) item; the rows hga_build_summaries(pos, pos + 1) writes, per sequence).
+cudaError_t launch_append_per_sequence(const LayerParams& p, int dtype, const void* k,
+                                       const int64_t* pos, float* chunk_sum, float* group_sum,
+                                       cudaStream_t s);
 
 // Workspace bytes of launch_attend for p (0 when the launch needs none).
 size_t attend_workspace_bytes(const LayerParams& p, int dtype);

@@ -38,9 +38,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// `max_iter` polls or 50 ms, whichever comes first, and returns false (the
-// caller flags a timeout); legitimate waits here last microseconds.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_iter) {
+// `max_iter` polls or `limit_ns` of %globaltimer, whichever comes first, and
+// returns false (the caller flags a timeout); legitimate waits here last
+// microseconds.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint32_t max_iter,
+                                             uint64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
   uint64_t t0 = 0;
   for (uint32_t i = 0; i < max_iter; ++i) {
@@ -52,13 +54,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
         : "r"(addr), "r"(parity)
         : "memory");
     if (done) return true;
-    if ((i & 1023) == 0) {
+    if ((i & 255) == 0) {
       const uint64_t now = globaltimer_ns();
       if (i == 0) t0 = now;
-      else if (now - t0 > 50000000ull) return false;
+      else if (now - t0 > limit_ns) return false;
     }
   }
   return false;
+}
+
+// mbar_wait_ns with a 50 ms limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_iter) {
+  return mbar_wait_ns(bar, parity, max_iter, 50000000ull);
 }
 
 // 2-D tiled TMA load of one box into shared memory, completing on `bar`.

@@ -325,8 +325,9 @@ route_groups_kernel(const T* __restrict__ q, const int64_t* __restrict__ pos,
 // no more CTAs in total than fit at once (4 per SM), slices of >= 32 rows.
 int chunk_cluster_size(const LayerParams& p) {
   const int64_t items = static_cast<int64_t>(p.B) * p.Hkv * p.nblk;
+  const int64_t sms = device_sm_count();
   int cl = 1;
-  while (cl < 8 && items * cl * 2 <= 148 * 4 && p.n_chunks / (cl * 2) >= 32) cl *= 2;
+  while (cl < 8 && items * cl * 2 <= sms * 4 && p.n_chunks / (cl * 2) >= 32) cl *= 2;
   return cl;
 }
 

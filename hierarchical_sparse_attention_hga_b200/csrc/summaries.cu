@@ -21,27 +21,13 @@
 // the same bits.
 #include "common.cuh"
 #include "kernels.h"
+#include "summary_math.cuh"
 
 namespace hga {
 namespace {
 
-template <typename T, int PPL> struct PairLoad;
-template <> struct PairLoad<float, 2> {
-  static __device__ __forceinline__ void run(const float* p, float (&o)[2]) { load2(p, o); }
-};
-template <> struct PairLoad<__nv_bfloat16, 2> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&o)[2]) { load2(p, o); }
-};
-template <> struct PairLoad<float, 1> {
-  static __device__ __forceinline__ void run(const float* p, float (&o)[1]) { o[0] = __ldg(p); }
-};
-template <> struct PairLoad<__nv_bfloat16, 1> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&o)[1]) {
-    o[0] = __bfloat162float(p[0]);
-  }
-};
-
-constexpr int kGroup = 16;
+using summ::PairLoad;
+using summ::kGroup;
 
 template <typename T, int D, bool PRELOAD>
 __global__ void __launch_bounds__(256)
@@ -52,7 +38,6 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   constexpr int PPL = P / 32;
   extern __shared__ float2 smem_tab[];
   __shared__ float s_gsum[8][D];             // raw group sums of one chunk
-  __shared__ double s_omega[P];
   const int n_lo = P - p.n_high;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
@@ -77,23 +62,10 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
       PairLoad<T, PPL>::run(row + P, y0[o]);
     }
   }
-  for (int i = threadIdx.x; i < n_lo; i += blockDim.x)
-    s_omega[i] = pow(p.theta, -2.0 * (p.n_high + i) / D);
-  __syncthreads();
   float2* tab_g = smem_tab;                  // [g][n_lo]: rotation by (g-1)/2 - o
   float2* tab_s = smem_tab + kGroup * n_lo;  // [Ng][n_lo]: rotation by (C-g)/2 - w*g
-  // Angles are formed in double from omega_i = theta^(-2i/D) and the exact
-  // half-integer offset, then rounded once to float for sincosf.
-  for (int idx = threadIdx.x; idx < (kGroup + p.Ng) * n_lo; idx += blockDim.x) {
-    const bool is_g = idx < kGroup * n_lo;
-    const int j = is_g ? idx : idx - kGroup * n_lo;
-    const int o = j / n_lo;
-    const double omega = s_omega[j % n_lo];
-    const double off = is_g ? 0.5 * (kGroup - 1) - o : 0.5 * (p.C - kGroup) - o * kGroup;
-    float s, c;
-    sincosf(static_cast<float>(off * omega), &s, &c);
-    smem_tab[idx] = make_float2(c, s);
-  }
+  for (int idx = threadIdx.x; idx < summ::table_entries(p, D); idx += blockDim.x)
+    smem_tab[idx] = summ::table_entry(p, D, idx);
   __syncthreads();
   pdl_wait();
 
@@ -107,8 +79,6 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
       const bool fin_g = g0 + kGroup - 1 >= t_begin && g0 + kGroup - 1 < t_end;
       if (fin_c || fin_g) {
         float gx[PPL], gy[PPL];
-#pragma unroll
-        for (int u = 0; u < PPL; ++u) gx[u] = gy[u] = 0.f;
         float x[kGroup][PPL], y[kGroup][PPL];
         if (PRELOAD && ci == static_cast<int>(blockIdx.x)) {
 #pragma unroll
@@ -126,27 +96,13 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
             PairLoad<T, PPL>::run(row + P, y[o]);
           }
         }
-#pragma unroll
-        for (int o = 0; o < kGroup; ++o) {
-#pragma unroll
-          for (int u = 0; u < PPL; ++u) {
-            const int i = lane * PPL + u;
-            if (i < p.n_high) {
-              gx[u] += x[o][u];
-              gy[u] += y[o][u];
-            } else {
-              const float2 r = tab_g[o * n_lo + i - p.n_high];
-              gx[u] += x[o][u] * r.x - y[o][u] * r.y;
-              gy[u] += x[o][u] * r.y + y[o][u] * r.x;
-            }
-          }
-        }
+        summ::group_raw_sum<PPL>(x, y, tab_g, p.n_high, n_lo, lane, gx, gy);
         if (fin_g) {
           float* dst = group_sum + ((static_cast<size_t>(bh) * p.n_chunks + c) * p.Ng + warp) * D;
 #pragma unroll
           for (int u = 0; u < PPL; ++u) {
-            dst[lane * PPL + u] = gx[u] * (1.0f / kGroup);
-            dst[P + lane * PPL + u] = gy[u] * (1.0f / kGroup);
+            dst[lane * PPL + u] = __fmul_rn(gx[u], 1.0f / kGroup);
+            dst[P + lane * PPL + u] = __fmul_rn(gy[u], 1.0f / kGroup);
           }
         }
 #pragma unroll
@@ -161,20 +117,9 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
       const float inv_c = 1.0f / p.C;
       float* dst = chunk_sum + (static_cast<size_t>(bh) * p.n_chunks + c) * D;
       for (int i = threadIdx.x; i < P; i += blockDim.x) {
-        float sx = 0.f, sy = 0.f;
-        for (int w = 0; w < p.Ng; ++w) {
-          const float gx = s_gsum[w][i], gy = s_gsum[w][P + i];
-          if (i < p.n_high) {
-            sx += gx;
-            sy += gy;
-          } else {
-            const float2 r = tab_s[w * n_lo + i - p.n_high];
-            sx += gx * r.x - gy * r.y;
-            sy += gx * r.y + gy * r.x;
-          }
-        }
-        dst[i] = sx * inv_c;
-        dst[P + i] = sy * inv_c;
+        const float2 sc = summ::chunk_pair<D>(s_gsum, tab_s, p.Ng, p.n_high, n_lo, i);
+        dst[i] = __fmul_rn(sc.x, inv_c);
+        dst[P + i] = __fmul_rn(sc.y, inv_c);
       }
     }
     __syncthreads();
@@ -193,7 +138,7 @@ cudaError_t launch_summaries_t(const LayerParams& p, const void* k, int64_t t_be
   const int c_count = c_last - c_first + 1;
   const int bh = p.B * p.Hkv;
   // enough CTAs for ~8 per SM, each looping over several chunks of one (b, h)
-  int gx = static_cast<int>((148 * 8 + bh - 1) / bh);
+  int gx = static_cast<int>((device_sm_count() * 8 + bh - 1) / bh);
   gx = gx < 1 ? 1 : (gx > c_count ? c_count : gx);
   dim3 grid(gx, bh);
   const int n_lo = D / 2 - p.n_high;
@@ -207,7 +152,47 @@ cudaError_t launch_summaries_t(const LayerParams& p, const void* k, int64_t t_be
                     group_sum);
 }
 
+// Summary append of a decode step with per-sequence positions: one warp per
+// (sequence, KV head) item writes the rows its token pos[b] closes, with the
+// batch builder's arithmetic.
+template <typename T, int D>
+__global__ void __launch_bounds__(32)
+append_kernel(const T* __restrict__ k, const int64_t* __restrict__ pos, LayerParams p,
+              float* __restrict__ chunk_sum, float* __restrict__ group_sum) {
+  extern __shared__ float2 smem_tab[];
+  __shared__ float s_gsum[8][D];
+  for (int i = threadIdx.x; i < summ::table_entries(p, D); i += 32) smem_tab[i] = summ::table_entry(p, D, i);
+  __syncwarp();
+  pdl_wait();
+  const int item = blockIdx.x;
+  const int64_t pb = pos[item / p.Hkv];
+  if (pb >= 0 && pb < p.n_alloc)
+    summ::append_closed_rows<T, D>(k + static_cast<size_t>(item) * p.n_alloc * D,
+                                   chunk_sum + static_cast<size_t>(item) * p.n_chunks * D,
+                                   group_sum + static_cast<size_t>(item) * p.n_chunks * p.Ng * D,
+                                   p, pb, smem_tab, s_gsum);
+  pdl_trigger();
+}
+
+template <typename T, int D>
+cudaError_t launch_append_t(const LayerParams& p, const void* k, const int64_t* pos,
+                            float* chunk_sum, float* group_sum, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(summ::table_entries(p, D)) * sizeof(float2);
+  return launch_pdl(append_kernel<T, D>, dim3(p.B * p.Hkv), dim3(32), smem, s, 1,
+                    static_cast<const T*>(k), pos, p, chunk_sum, group_sum);
+}
+
 }  // namespace
+
+cudaError_t launch_append_per_sequence(const LayerParams& p, int dtype, const void* k,
+                                       const int64_t* pos, float* chunk_sum, float* group_sum,
+                                       cudaStream_t s) {
+  if (dtype == 0)
+    return p.D == 64 ? launch_append_t<float, 64>(p, k, pos, chunk_sum, group_sum, s)
+                     : launch_append_t<float, 128>(p, k, pos, chunk_sum, group_sum, s);
+  return p.D == 64 ? launch_append_t<__nv_bfloat16, 64>(p, k, pos, chunk_sum, group_sum, s)
+                   : launch_append_t<__nv_bfloat16, 128>(p, k, pos, chunk_sum, group_sum, s);
+}
 
 cudaError_t launch_summaries(const LayerParams& p, int dtype, const void* k, int64_t t_begin,
                              int64_t t_end, float* chunk_sum, float* group_sum, cudaStream_t s) {

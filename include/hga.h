@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define HGA_ABI_VERSION 1
+#define HGA_ABI_VERSION 2
 
 typedef enum hga_status {
   HGA_OK = 0,
@@ -97,11 +97,25 @@ const char* hga_status_string(hga_status status);
 const char* hga_last_error(void);
 
 /*
- * Synchronises `stream`, then returns HGA_ERR_DEVICE_CHECK if any kernel of this
- * library on the current device has set the device error word since the last
- * call, and clears it; HGA_OK otherwise (HGA_ERR_CUDA if the sync failed).
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device: HGA_ERR_TIMEOUT if a kernel of this library gave up a bounded
+ * wait since the last call, else HGA_ERR_DEVICE_CHECK if a device-side argument
+ * check failed, HGA_OK otherwise (HGA_ERR_CUDA if the sync failed).  Every wait
+ * inside the kernels is bounded (a poll count and 50 ms), so a kernel always
+ * returns; the work item that gave up writes an empty result.
  */
 hga_status hga_device_status(void* stream);
+
+/*
+ * Test hook, not for production use: sets the debug flags that every later
+ * launch of this process copies (returns the previous flags; 0 = none).  Flag 1
+ * makes the one-launch kernel of hga_decode_step skip one warp's group-summary
+ * copy for the first item of each CTA while the warp still waits for it, so that
+ * bounded wait (nothing is in flight into that stage; limited to 2 ms under this
+ * flag) runs out; the kernel still reaches every barrier and returns, and
+ * hga_device_status() then reports HGA_ERR_TIMEOUT.
+ */
+int32_t hga_debug_inject(int32_t flags);
 
 /*
  * Bytes of device workspace hga_attend needs for (cfg, n_alloc, q_len).  Zero
@@ -266,30 +280,52 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
                       void* stream);
 
 /*
- * Steps 2-5 of one decode step: level-1 and level-2 routing (HGA technical
- * summary, "Metodologia -> Meccanismo Core", item 2), then the gather and exact
- * attention of the chosen tokens (item 4).  It writes what hga_route followed by
- * hga_attend writes: chunk_idx, group_idx and the scores bit for bit, out and lse
- * up to the bf16 rounding of the softmax weights (the units are attended in
- * another grouping).
+ * One whole decode step: the summary append (HGA technical summary,
+ * "Metodologia -> Meccanismo Core", item 3), level-1 and level-2 routing (item
+ * 2), then the gather and exact attention of the chosen tokens (item 4).  It
+ * writes what hga_build_summaries (per sequence, for the rows token pos[b]
+ * closes), hga_route and hga_attend write: the summary rows bit for bit,
+ * chunk_idx, group_idx and the scores bit for bit, out and lse up to the bf16
+ * rounding of the softmax weights (the units are attended in another
+ * grouping).
  *
- * When the batch holds about one (sequence, KV head) item per SM (B * Hkv
- * between half the SM count and the SM count), the step is one launch: one CTA
- * per item streams its chunk summaries with bulk copies, attends the sink,
- * local and current chunks while the chosen chunks' group summaries load, then
- * routes level 2 and attends the routed groups.  Other batches get hga_route's
- * and hga_attend's kernels, launched by this call.  Decode only (q_len is 1):
- * bf16 K/V in device memory (kv_loc HGA_KV_DEVICE), head_dim 128, group 16, at
- * most 16 query heads per KV head, topk_groups <= 1024; other shapes return
- * HGA_ERR_UNSUPPORTED (use hga_route + hga_attend).  Arguments and layouts are
- * those of hga_route and hga_attend; chunk_score, group_score and lse may be
- * NULL.  No workspace.
+ * With append != 0, for every sequence b the summary rows whose last token is
+ * pos[b] (the group pos[b] ends, and its chunk when pos[b] ends that too) are
+ * computed from k and stored in chunk_sum / group_sum; those rows belong to
+ * the current chunk, which the step attends in full and never routes.  With
+ * append == 0 the tables are only read.
+ *
+ * When the batch holds at least half a (sequence, KV head) item per SM, the
+ * step is one launch: each CTA works through items (one at a time; one CTA per
+ * SM up to one item per SM, two per SM above); its warps stream the candidate
+ * chunk summaries and the K/V units of the always-visible chunks through
+ * shared-memory rings, one warp merges the level-1 picks and runs level 2
+ * while the others attend, then all attend the routed groups, and another warp
+ * does the summary append.  Smaller batches get the append, routing and
+ * attention kernels, launched by this call (hga_decode_step_launches says
+ * which).  Decode only (q_len is 1): bf16 K/V in device memory (kv_loc
+ * HGA_KV_DEVICE), head_dim 128, group 16, at most 16 query heads per KV head,
+ * topk_groups <= 1024 (the one-launch kernel: topk_chunks <= 64 and
+ * topk_groups <= 128); other shapes return HGA_ERR_UNSUPPORTED (use hga_route +
+ * hga_attend).  Arguments and layouts are those of hga_build_summaries,
+ * hga_route and hga_attend; chunk_score, group_score and lse may be NULL.  No
+ * workspace.
  */
 hga_status hga_decode_step(const hga_config* cfg, const void* q, const int64_t* pos,
-                           const float* chunk_sum, const float* group_sum, int64_t n_alloc,
-                           const void* k, const void* v, int32_t* chunk_idx, float* chunk_score,
+                           float* chunk_sum, float* group_sum, int64_t n_alloc, const void* k,
+                           const void* v, int32_t* chunk_idx, float* chunk_score,
                            int32_t* group_idx, float* group_score, void* out, float* lse,
-                           void* stream);
+                           int32_t append, void* stream);
+
+/*
+ * How many kernel launches hga_decode_step makes for (cfg, n_alloc) on the
+ * current device: 1 when it runs the one-launch kernel (routing and attention
+ * of every (sequence, KV head) item in one grid), 2 when it launches the
+ * routing kernel and then the attention kernel.  A pure host query (it reads
+ * the device's SM count); no launch.  Returns HGA_ERR_UNSUPPORTED for shapes
+ * hga_decode_step does not take.
+ */
+hga_status hga_decode_step_launches(const hga_config* cfg, int64_t n_alloc, int32_t* launches);
 
 /*
  * hga_attend for callers that cannot allocate device memory.  The paper has no

@@ -1,7 +1,8 @@
-"""hga_decode_step against hga_route + hga_attend and the oracle.
+"""hga_decode_step against hga_build_summaries + hga_route + hga_attend and the oracle.
 
-Batches with about one (sequence, KV head) item per SM run the one-launch kernel
-(one CTA per item); smaller and larger batches run the routing and attention
+Batches with at least half a (sequence, KV head) item per SM run the one-launch
+kernel (one CTA per SM up to one item per SM, two CTAs per SM above, each
+working through items); smaller batches run the append, routing and attention
 kernels through the same call.  The one-launch kernel scores with the routing
 kernel's arithmetic, so the routed indices and scores must be bit-identical.  Its
 warps attend the units in another grouping, so the running maxima against which P
@@ -147,3 +148,115 @@ def test_decode_step_one_cta_per_item(name, kw):
     check_same_routing_close_output(sep, fus, 1e-2)
     for b in (0, 1, 2, wl.batch - 1):
         compare_head(wl, x, fus, b, 0)
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("wide_head_decode_64k", dict(batch=32, context=4096)),                    # 256 items: 2 CTAs/SM
+    ("wide_head_decode_64k", dict(batch=12, context=8192, topk_chunks=64, topk_groups=128)),
+    ("wide_head_decode_64k", dict(batch=12, context=8192, chunk=128, topk_chunks=32,
+                                  topk_groups=64)),
+])
+def test_decode_step_one_launch_wide_shapes(name, kw):
+    """More items than SMs (persistent CTAs, two per SM), and the widest routing lists
+    (top-64 chunks / top-128 groups; C = 128 with top-32 / top-64)."""
+    wl = S.workload(name, **kw)
+    x = S.make_inputs(wl, 34)
+    rng = np.random.default_rng(6)
+    pos = rng.integers(wl.chunk, wl.context, size=wl.batch)
+    pos[0], pos[1] = wl.context - 1, 3 * wl.chunk + 9
+    x["pos"] = pos.astype(np.int64)
+    assert B.hga_decode_step_launches(layer_of(wl), wl.context) == 1
+    sep, fus = run_both(wl, x)
+    check_same_routing_close_output(sep, fus, 1e-2)
+    for b in (0, 1, wl.batch - 1):
+        compare_head(wl, x, fus, b, wl.heads_kv - 1)
+
+
+@pytest.mark.parametrize("batch", [2, 10])
+def test_decode_step_append_is_bitwise_the_batch_build(batch):
+    """With append, hga_decode_step writes the summary rows each sequence's token closes
+    (a group; a group and its chunk; nothing), bit for bit as hga_build_summaries does,
+    on the one-launch kernel (batch 10: 80 items) and on the kernel sequence (batch 2)."""
+    wl = S.workload("llama3_8b_decode_32k", batch=batch, context=4096, needles=0)
+    x = S.make_inputs(wl, 35)
+    n = wl.context
+    pos = np.array([n - 1, 2 * 64 * 9 + 15, 1000, 64 * 20 - 1, 64 * 33 + 47, 3000, 16 * 100 - 1,
+                    64 * 50 + 31, 2048 + 63, 4000][:batch], dtype=np.int64)
+    x["pos"] = pos
+    layer = layer_of(wl)
+    assert B.hga_decode_step_launches(layer, n) == (1 if batch == 10 else 2)
+    bh, nc, ng = wl.batch * wl.heads_kv, n // wl.chunk, wl.chunk // wl.group
+    q, k, v = (to_device(x[t], wl.dtype) for t in ("q", "k", "v"))
+    pos_t = torch.as_tensor(pos, device="cuda")
+    full_c = torch.full((bh, nc, wl.head_dim), float("nan"), device="cuda")
+    full_g = torch.full((bh, nc, ng, wl.head_dim), float("nan"), device="cuda")
+    B.hga_build_summaries(layer, k, n, 0, n, full_c, full_g)
+    # every sequence's tables as a decode loop holds them before its token: rows closed
+    # by the token itself or later are unset (NaN)
+    cs, gs = full_c.clone(), full_g.clone()
+    for b in range(batch):
+        p = int(pos[b])
+        rows = slice(b * wl.heads_kv, (b + 1) * wl.heads_kv)
+        cs[rows, (p + 1) // wl.chunk - (1 if (p + 1) % wl.chunk == 0 else 0):] = float("nan")
+        gs_flat = gs[rows].reshape(wl.heads_kv, nc * ng, wl.head_dim)
+        gs_flat[:, (p + 1) // wl.group - (1 if (p + 1) % wl.group == 0 else 0):] = float("nan")
+        gs[rows] = gs_flat.reshape(wl.heads_kv, nc, ng, wl.head_dim)
+    ci = torch.empty((bh, 1, wl.topk_chunks), dtype=torch.int32, device="cuda")
+    gi = torch.empty((bh, 1, wl.topk_groups), dtype=torch.int32, device="cuda")
+    out = torch.empty((wl.batch, wl.heads_q, 1, wl.head_dim), device="cuda")
+    B.hga_decode_step(layer, q, pos_t, cs, gs, n, k, v, ci, gi, out, append=True)
+    torch.cuda.synchronize()
+    assert B.hga_device_status() == 0
+    for b in range(batch):
+        p = int(pos[b])
+        rows = slice(b * wl.heads_kv, (b + 1) * wl.heads_kv)
+        c_done = (p + 1) // wl.chunk        # chunk rows complete through the token
+        g_done = (p + 1) // wl.group
+        got_c, want_c = cs[rows, :c_done], full_c[rows, :c_done]
+        assert torch.equal(got_c.view(torch.int32), want_c.view(torch.int32)), b
+        got_g = gs[rows].reshape(wl.heads_kv, nc * ng, -1)[:, :g_done]
+        want_g = full_g[rows].reshape(wl.heads_kv, nc * ng, -1)[:, :g_done]
+        assert torch.equal(got_g.view(torch.int32), want_g.view(torch.int32)), b
+        assert torch.isnan(cs[rows, c_done:]).all() and \
+            torch.isnan(gs[rows].reshape(wl.heads_kv, nc * ng, -1)[:, g_done:]).all()
+    # the step's routing and output are those of the separate calls on the full tables
+    sep, fus = run_both(wl, x)
+    assert np.array_equal(ci.cpu().numpy().reshape(sep["chunk_idx"].shape), sep["chunk_idx"])
+    assert np.array_equal(gi.cpu().numpy().reshape(sep["group_idx"].shape), sep["group_idx"])
+    np.testing.assert_allclose(out.cpu().numpy(), sep["out"], atol=1e-2, rtol=0)
+
+
+def test_decode_step_bounded_wait_times_out_and_recovers():
+    """A wait that runs out ends the kernel with HGA_ERR_TIMEOUT instead of hanging.
+
+    The debug hook makes one warp skip a group-summary copy it then waits for
+    (nothing is in flight into that stage); the wait gives up after 2 ms, the
+    item's partial is dropped and every barrier is still reached.  The next call
+    without the hook is correct again.
+    """
+    wl = S.workload("llama3_8b_decode_32k", batch=10, context=2048, needles=0)
+    x = S.make_inputs(wl, 36)
+    layer = layer_of(wl)
+    assert B.hga_decode_step_launches(layer, wl.context) == 1
+    n = wl.context
+    bh, nc, ng = wl.batch * wl.heads_kv, n // wl.chunk, wl.chunk // wl.group
+    q, k, v = (to_device(x[t], wl.dtype) for t in ("q", "k", "v"))
+    pos = torch.as_tensor(x["pos"], device="cuda")
+    cs = torch.empty((bh, nc, wl.head_dim), device="cuda")
+    gs = torch.empty((bh, nc, ng, wl.head_dim), device="cuda")
+    B.hga_build_summaries(layer, k, n, 0, n, cs, gs)
+    ci = torch.empty((bh, 1, wl.topk_chunks), dtype=torch.int32, device="cuda")
+    gi = torch.empty((bh, 1, wl.topk_groups), dtype=torch.int32, device="cuda")
+    out = torch.empty((wl.batch, wl.heads_q, 1, wl.head_dim), device="cuda")
+    assert B.hga_device_status() == 0
+    old = B.hga_debug_inject(1)
+    try:
+        B.hga_decode_step(layer, q, pos, cs, gs, n, k, v, ci, gi, out)
+        torch.cuda.synchronize()
+    finally:
+        B.hga_debug_inject(old)
+    assert B.hga_device_status() == 5  # HGA_ERR_TIMEOUT
+    assert B.hga_device_status() == 0  # read and cleared
+    sep, fus = run_both(wl, x)
+    check_same_routing_close_output(sep, fus, 1e-2)
+    compare_head(wl, x, fus, 0, 0)

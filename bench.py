@@ -1,14 +1,20 @@
-"""Benchmark of the HGA decode hot path on B200.
+"""Benchmark of the HGA hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--batch B]
+                    [--layers L] [--no-workloads]
     python bench.py --impl reference ...      # the float64 CPU oracle, timed on host cores
 
-One step = one decode step of one attention layer for the whole batch: append
-the new token's summary rows, route chunks, route groups, attend (steps 1-5 of
-the HGA hot path), on inputs already resident in HBM.  The append writes rows
-of the current chunk only, which the same step never routes, so it runs on a
-side stream beside the routing/attention chain (one CUDA graph per step).  L2 is flushed (a 256 MB
-write) before every timed step, outside the timed events.  Prints one JSON line.
+One step = one decode step of a stack of L attention layers for the whole batch:
+in every layer, append the new token's summary rows, route chunks, route groups
+and attend (steps 1-5 of the HGA hot path), on inputs already resident in HBM.
+Every layer has its own K/V cache and summary tables, so no layer reads what
+another one brought into L2; the layers run back to back in one CUDA graph, as
+a model's decode step runs them, and the attention time per layer is the step
+time over L.  L2 is flushed (a 256 MB write, then a 256 MB read so that no dirty
+line is left to write back) before every timed step, outside the timed events.
+Prints one JSON line; with one GPU and the default workload it also carries a
+`workloads` key with the prefill, wide-head, host-tier and small-batch decode
+workloads, each measured the same way.
 
 Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch of
 independent sequences (weak scaling, no collective on the data path); the
@@ -45,8 +51,12 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b_decode_32k")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--context", type=int, default=None, help="override the context length")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="attention layers per decode step (0: 4, or 1 for the host tier)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads' sub-records")
     return ap.parse_args()
 
 
@@ -233,291 +243,334 @@ def job_rate(units_per_rank: float, world: int, ms_step: float) -> float:
 
 # ------------------------------------------------------------------ CUDA arm
 
-def run_hga(args, rank: int, world: int):
+
+# ------------------------------------------------------------------ inputs
+
+L2_NOTE = ("flushed before every timed step: a 256 MB write, then a 256 MB read "
+           "(no dirty line left for the timed step to write back)")
+
+
+class Flush:
+    """Evicts L2 (126 MB) before a timed step: writes one buffer larger than L2,
+    then reads another, so the timed step starts with a clean L2 holding none of
+    its inputs."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+
+def host_to_device(a, wl, dev):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16 if wl.dtype == "bf16" else np.float32))
+    return (t.view(torch.bfloat16) if wl.dtype == "bf16" else t).to(dev)
+
+
+def device_inputs(wl: S.Workload, seed: int, dev):
+    """Inputs of the workload's shape drawn on the device (torch's generator): q, k,
+    v ~ N(0,1) stored as bf16, with the workload's log-normal key norms.  Used
+    for the large sub-workloads, whose host generation would take minutes; the
+    work of a step does not depend on the values (the routing always keeps kc
+    chunks and kg groups)."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    bf = torch.bfloat16
+    q_len = wl.context if wl.prefill else 1
+    q = torch.empty(wl.batch, wl.heads_q, q_len, wl.head_dim, dtype=bf, device=dev)
+    k = torch.empty(wl.batch, wl.heads_kv, wl.context, wl.head_dim, dtype=bf, device=dev)
+    v = torch.empty_like(k)
+    for b in range(wl.batch):
+        q[b] = torch.randn(q[b].shape, generator=gen, device=dev).to(bf)
+        kb = torch.randn(k[b].shape, generator=gen, device=dev)
+        if wl.lognormal_sigma:
+            kb *= torch.exp(wl.lognormal_sigma *
+                            torch.randn(wl.heads_kv, wl.context, 1, generator=gen, device=dev))
+        k[b] = kb.to(bf)
+        v[b] = torch.randn(v[b].shape, generator=gen, device=dev).to(bf)
+    pos = torch.full((wl.batch,), wl.context - 1, dtype=torch.int64, device=dev)
+    return q, k, v, pos
+
+
+def make_layer(B, wl, out_dtype):
+    return B.Layer(batch=wl.batch, heads_q=wl.heads_q, heads_kv=wl.heads_kv, head_dim=wl.head_dim,
+                   chunk=wl.chunk, group=wl.group, sink_chunks=wl.sink, local_chunks=wl.local,
+                   topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
+                   n_high_pairs=wl.n_high_pairs, rope_theta=wl.rope_theta,
+                   dtype=B.HGA_BF16 if wl.dtype == "bf16" else B.HGA_F32, out_dtype=out_dtype)
+
+
+def timed_graph(g, iters, flush, stream):
+    """Mean ms of `iters` replays of graph g, each after an L2 flush (outside the events)."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    for a_, b_ in ev:
+        flush()
+        a_.record(stream)
+        g.replay()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    return sum(a_.elapsed_time(b_) for a_, b_ in ev) / iters
+
+
+def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, world: int,
+                  ranks, seed: int, x=None, compare: bool = True) -> dict:
+    """One decode workload: the timed L-layer step, per-call times, the roofline of
+    the dominant kernel, the end-to-end rate through host buffers and clocks."""
     import torch
     from hierarchical_sparse_attention_hga_b200 import binding as B
-    from hierarchical_sparse_attention_hga_b200.build import build
 
-    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-    build()
-    B.load_library()
-    wl = S.workload(args.workload)
-    if args.batch:
-        wl = wl.with_(batch=args.batch)
-    if args.context:
-        wl = wl.with_(context=args.context)
-    if wl.prefill:
-        return run_prefill(args, rank, world, wl)
     dev = torch.device("cuda")
-    seed = rank_seed(args.workload, rank)
-    x = S.make_inputs(wl, seed)
     n = wl.context
     p = n - 1
-
-    def to_dev(a):
-        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16 if wl.dtype == "bf16" else np.float32))
-        return (t.view(torch.bfloat16) if wl.dtype == "bf16" else t).to(dev)
-
-    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
-    pos = torch.as_tensor(x["pos"], device=dev)
-    layer = B.Layer(batch=wl.batch, heads_q=wl.heads_q, heads_kv=wl.heads_kv, head_dim=wl.head_dim,
-                    chunk=wl.chunk, group=wl.group, sink_chunks=wl.sink, local_chunks=wl.local,
-                    topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
-                    n_high_pairs=wl.n_high_pairs, rope_theta=wl.rope_theta,
-                    dtype=B.HGA_BF16 if wl.dtype == "bf16" else B.HGA_F32, out_dtype=B.HGA_F32)
+    hot = wl.name.startswith("host_tier")
+    if x is not None:
+        q0, k0, v0 = (host_to_device(x[t], wl, dev) for t in ("q", "k", "v"))
+        pos = torch.as_tensor(x["pos"], device=dev)
+        data = ("synthetic (seeded N(0,1) q/k/v from the host generator" +
+                (f"; {wl.needles} needle chunks per KV head" if wl.needles else "") + ")")
+    else:
+        q0, k0, v0, pos = device_inputs(wl, seed, dev)
+        data = ("synthetic (N(0,1) q/k/v drawn on the device" +
+                (f"; log-normal key norms, sigma {wl.lognormal_sigma}" if wl.lognormal_sigma else "") + ")")
+    layer = make_layer(B, wl, B.HGA_F32)
     bh = wl.batch * wl.heads_kv
     nc, ng = n // wl.chunk, wl.chunk // wl.group
-    # Host tier: the whole K/V cache in pinned host memory; the GPU keeps the
-    # summaries and a working buffer (windows + the step's routed groups).
-    hot = wl.name.startswith("host_tier")
-    if hot:
-        layer.kv_loc = B.HGA_KV_HOST_PINNED
-        k_host, v_host = k.cpu().pin_memory(), v.cpu().pin_memory()
-        del k, v
-        torch.cuda.empty_cache()
-        rows = B.hga_hot_rows(layer)
-        k_work = torch.empty(bh, rows, wl.head_dim, dtype=torch.bfloat16, device=dev)
-        v_work = torch.empty_like(k_work)
-        k_src, v_src = k_host, v_host
-    else:
-        k_src, v_src = k, v
-    cs = torch.empty(bh, nc, wl.head_dim, device=dev)
-    gs = torch.empty(bh, nc, ng, wl.head_dim, device=dev)
-    ci = torch.empty(bh, wl.topk_chunks, dtype=torch.int32, device=dev)
-    gi = torch.empty(bh, wl.topk_groups, dtype=torch.int32, device=dev)
-    out = torch.empty(wl.batch, wl.heads_q, 1, wl.head_dim, device=dev)
-    lse = torch.empty(wl.batch, wl.heads_q, 1, device=dev)
-    wsb = B.hga_workspace_size(layer, n, 1)
-    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = Flush(dev)
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
-    # prefix summaries (setup, untimed): every row closed before the new token
-    B.hga_build_summaries(layer, k_src, n, 0, p, cs, gs, stream=sh)
-    if hot:  # fill the working buffer's windows once
-        B.hga_route(layer, q, 1, pos, cs, gs, n, ci, gi, stream=sh)
-        B.hga_gather_host(layer, k_host, v_host, n, pos, gi, k_work, v_work, refresh_window=True,
-                          stream=sh)
 
-    parts = {
-        "summaries": lambda st: B.hga_build_summaries(layer, k_src, n, p, p + 1, cs, gs, stream=st),
-        "route": lambda st: B.hga_route(layer, q, 1, pos, cs, gs, n, ci, gi, stream=st),
-        "attend": lambda st: B.hga_attend(layer, q, 1, pos, k_work if hot else k_src,
-                                          v_work if hot else v_src, n, gi, out, lse, ws, wsb,
-                                          stream=st),
-        "route_chunks": lambda st: B.hga_route_chunks(layer, q, 1, pos, cs, n, ci, stream=st),
-        "route_groups": lambda st: B.hga_route_groups(layer, q, 1, pos, gs, n, ci, gi, stream=st),
-    }
+    # every layer: its own caches, summaries, routing buffers and outputs
+    L_ = []
+    for li in range(layers):
+        q, k, v = (q0, k0, v0) if li == 0 else (q0.clone(), k0.clone(), v0.clone())
+        d = dict(q=q, k=k, v=v,
+                 cs=torch.empty(bh, nc, wl.head_dim, device=dev),
+                 gs=torch.empty(bh, nc, ng, wl.head_dim, device=dev),
+                 ci=torch.empty(bh, wl.topk_chunks, dtype=torch.int32, device=dev),
+                 gi=torch.empty(bh, wl.topk_groups, dtype=torch.int32, device=dev),
+                 out=torch.empty(wl.batch, wl.heads_q, 1, wl.head_dim, device=dev),
+                 lse=torch.empty(wl.batch, wl.heads_q, 1, device=dev))
+        L_.append(d)
+    del q0, k0, v0
+    if hot:  # the whole K/V cache in pinned host memory; the GPU keeps summaries and windows
+        layer.kv_loc = B.HGA_KV_HOST_PINNED
+        d = L_[0]
+        d["k_host"], d["v_host"] = d["k"].cpu().pin_memory(), d["v"].cpu().pin_memory()
+        del d["k"], d["v"]
+        torch.cuda.empty_cache()
+        rows = B.hga_hot_rows(layer)
+        d["k_work"] = torch.empty(bh, rows, wl.head_dim, dtype=torch.bfloat16, device=dev)
+        d["v_work"] = torch.empty_like(d["k_work"])
+    wsb = B.hga_workspace_size(layer, n, 1)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+    for d in L_:  # prefix summaries (setup, untimed): every row closed before the new token
+        k_src = d["k_host"] if hot else d["k"]
+        B.hga_build_summaries(layer, k_src, n, 0, p, d["cs"], d["gs"], stream=sh)
     if hot:
-        parts["gather"] = lambda st: B.hga_gather_host(layer, k_host, v_host, n, pos, gi, k_work,
-                                                       v_work, stream=st)
-    # routing and attention in one launch (bf16, D = 128, K/V in device memory)
-    fused = not hot and wl.dtype == "bf16" and wl.head_dim == 128 and wl.group == 16 and wl.gqa <= 16
-    if fused:  # the whole step: summary append, routing and attention
-        parts["decode_step"] = lambda st: B.hga_decode_step(layer, q, pos, cs, gs, n, k_src, v_src,
-                                                            ci, gi, out, lse, append=True,
-                                                            stream=st)
+        d = L_[0]
+        B.hga_route(layer, d["q"], 1, pos, d["cs"], d["gs"], n, d["ci"], d["gi"], stream=sh)
+        B.hga_gather_host(layer, d["k_host"], d["v_host"], n, pos, d["gi"], d["k_work"],
+                          d["v_work"], refresh_window=True, stream=sh)
 
+    def parts_of(d):
+        k_src, v_src = (d["k_host"], d["v_host"]) if hot else (d["k"], d["v"])
+        k_att, v_att = (d["k_work"], d["v_work"]) if hot else (d["k"], d["v"])
+        pr = {
+            "summaries": lambda st: B.hga_build_summaries(layer, k_src, n, p, p + 1, d["cs"], d["gs"],
+                                                          stream=st),
+            "route": lambda st: B.hga_route(layer, d["q"], 1, pos, d["cs"], d["gs"], n, d["ci"],
+                                            d["gi"], stream=st),
+            "attend": lambda st: B.hga_attend(layer, d["q"], 1, pos, k_att, v_att, n, d["gi"],
+                                              d["out"], d["lse"], ws, wsb, stream=st),
+            "route_chunks": lambda st: B.hga_route_chunks(layer, d["q"], 1, pos, d["cs"], n, d["ci"],
+                                                          stream=st),
+            "route_groups": lambda st: B.hga_route_groups(layer, d["q"], 1, pos, d["gs"], n, d["ci"],
+                                                          d["gi"], stream=st),
+        }
+        if hot:
+            pr["gather"] = lambda st: B.hga_gather_host(layer, d["k_host"], d["v_host"], n, pos,
+                                                        d["gi"], d["k_work"], d["v_work"], stream=st)
+        else:
+            # the whole step in one call: summary append, routing and attention
+            pr["decode_step"] = lambda st: B.hga_decode_step(layer, d["q"], pos, d["cs"], d["gs"], n,
+                                                             d["k"], d["v"], d["ci"], d["gi"],
+                                                             d["out"], d["lse"], append=True,
+                                                             stream=st)
+        return pr
+
+    parts_l = [parts_of(d) for d in L_]
+    parts = parts_l[0]
     side = torch.cuda.Stream()
 
-    def make_step(chain):
+    def chain_step(pr, chain):
+        """The append on a side stream beside a routing/attention chain (the rows the
+        new token closes belong to the current chunk, which the step never routes)."""
         def step(st):
-            # The rows the new token closes belong to the current chunk, which
-            # this step never routes (it is always visible), so the append runs
-            # on a side stream, concurrently with routing and attention.
-            main = torch.cuda.current_stream()
-            side.wait_stream(main)
+            main_s = torch.cuda.current_stream()
+            side.wait_stream(main_s)
             with torch.cuda.stream(side):
-                parts["summaries"](side.cuda_stream)
+                pr["summaries"](side.cuda_stream)
             for name in chain:
-                parts[name](st)
-            main.wait_stream(side)
+                pr[name](st)
+            main_s.wait_stream(side)
         return step
 
     if hot:
-        step = make_step(("route", "gather", "attend"))
-        step2 = step
-        step4 = make_step(("route_chunks", "route_groups", "gather", "attend"))
+        one_layer = chain_step(parts, ("route", "gather", "attend"))
+        step = one_layer
+        comparisons = {"four_call_step_us": chain_step(parts, ("route_chunks", "route_groups",
+                                                                "gather", "attend"))}
     else:
-        # The timed step: hga_decode_step with the summary append (one launch when the
-        # batch has at least half a (sequence, KV head) item per SM, else the append,
-        # routing and attention kernels); the two-call and four-call steps (append on a
-        # side stream) are reported beside it.
-        step2 = make_step(("route", "attend"))
-        step = parts["decode_step"] if fused else step2
-        step4 = make_step(("route_chunks", "route_groups", "attend"))
+        def step(st):
+            for pr in parts_l:
+                pr["decode_step"](st)
+        comparisons = {"two_call_step_us": chain_step(parts, ("route", "attend")),
+                       "four_call_step_us": chain_step(parts, ("route_chunks", "route_groups",
+                                                               "attend"))} if compare else {}
 
-    # eager warm-up, then one CUDA graph for the whole step and one per call
-    for _ in range(max(1, args.warmup)):
+    for _ in range(max(1, warmup)):
         step(sh)
     torch.cuda.synchronize()
     assert B.hga_device_status(sh) == 0
     graphs = {}
-    steps = [("step", step), ("step2", step2), ("step4", step4)]
-    for name, fn in list(parts.items()) + steps:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+    for name, fn in [("step", step)] + list(comparisons.items()) + list(parts.items()):
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_):
             fn(torch.cuda.current_stream().cuda_stream)
-        graphs[name] = g
+        graphs[name] = g_
     torch.cuda.synchronize()
-
-    def timed(g, iters):
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(iters)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(iters)]
-        for i in range(iters):
-            flush.zero_()              # L2 flush, outside the timed events
-            starts[i].record(stream)
-            g.replay()
-            ends[i].record(stream)
-        return starts, ends
-
-    for _ in range(args.warmup):
-        flush.zero_()
+    for _ in range(warmup):
+        flush()
         graphs["step"].replay()
-    ranks = Ranks(world, dev)
     torch.cuda.synchronize()
     ranks.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        starts, ends = timed(graphs["step"], args.steps)
-        torch.cuda.synchronize()
+        ms_step = timed_graph(graphs["step"], steps, flush, stream)
     ranks.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    ms_step = sum(step_ms) / len(step_ms)
-    a4, b4 = timed(graphs["step4"], min(args.steps, 200))
-    torch.cuda.synchronize()
-    ms_step4 = sum(x.elapsed_time(y) for x, y in zip(a4, b4)) / len(a4)
-    a2, b2 = timed(graphs["step2"], min(args.steps, 200))
-    torch.cuda.synchronize()
-    ms_step2 = sum(x.elapsed_time(y) for x, y in zip(a2, b2)) / len(a2)
     ms_step = ranks.max(ms_step)
     assert B.hga_device_status(sh) == 0
-    # timing floor: an empty graph-sized launch measured the same way
-    g_floor = torch.cuda.CUDAGraph()
-    dummy = torch.zeros(1, device=dev)
-    with torch.cuda.graph(g_floor):
-        dummy.add_(1)
-    a_, b_ = timed(g_floor, 50)
-    torch.cuda.synchronize()
-    floor_us = 1e3 * sum(x.elapsed_time(y) for x, y in zip(a_, b_)) / len(a_)
-    # per-call breakdown: each call's graph replayed alone after an L2 flush
-    ms = {}
-    for name in parts:
-        a_, b_ = timed(graphs[name], min(args.steps, 200))
-        torch.cuda.synchronize()
-        ms[name] = sum(x.elapsed_time(y) for x, y in zip(a_, b_)) / len(a_)
+    n_side = min(steps, 100)
+    side_ms = {name: timed_graph(graphs[name], n_side, flush, stream) for name in comparisons}
+    ms = {name: timed_graph(graphs[name], n_side, flush, stream) for name in parts}
 
-    # ---- e2e: host (pinned) q and new K/V rows in, output back, every step
-    q_host = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).pin_memory() \
-        if wl.dtype == "bf16" else torch.from_numpy(x["q"]).pin_memory()
-    kv_new = torch.empty(2, wl.batch, wl.heads_kv, wl.head_dim, dtype=torch.bfloat16).pin_memory()
-    kv_new[0].copy_(k_src[:, :, p].cpu())
-    kv_new[1].copy_(v_src[:, :, p].cpu())
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    qv = q.view(torch.int16) if wl.dtype == "bf16" else q
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e = []
-    for i in range(args.warmup + min(args.steps, 200)):
-        flush.zero_()
-        e0.record(stream)
-        qv.copy_(q_host, non_blocking=True)
-        if hot:  # the new token's K/V goes into the host cache, a host-side write
-            k_host[:, :, p].copy_(kv_new[0])
-            v_host[:, :, p].copy_(kv_new[1])
-        else:
-            k_src[:, :, p].copy_(kv_new[0], non_blocking=True)
-            v_src[:, :, p].copy_(kv_new[1], non_blocking=True)
-        graphs["step"].replay()
-        out_host.copy_(out, non_blocking=True)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= args.warmup:
-            e2e.append(e0.elapsed_time(e1))
-    ms_e2e = sum(e2e) / len(e2e)
-    ms_e2e = ranks.max(ms_e2e)
-    h2d = q_host.numel() * q_host.element_size() + (0 if hot else kv_new.numel() * kv_new.element_size())
-    d2h = out_host.numel() * out_host.element_size()
-
+    # roofline kernel: CUDA events around direct launches queued behind the flush
+    # (the host enqueues them while the flush runs, so the events bracket GPU work)
     nb = step_bytes(wl)
     nb["route"] = nb["route_chunks"] + nb["route_groups"]
-    # one launch reads the query rows once
     nb["decode_step"] = nb["summaries"] + nb["route"] + nb["attend"] - \
-        2 * wl.batch * wl.heads_kv * wl.gqa * wl.head_dim * (2 if wl.dtype == "bf16" else 4)
-    # the library says whether hga_decode_step is its one-launch kernel for this shape
-    one_launch = fused and B.hga_decode_step_launches(layer, n) == 1
-    kern = "decode_step" if one_launch else max(("route", "attend"), key=lambda kk: ms[kk])
+        2 * bh * wl.gqa * wl.head_dim * (2 if wl.dtype == "bf16" else 4)
+    one_launch = not hot and B.hga_decode_step_launches(layer, n) == 1
+    if one_launch:
+        kern = "decode_step"
+    else:
+        kern = max(("route", "attend"), key=lambda kk: ms[kk])
     kernel_name = {"decode_step": "decode_step_kernel", "route": "route_decode_kernel",
                    "attend": "attend_decode_bf16_kernel"}[kern]
-    # The roofline kernel's duration: CUDA events on the launch stream around a direct
-    # launch queued behind the L2 flush (the host enqueues the call while the flush
-    # runs, so the events bracket the GPU work, without the graph launch latency
-    # that the per-call graph replays above include).
-    n_direct = min(args.steps, 200)
-    ds = [torch.cuda.Event(enable_timing=True) for _ in range(n_direct)]
-    de = [torch.cuda.Event(enable_timing=True) for _ in range(n_direct)]
-    for i in range(n_direct):
-        flush.zero_()
+    lay = layers if kern == "decode_step" else 1
+    ds = [torch.cuda.Event(enable_timing=True) for _ in range(n_side)]
+    de = [torch.cuda.Event(enable_timing=True) for _ in range(n_side)]
+    for i in range(n_side):
+        flush()
         ds[i].record(stream)
-        parts[kern](sh)
+        for pr in parts_l[:lay]:
+            pr[kern](sh)
         de[i].record(stream)
     torch.cuda.synchronize()
-    kern_ms = ranks.max(sum(x.elapsed_time(y) for x, y in zip(ds, de)) / n_direct)
+    kern_ms = ranks.max(sum(a_.elapsed_time(b_) for a_, b_ in zip(ds, de)) / n_side / lay)
     assert B.hga_device_status(sh) == 0
     hbm, peak_kind = peaks()
     achieved = nb[kern] / (kern_ms * 1e-3) / 1e9
+
+    # e2e: every step, the new token's q and K/V rows of every layer come in from
+    # pinned host memory and every layer's output goes back
+    q_host = [torch.empty(d["q"].shape, dtype=d["q"].dtype).pin_memory() for d in L_]
+    for qh, d in zip(q_host, L_):
+        qh.copy_(d["q"])
+    kv_new = torch.empty(len(L_), 2, wl.batch, wl.heads_kv, wl.head_dim,
+                         dtype=torch.bfloat16).pin_memory()
+    for li, d in enumerate(L_):
+        kv_new[li, 0].copy_((d["k_host"] if hot else d["k"])[:, :, p].cpu())
+        kv_new[li, 1].copy_((d["v_host"] if hot else d["v"])[:, :, p].cpu())
+    out_host = [torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory() for d in L_]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e = []
+    for i in range(warmup + min(steps, 100)):
+        flush()
+        e0.record(stream)
+        for li, d in enumerate(L_):
+            d["q"].copy_(q_host[li], non_blocking=True)
+            if hot:  # the new token's K/V goes into the host cache, a host-side write
+                d["k_host"][:, :, p].copy_(kv_new[li, 0])
+                d["v_host"][:, :, p].copy_(kv_new[li, 1])
+            else:
+                d["k"][:, :, p].copy_(kv_new[li, 0], non_blocking=True)
+                d["v"][:, :, p].copy_(kv_new[li, 1], non_blocking=True)
+        graphs["step"].replay()
+        for li, d in enumerate(L_):
+            out_host[li].copy_(d["out"], non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= warmup:
+            e2e.append(e0.elapsed_time(e1))
+    ms_e2e = ranks.max(sum(e2e) / len(e2e))
+    h2d = sum(t.numel() * t.element_size() for t in q_host) + \
+        (0 if hot else kv_new.numel() * kv_new.element_size())
+    d2h = sum(t.numel() * t.element_size() for t in out_host)
+
+    per_layer_ms = ms_step / layers
     total_bytes = nb["summaries"] + nb["route"] + nb["attend"]
     if one_launch:
-        launches_per_step = 1  # the decode step, summary append included
-    elif fused:
-        launches_per_step = 3  # summary append, routing, attention
-    else:
-        # summaries, route, (gather,) attend (+ the split-K combine when a workspace is used)
-        launches_per_step = 3 + (1 if wsb > 0 else 0) + (1 if hot else 0)
-    tokens = wl.batch  # per rank
-    line = {
-        "metric": METRIC,
-        "value": job_rate(tokens, world, ms_step),
-        "unit": "decode tokens/s (one attention layer)",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        launches = layers
+    else:  # append, route, (gather,) attend (+ the split-K combine with a workspace)
+        launches = layers * (3 + (1 if wsb > 0 else 0) + (1 if hot else 0))
+    unit = "decode tokens/s (one attention layer)"
+    rec = {
+        "value": job_rate(wl.batch, world, per_layer_ms),
+        "unit": unit,
         "ms_per_step": ms_step,
-        "attn_us_per_layer": ms_step * 1e3,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16 K/V, fp32 accumulation" if wl.dtype == "bf16" else "f32",
-        "data": "synthetic (seeded N(0,1) q/k/v" +
-                (f"; {wl.needles} needle chunks per KV head" if wl.needles else "") +
-                (f"; log-normal key norms, sigma {wl.lognormal_sigma}" if wl.lognormal_sigma else "") +
-                ("; K/V in pinned host memory" if hot else "") + ")",
+        "attn_us_per_layer": per_layer_ms * 1e3,
+        "layers_per_step": layers,
+        "data": data,
         "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": n,
                    "heads_q": wl.heads_q, "heads_kv": wl.heads_kv, "head_dim": wl.head_dim,
                    "chunk": wl.chunk, "group": wl.group, "sink": wl.sink, "local": wl.local,
                    "topk_chunks": wl.topk_chunks, "topk_groups": wl.topk_groups,
-                   "tokens_attended_per_kv_head": nb["tokens"],
-                   "l2": "flushed (256 MB write) before every timed step",
-                   "parallelism": f"replicas x{world} (independent sequences per GPU)"},
+                   "tokens_attended_per_kv_head": nb["tokens"], "layers_per_step": layers,
+                   "l2": L2_NOTE, "parallelism": f"replicas x{world} (independent sequences per GPU)"},
         "per_kernel_us": {kk: ms[kk] * 1e3 for kk in parts},
-        "two_call_step_us": ms_step2 * 1e3,
-        "four_call_step_us": ms_step4 * 1e3,
-        "timing_floor_us": floor_us,
-        "step_hbm_bytes": total_bytes,
-        "step_hbm_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
+        **{name: t * 1e3 for name, t in side_ms.items()},
+        "step_hbm_bytes_per_layer": total_bytes,
+        "step_hbm_gbs": total_bytes / (per_layer_ms * 1e-3) / 1e9,
         "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": profile_traffic(kernel_name, wl),
                      "algorithmic_bytes": nb[kern], "kernel_us": kern_ms * 1e3,
-                     "graph_replay_us": ms[kern] * 1e3,
-                     "duration": "CUDA events on the launch stream around a direct launch of the "
-                                 "call, queued behind the L2 flush (mean of the timed launches); "
-                                 "graph_replay_us is the call's CUDA graph replayed the same way"},
-        "e2e": {"value": job_rate(tokens, world, ms_e2e), "unit": "decode tokens/s (one attention layer)",
+                     "duration": ("CUDA events on the launch stream around " +
+                                  (f"{lay} back-to-back launches (one per layer), divided by {lay}"
+                                   if lay > 1 else "one direct launch") +
+                                  ", queued behind the L2 flush; per_kernel_us holds each call's "
+                                  "one-layer CUDA graph replayed the same way")},
+        "e2e": {"value": job_rate(wl.batch, world, ms_e2e / layers), "unit": unit,
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
-        "host_link": host_link_report(wl, ms, dev) if hot else None,
-        "timing": "CUDA graph of the step replayed per timed step; CUDA events on the launch stream",
+        "gpu_launches": launches * steps,
+        "timing": (f"CUDA graph of the {layers}-layer step replayed per timed step; CUDA events on "
+                   "the launch stream; attention time per layer = step time / layers"),
         "clocks": clk.report(),
     }
-    return line, wl, seed, x
+    if hot:
+        rec["host_link"] = host_link_report(wl, ms, dev)
+    del L_, graphs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
 
 
 def host_link_report(wl: S.Workload, ms: dict, dev) -> dict:
@@ -574,24 +627,21 @@ def tensor_peak():
         return 1590.0, "fallback"
 
 
-def run_prefill(args, rank: int, world: int, wl: S.Workload):
+def prefill_record(args, wl: S.Workload, steps: int, warmup: int, world: int, ranks,
+                   seed: int, x=None) -> dict:
     """One prefill step of one layer: summaries of the whole prompt, routing of
     every 64-query block, attention of every query (steps 1-5)."""
     import torch
     from hierarchical_sparse_attention_hga_b200 import binding as B
 
     dev = torch.device("cuda")
-    seed = rank_seed(args.workload, rank)
-    x = S.make_inputs(wl, seed)
     n = wl.context
     nblk = n // wl.chunk
-
-    def to_dev(a):
-        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16))
-        return t.view(torch.bfloat16).to(dev)
-
-    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
-    pos = torch.as_tensor(x["pos"], device=dev)
+    if x is not None:
+        q, k, v = (host_to_device(x[t], wl, dev) for t in ("q", "k", "v"))
+        pos = torch.as_tensor(x["pos"], device=dev)
+    else:
+        q, k, v, pos = device_inputs(wl, seed, dev)
     layer = B.Layer(batch=wl.batch, heads_q=wl.heads_q, heads_kv=wl.heads_kv, head_dim=wl.head_dim,
                     chunk=wl.chunk, group=wl.group, sink_chunks=wl.sink, local_chunks=wl.local,
                     topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
@@ -604,7 +654,7 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
     gi = torch.empty(bh, nblk, wl.topk_groups, dtype=torch.int32, device=dev)
     out = torch.empty(wl.batch, wl.heads_q, n, wl.head_dim, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(wl.batch, wl.heads_q, n, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = Flush(dev)
     parts = {
         "summaries": lambda: B.hga_build_summaries(layer, k, n, 0, n, cs, gs),
         "route": lambda: B.hga_route(layer, q, n, pos, cs, gs, n, ci, gi),
@@ -615,7 +665,7 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
         for fn in parts.values():
             fn()
 
-    for _ in range(max(1, args.warmup)):
+    for _ in range(max(1, warmup)):
         step()
     torch.cuda.synchronize()
     assert B.hga_device_status() == 0
@@ -629,33 +679,25 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
     stream = torch.cuda.current_stream()
 
     def timed(g_, iters):
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(iters)]
-        for a_, b_ in ev:
-            flush.zero_()
-            a_.record(stream)
-            g_.replay()
-            b_.record(stream)
-        torch.cuda.synchronize()
-        return sum(a_.elapsed_time(b_) for a_, b_ in ev) / iters
+        return timed_graph(g_, iters, flush, stream)
 
-    ranks = Ranks(world, dev)
     ranks.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        ms_step = timed(graphs["step"], args.steps)
+        ms_step = timed(graphs["step"], steps)
     ranks.barrier()
     ms_step = ranks.max(ms_step)
-    ms = {name: timed(graphs[name], max(3, min(args.steps, 20))) for name in parts}
+    ms = {name: timed(graphs[name], max(3, min(steps, 20))) for name in parts}
     assert B.hga_device_status() == 0
 
     # e2e: host q in (pinned), host output back, every step; k/v resident
-    q_host = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).pin_memory()
+    q_host = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    q_host.copy_(q)
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e = []
-    for i in range(1 + min(args.steps, 5)):
-        flush.zero_()
+    for i in range(1 + min(steps, 5)):
+        flush()
         e0.record(stream)
         q.view(torch.int16).copy_(q_host, non_blocking=True)
         graphs["step"].replay()
@@ -670,20 +712,18 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
     peak, peak_kind = tensor_peak()
     achieved = flops / (ms["attend"] * 1e-3) / 1e12
     tokens = wl.batch * n  # per rank
-    line = {
-        "metric": METRIC + " (prefill)",
+    rec = {
         "value": job_rate(tokens, world, ms_step),
         "unit": "prefill tokens/s (one attention layer)",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_step, "attn_us_per_layer": ms_step * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": ms_step, "attn_us_per_layer": ms_step * 1e3, "layers_per_step": 1,
         "dtype": "bf16 q/k/v, fp32 accumulation (tcgen05)",
-        "data": "synthetic (seeded N(0,1) q/k/v)",
+        "data": ("synthetic (seeded N(0,1) q/k/v from the host generator)" if x is not None else
+                 "synthetic (N(0,1) q/k/v drawn on the device)"),
         "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": n,
                    "heads_q": wl.heads_q, "heads_kv": wl.heads_kv, "head_dim": wl.head_dim,
                    "chunk": wl.chunk, "query_block": wl.chunk, "topk_chunks": wl.topk_chunks,
                    "topk_groups": wl.topk_groups,
-                   "l2": "flushed (256 MB write) before every timed step",
+                   "l2": L2_NOTE,
                    "parallelism": f"replicas x{world}"},
         "per_kernel_us": {kk: vv * 1e3 for kk, vv in ms.items()},
         "attend_flops": flops,
@@ -694,162 +734,194 @@ def run_prefill(args, rank: int, world: int, wl: S.Workload):
         "e2e": {"value": job_rate(tokens, world, ms_e2e), "unit": "prefill tokens/s (one attention layer)",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": q_host.numel() * 2,
                 "d2h_bytes_per_step": out_host.numel() * 2},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 3 * steps,
         "timing": "CUDA graph of the step replayed per timed step; CUDA events on the launch stream",
         "clocks": clk.report(),
     }
-    return line, wl, seed, x
+    del q, k, v, out, graphs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
 
 
-def oracle_prefill_rate(wl: S.Workload, seed: int, budget_s: float, x=None):
-    """Oracle prefill on a bounded sample of (KV head, query block) units: routing
-    of the block and attention of its G*C query rows.  Returns prompt tokens/s."""
+# ------------------------------------------------------------ oracle (CPU) arm
+
+def _oracle_worker(task):
+    """One oracle process: prepares its units from the seeded host generator (the
+    prefix summaries are state, not step work, so they are built untimed), then
+    times the oracle's work on them in turn, `rounds` times for `budget` seconds.
+    Decode unit (b, h): the summary rows the new token closes, level-1 and
+    level-2 routing, the token set and exact attention of the G query heads.
+    Prefill unit (h, j): routing of query block j and attention of its G*C rows.
+    Returns [(runs, seconds)] per round."""
     from threadpoolctl import threadpool_limits
 
     from oracle import hga_oracle as O
+    kind, wl, seed, units, budget, rounds = task
     prm = O.HGAParams(head_dim=wl.head_dim, heads_q=wl.heads_q, heads_kv=wl.heads_kv,
                       chunk=wl.chunk, group=wl.group, sink=wl.sink, local=wl.local,
                       topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
                       n_high_pairs=wl.n_high_pairs, rope_theta=wl.rope_theta)
     g, c = wl.gqa, wl.chunk
-    nblk = wl.context // c
-    rng = np.random.default_rng(0)
-    units = [(h, int(j)) for h in range(wl.heads_kv) for j in rng.permutation(nblk)[:8]]
-    times, spent = [], 0.0
+    out = []
     with threadpool_limits(limits=1):
-        cache = {}
-        for h, j in units:
-            if spent >= budget_s:
-                break
-            if h not in cache:
-                kb = x["k"][0, h] if x is not None else S.key_slice(wl, seed, 0, h)
-                vb = x["v"][0, h] if x is not None else S.value_slice(wl, seed, 0, h)
-                k64, v64 = S.widen(kb, wl.dtype), S.widen(vb, wl.dtype)
-                cache = {h: (k64, v64, O.build_summaries(k64, prm))}
-            k64, v64, (cs, gs) = cache[h]
-            qb = (x["q"][0, h * g:(h + 1) * g, j * c:(j + 1) * c] if x is not None else
-                  S.query_slice(wl, seed, 0)[h * g:(h + 1) * g, j * c:(j + 1) * c])
-            q64 = S.widen(qb, wl.dtype)
-            t0 = time.perf_counter()
-            qbar = O.routing_query(q64)
-            cidx, _, _ = O.route_chunks(qbar, cs, j, prm)
-            gidx, _, _ = O.route_groups(qbar, gs, cidx, prm)
-            for i in range(c):
-                toks = O.visible_tokens(j * c + i, j, gidx, prm)
-                for hh in range(g):
-                    O.attend(q64[hh, i], k64, v64, toks)
-            dt = time.perf_counter() - t0
-            times.append(dt)
-            spent += dt
-    per_unit = sum(times) / len(times)
-    step_s = per_unit * wl.heads_kv * nblk * wl.batch
-    sample = (f"{len(times)} (KV head, 64-query block) units of the {wl.context}-token prefill "
-              f"(routing + attention of every row), extrapolated ({sum(times):.1f} s of oracle time)")
-    return wl.batch * wl.context / step_s, sample, 1
-
-
-# ------------------------------------------------------------ oracle (CPU) arm
-
-def oracle_decode_rate(wl: S.Workload, seed: int, budget_s: float, x=None):
-    """Oracle decode step, timed per (sequence, KV head) unit on a bounded sample.
-
-    Per unit: summaries of the rows the new token closes, level-1 and level-2
-    routing, token set and exact attention of the G query heads.  The prefix
-    summaries are built before timing (they are state, not step work).
-    Returns (tokens/s for the whole batch, sample description, threads used).
-    """
-    from threadpoolctl import threadpool_limits
-
-    from oracle import hga_oracle as O
-    prm = O.HGAParams(head_dim=wl.head_dim, heads_q=wl.heads_q, heads_kv=wl.heads_kv,
-                      chunk=wl.chunk, group=wl.group, sink=wl.sink, local=wl.local,
-                      topk_chunks=wl.topk_chunks, topk_groups=wl.topk_groups,
-                      n_high_pairs=wl.n_high_pairs, rope_theta=wl.rope_theta)
-    p = wl.context - 1
-    cur = p // wl.chunk
-    g = wl.gqa
-    times = []
-    spent = 0.0
-    units = [(b, h) for b in range(wl.batch) for h in range(wl.heads_kv)]
-    # A few (sequence, KV head) units, prepared once (their prefix summaries are
-    # state, not step work), then timed in turn until the budget is spent.
-    sample_units = units[:: max(1, len(units) // 4)][:4]
-    prepared = []
-    with threadpool_limits(limits=1):
-        for b, h in sample_units:
-            if x is not None:
-                qb, kb, vb = x["q"][b, h * g:(h + 1) * g], x["k"][b, h], x["v"][b, h]
-            else:
+        prepared = []
+        for u in units:
+            if kind == "decode":
+                b, h = u
                 q1 = S.query_slice(wl, seed, b, 1)
-                qb = q1[h * g:(h + 1) * g]
                 kb, vb = S.key_slice(wl, seed, b, h, q1), S.value_slice(wl, seed, b, h)
-            q64, k64, v64 = S.widen(qb, wl.dtype), S.widen(kb, wl.dtype), S.widen(vb, wl.dtype)
-            cs, gs = O.build_summaries(k64[:cur * wl.chunk], prm)
-            cs = np.concatenate([cs, np.full((1, wl.head_dim), np.nan)])
-            gs = np.concatenate([gs, np.full((1, gs.shape[1], wl.head_dim), np.nan)])
-            prepared.append((q64, k64, v64, cs, gs))
-        i = 0
-        while spent < budget_s or not times:
-            q64, k64, v64, cs0, gs0 = prepared[i % len(prepared)]
-            cs, gs = cs0.copy(), gs0.copy()
-            t0 = time.perf_counter()
-            c0 = cur * wl.chunk
-            cs[cur] = O.span_summary(k64[c0:c0 + wl.chunk], c0, prm.n_high_pairs, prm.rope_theta)
-            g0 = p + 1 - wl.group
-            gs[cur, -1] = O.span_summary(k64[g0:p + 1], g0, prm.n_high_pairs, prm.rope_theta)
-            qbar = O.routing_query(q64[:, 0])
-            cidx, _, _ = O.route_chunks(qbar, cs, cur, prm)
-            gidx, _, _ = O.route_groups(qbar, gs, cidx, prm)
-            toks = O.visible_tokens(p, cur, gidx, prm)
-            for hh in range(g):
-                O.attend(q64[hh, 0], k64, v64, toks)
-            dt = time.perf_counter() - t0
-            times.append(dt)
-            spent += dt
-            i += 1
-    per_unit = sum(times) / len(times)
-    step_s = per_unit * len(units)
-    sample = (f"{len(times)} timed runs over {len(prepared)} of the {len(units)} (sequence, KV "
-              f"head) units of a decode step at position {p}; mean per unit times the batch's "
-              f"units ({sum(times):.1f} s of oracle time)")
-    return wl.batch / step_s, sample, 1
+                q64 = S.widen(q1[h * g:(h + 1) * g], wl.dtype)
+                k64, v64 = S.widen(kb, wl.dtype), S.widen(vb, wl.dtype)
+                cur = (wl.context - 1) // c
+                cs, gs = O.build_summaries(k64[:cur * c], prm)
+                cs = np.concatenate([cs, np.full((1, wl.head_dim), np.nan)])
+                gs = np.concatenate([gs, np.full((1, gs.shape[1], wl.head_dim), np.nan)])
+                prepared.append((q64, k64, v64, cs, gs))
+            else:
+                h, j = u
+                k64 = S.widen(S.key_slice(wl, seed, 0, h), wl.dtype)
+                v64 = S.widen(S.value_slice(wl, seed, 0, h), wl.dtype)
+                # the block's queries: N(0,1) rows of the stored type (the whole
+                # prompt's query tensor is not drawn for one block)
+                rng = np.random.default_rng([seed, 99, h, j])
+                q64 = S.widen(S.store(rng.standard_normal((g, c, wl.head_dim), dtype=np.float32),
+                                      wl.dtype), wl.dtype)
+                prepared.append((q64, k64, v64, O.build_summaries(k64, prm), j))
+        for _ in range(rounds):
+            runs, spent, i = 0, 0.0, 0
+            while spent < budget or runs == 0:
+                t0 = time.perf_counter()
+                if kind == "decode":
+                    q64, k64, v64, cs0, gs0 = prepared[i % len(prepared)]
+                    p = wl.context - 1
+                    cur = p // c
+                    cs, gs = cs0.copy(), gs0.copy()
+                    c0 = cur * c
+                    if (p + 1) % c == 0:
+                        cs[cur] = O.span_summary(k64[c0:c0 + c], c0, prm.n_high_pairs, prm.rope_theta)
+                    if (p + 1) % wl.group == 0:
+                        g0 = p + 1 - wl.group
+                        gs[cur, (p % c) // wl.group] = O.span_summary(k64[g0:p + 1], g0,
+                                                                      prm.n_high_pairs, prm.rope_theta)
+                    qbar = O.routing_query(q64[:, 0])
+                    cidx, _, _ = O.route_chunks(qbar, cs, cur, prm)
+                    gidx, _, _ = O.route_groups(qbar, gs, cidx, prm)
+                    toks = O.visible_tokens(p, cur, gidx, prm)
+                    for hh in range(g):
+                        O.attend(q64[hh, 0], k64, v64, toks)
+                else:
+                    q64, k64, v64, (cs, gs), j = prepared[i % len(prepared)]
+                    qbar = O.routing_query(q64)
+                    cidx, _, _ = O.route_chunks(qbar, cs, j, prm)
+                    gidx, _, _ = O.route_groups(qbar, gs, cidx, prm)
+                    for r in range(c):
+                        toks = O.visible_tokens(j * c + r, j, gidx, prm)
+                        for hh in range(g):
+                            O.attend(q64[hh, r], k64, v64, toks)
+                spent += time.perf_counter() - t0
+                runs += 1
+                i += 1
+            out.append((runs, spent))
+    return out
 
 
-def run_reference(args, rank: int):
-    """The oracle arm: the float64 CPU oracle timed on the host cores, rank 0 only.
+def oracle_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
-    Each step is a bounded sample of the same workload (sized so the whole
-    run stays within a few minutes), extrapolated to the arm's unit.
-    """
-    if rank != 0:
-        return None
+
+def oracle_rates(wl: S.Workload, seed: int, budget: float, rounds: int = 1, max_procs: int = 64):
+    """The oracle on the host's cores: one single-threaded process per core (spawned),
+    each timing a few of the workload's independent units.  Returns (per-round
+    tokens/s, sample description, processes)."""
+    import multiprocessing as mp
+    kind = "prefill" if wl.prefill else "decode"
+    nblk = wl.context // wl.chunk
+    if kind == "decode":
+        all_units = [(b, h) for b in range(wl.batch) for h in range(wl.heads_kv)]
+        units_per_step, tokens_per_step = len(all_units), wl.batch
+    else:
+        rng = np.random.default_rng(0)
+        all_units = [(h, int(j)) for h in range(wl.heads_kv) for j in rng.permutation(nblk)[:8]]
+        units_per_step, tokens_per_step = wl.heads_kv * nblk * wl.batch, wl.batch * wl.context
+    # memory per process grows with the context: fewer processes for long ones
+    procs = max(1, min(oracle_cores(), max_procs, 16 if wl.context > 65536 else max_procs,
+                       len(all_units)))
+    per = [all_units[i::procs][:2] for i in range(procs)]
+    tasks = [(kind, wl, seed, u, budget, rounds) for u in per]
+    with mp.get_context("spawn").Pool(procs) as pool:
+        res = pool.map(_oracle_worker, tasks)
+    rates = []
+    for r in range(rounds):
+        units_per_s = sum(w[r][0] / w[r][1] for w in res)
+        rates.append(units_per_s / units_per_step * tokens_per_step)
+    n_runs = sum(w[r][0] for w in res for r in range(rounds))
+    what = ("(sequence, KV head) units of a decode step at position "
+            f"{wl.context - 1}" if kind == "decode" else
+            f"(KV head, 64-query block) units of the {wl.context}-token prefill")
+    sample = (f"{procs} single-threaded processes, {n_runs} timed runs over "
+              f"{sum(len(u) for u in per)} {what}, each process timing its units for "
+              f"{budget:.1f} s per round; throughput summed over the processes and scaled "
+              f"to the step's {units_per_step} units")
+    return rates, sample, procs
+
+
+def cpu_baseline(wl, seed, budget, unit):
+    rates, sample, procs = oracle_rates(wl, seed, budget)
+    return {"value": rates[0], "unit": unit, "cores": procs, "kind": "oracle", "sample": sample}
+
+
+def workload_of(args) -> S.Workload:
     wl = S.workload(args.workload)
     if args.batch:
         wl = wl.with_(batch=args.batch)
     if args.context:
         wl = wl.with_(context=args.context)
+    return wl
+
+
+def run_reference(args, rank: int):
+    """The oracle arm: the float64 CPU oracle timed on the host cores, rank 0 only.
+
+    Each step is a bounded sample of the same workload (sized so the whole run
+    stays within a few minutes), extrapolated to the arm's unit.
+    """
+    if rank != 0:
+        return None
+    wl = workload_of(args)
     seed = rank_seed(args.workload, 0)
-    rate_fn = oracle_prefill_rate if wl.prefill else oracle_decode_rate
-    rates = []
-    budget = max(0.02, min(args.cpu_seconds / 10, 150.0 / (args.warmup + args.steps)))
-    for i in range(args.warmup + args.steps):
-        r, sample, cores = rate_fn(wl, seed, budget_s=budget)
-        if i >= args.warmup:
-            rates.append(r)
-    value = statistics.median(rates)
+    rounds = args.warmup + args.steps
+    budget = max(0.05, min(args.cpu_seconds / 4, 120.0 / rounds))
+    rates, sample, procs = oracle_rates(wl, seed, budget, rounds=rounds)
+    timed = rates[args.warmup:] or rates
+    value = statistics.median(timed)
     kind = "prefill" if wl.prefill else "decode"
     unit = f"{kind} tokens/s (one attention layer)"
     tokens_per_step = wl.batch * (wl.context if wl.prefill else 1)
     return {"impl": "reference", "metric": METRIC + (" (prefill)" if wl.prefill else ""),
             "value": value, "unit": unit,
-            "n_gpus": args.gpus, "steps": len(rates), "warmup": args.warmup,
+            "n_gpus": args.gpus, "steps": len(timed), "warmup": args.warmup,
             "ms_per_step": tokens_per_step / value * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded, same generator)",
             "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "context": wl.context},
-            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": unit, "cores": procs, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# Other workloads measured beside the headline (one GPU, default workload only):
+# name, workload, attention layers per step.
+SUB_WORKLOADS = (
+    ("llama3_8b_prefill_64k", S.workload("llama3_8b_prefill_64k"), 1),
+    ("wide_head_decode_64k_b32", S.workload("wide_head_decode_64k"), 2),
+    ("host_tier_decode_128k_b8", S.workload("host_tier_decode_128k"), 1),
+    ("llama3_8b_decode_32k_b4", S.workload("llama3_8b_decode_32k", batch=4, needles=0), 4),
+    ("llama3_8b_decode_32k_b1", S.workload("llama3_8b_decode_32k", batch=1, needles=0), 4),
+)
 
 
 def main():
@@ -861,17 +933,51 @@ def main():
         if line:
             print(json.dumps(line))
         return
+    import torch
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    from hierarchical_sparse_attention_hga_b200.build import build
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
     if world > 1:
-        import torch
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         rank, world = init_ranks("nccl")
-    line, wl, seed, x = run_hga(args, rank, world)
+    build()
+    B.load_library()
+    dev = torch.device("cuda")
+    ranks = Ranks(world, dev)
+    wl = workload_of(args)
+    seed = rank_seed(args.workload, rank)
+    x = S.make_inputs(wl, seed)
+    if wl.prefill:
+        rec = prefill_record(args, wl, args.steps, args.warmup, world, ranks, seed, x)
+    else:
+        layers = args.layers or (1 if wl.name.startswith("host_tier") else 4)
+        rec = decode_record(args, wl, layers, args.steps, args.warmup, world, ranks, seed, x)
+    line = {"metric": METRIC + (" (prefill)" if wl.prefill else ""), "value": rec.pop("value"),
+            "unit": rec.pop("unit"), "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": rec.pop("ms_per_step"), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": rec.pop("dtype", "bf16 K/V, fp32 accumulation" if wl.dtype == "bf16" else "f32"),
+            **rec}
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, seed, args.cpu_seconds, line["unit"])
+    default_run = args.workload == "llama3_8b_decode_32k" and not args.batch and not args.context
+    if world == 1 and default_run and not args.no_workloads:
+        del x
+        subs = {}
+        sub_steps = max(3, min(args.steps, 20))
+        for i, (name, swl, layers) in enumerate(SUB_WORKLOADS):
+            sseed = rank_seed(swl.name, 0) + 17 * (i + 1)
+            if swl.prefill:
+                r = prefill_record(args, swl, sub_steps, args.warmup, world, ranks, sseed)
+            else:
+                r = decode_record(args, swl, layers, sub_steps, args.warmup, world, ranks, sseed,
+                                  compare=False)
+            r["steps"] = sub_steps
+            if not args.no_cpu_baseline:
+                r["cpu_baseline"] = cpu_baseline(swl, sseed, 3.0, r["unit"])
+            subs[name] = r
+        line["workloads"] = subs
     if rank == 0:
-        if not args.no_cpu_baseline:
-            rate = oracle_prefill_rate if wl.prefill else oracle_decode_rate
-            val, sample, cores = rate(wl, seed, args.cpu_seconds, x)
-            line["cpu_baseline"] = {"value": val, "unit": line["unit"], "cores": cores,
-                                    "kind": "oracle", "sample": sample}
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

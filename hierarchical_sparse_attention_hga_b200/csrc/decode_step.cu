@@ -1,8 +1,8 @@
 // One decode step of the HGA hot path in one launch: the summary append
 // (step 1), chunk routing (2), group routing (3), and the gather and exact
 // attention of the chosen tokens (4, 5), for every (sequence, KV head) item of
-// the batch.  bf16 K/V, D = 128; batches of at least half an item per SM (the
-// routing and attention kernels serve smaller ones).
+// the batch.  bf16 K/V, D = 128, at most 64 chosen chunks and 128 routed groups
+// (the routing and attention kernels serve wider routing).
 //
 // HGA technical summary ("Hierarchical Global Attention (HGA)", gist.science
 // 2606.30709), "Metodologia -> Meccanismo Core": item 3 (RoPE-aware summaries
@@ -716,12 +716,10 @@ cudaError_t dispatch(const LayerParams& p, const StepShape& sh, const CUtensorMa
 }  // namespace
 
 bool decode_item_path(const LayerParams& p) {
-  const int64_t items = static_cast<int64_t>(p.B) * p.Hkv;
-  const int sms = device_sm_count();
   const StepShape sh = step_shape(p);
   // dynamic shared memory: one CTA per SM may take 225 KB, two per SM 112 KB each
   const size_t limit = sh.W == 7 ? 225 * 1024 : 112 * 1024;
-  return items * 2 >= sms && p.kc <= kKcMax && p.kg <= kKgMax && p.Ng <= 8 &&
+  return p.kc <= kKcMax && p.kg <= kKgMax && p.Ng <= 8 &&
          kRows % p.Ng == 0 && step_smem_bytes(p, sh.W) <= limit;
 }
 

@@ -113,8 +113,8 @@ cudaError_t launch_route_decode(const LayerParams& p, int dtype, bool level1, bo
                                 cudaStream_t s);
 
 // One decode step (optional summary append + routing + attention): one launch of
-// decode_step_kernel when decode_item_path (at least half a (sequence, KV head)
-// item per SM), else the append, routing and attention kernels; applies when
+// decode_step_kernel when decode_item_path (kc <= 64, kg <= 128 and the shared
+// memory fits), else the append, routing and attention kernels; applies when
 // decode_step_path (bf16, D = 128 decode, device-resident K/V).
 bool decode_item_path(const LayerParams& p);
 bool decode_step_path(const LayerParams& p, int dtype);

@@ -295,19 +295,17 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
  * the current chunk, which the step attends in full and never routes.  With
  * append == 0 the tables are only read.
  *
- * When the batch holds at least half a (sequence, KV head) item per SM, the
- * step is one launch: each CTA works through items (one at a time; one CTA per
- * SM up to one item per SM, two per SM above); its warps stream the candidate
- * chunk summaries and the K/V units of the always-visible chunks through
- * shared-memory rings, one warp merges the level-1 picks and runs level 2
- * while the others attend, then all attend the routed groups, and another warp
- * does the summary append.  Smaller batches get the append, routing and
- * attention kernels, launched by this call (hga_decode_step_launches says
- * which).  Decode only (q_len is 1): bf16 K/V in device memory (kv_loc
- * HGA_KV_DEVICE), head_dim 128, group 16, at most 16 query heads per KV head,
- * topk_groups <= 1024 (the one-launch kernel: topk_chunks <= 64 and
- * topk_groups <= 128); other shapes return HGA_ERR_UNSUPPORTED (use hga_route +
- * hga_attend).  Arguments and layouts are those of hga_build_summaries,
+ * With topk_chunks <= 64 and topk_groups <= 128 the step is one launch: each
+ * CTA works through (sequence, KV head) items, one at a time (one CTA per SM up
+ * to one item per SM, two per SM above); its warps stream the candidate chunk
+ * summaries and the K/V of the always-visible chunks through shared-memory
+ * rings, select the chunks and then the groups between barriers, attend the
+ * routed groups and merge their partials, while another warp does the summary
+ * append.  Wider routing gets the append, routing and attention kernels,
+ * launched by this call (hga_decode_step_launches says which).  Decode only
+ * (q_len is 1): bf16 K/V in device memory (kv_loc HGA_KV_DEVICE), head_dim 128,
+ * group 16, at most 16 query heads per KV head, topk_groups <= 1024; other
+ * shapes return HGA_ERR_UNSUPPORTED (use hga_route + hga_attend).  Arguments and layouts are those of hga_build_summaries,
  * hga_route and hga_attend; chunk_score, group_score and lse may be NULL.  No
  * workspace.
  */

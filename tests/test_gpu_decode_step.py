@@ -1,9 +1,9 @@
 """hga_decode_step against hga_build_summaries + hga_route + hga_attend and the oracle.
 
-Batches with at least half a (sequence, KV head) item per SM run the one-launch
-kernel (one CTA per SM up to one item per SM, two CTAs per SM above, each
-working through items); smaller batches run the append, routing and attention
-kernels through the same call.  The one-launch kernel scores with the routing
+Routing of at most 64 chunks and 128 groups runs the one-launch kernel (one CTA
+per SM up to one item per SM, two CTAs per SM above, each working through
+items); wider routing runs the append, routing and attention kernels through the
+same call.  The one-launch kernel scores with the routing
 kernel's arithmetic, so the routed indices and scores must be bit-identical.  Its
 warps attend the units in another grouping, so the running maxima against which P
 is rounded to bf16 differ and the outputs agree to that rounding (well inside the
@@ -136,8 +136,8 @@ def test_decode_step_llama3_8b_32k_batch16_full_size():
                                   topk_groups=16)),
 ])
 def test_decode_step_one_cta_per_item(name, kw):
-    """Batches with about one (sequence, KV head) item per SM take the one-CTA-per-item
-    variant; ragged positions, down to a sequence with no candidate chunk."""
+    """Batches of up to one (sequence, KV head) item per SM (one CTA per SM); ragged
+    positions, down to a sequence with no candidate chunk."""
     wl = S.workload(name, **kw)
     x = S.make_inputs(wl, 33)
     rng = np.random.default_rng(5)
@@ -172,19 +172,20 @@ def test_decode_step_one_launch_wide_shapes(name, kw):
         compare_head(wl, x, fus, b, wl.heads_kv - 1)
 
 
-@pytest.mark.parametrize("batch", [2, 10])
-def test_decode_step_append_is_bitwise_the_batch_build(batch):
+@pytest.mark.parametrize("batch,kg", [(2, 32), (10, 32), (2, 256)])
+def test_decode_step_append_is_bitwise_the_batch_build(batch, kg):
     """With append, hga_decode_step writes the summary rows each sequence's token closes
     (a group; a group and its chunk; nothing), bit for bit as hga_build_summaries does,
-    on the one-launch kernel (batch 10: 80 items) and on the kernel sequence (batch 2)."""
-    wl = S.workload("llama3_8b_decode_32k", batch=batch, context=4096, needles=0)
+    on the one-launch kernel and on the kernel sequence (top-256 groups)."""
+    wl = S.workload("llama3_8b_decode_32k", batch=batch, context=4096, needles=0,
+                    topk_chunks=64 if kg > 128 else 16, topk_groups=kg)
     x = S.make_inputs(wl, 35)
     n = wl.context
     pos = np.array([n - 1, 2 * 64 * 9 + 15, 1000, 64 * 20 - 1, 64 * 33 + 47, 3000, 16 * 100 - 1,
                     64 * 50 + 31, 2048 + 63, 4000][:batch], dtype=np.int64)
     x["pos"] = pos
     layer = layer_of(wl)
-    assert B.hga_decode_step_launches(layer, n) == (1 if batch == 10 else 2)
+    assert B.hga_decode_step_launches(layer, n) == (1 if kg <= 128 else 2)
     bh, nc, ng = wl.batch * wl.heads_kv, n // wl.chunk, wl.chunk // wl.group
     q, k, v = (to_device(x[t], wl.dtype) for t in ("q", "k", "v"))
     pos_t = torch.as_tensor(pos, device="cuda")

@@ -239,3 +239,98 @@ def check_properties(wl: S.Workload, res: dict):
         gv = g[g >= 0]
         assert (np.diff(gv) > 0).all() and (g[len(gv):] == -1).all()
         assert set((gv // ng).tolist()) <= set(valid.tolist())
+
+
+# ------------------------------------------------- routing of every unit at full size
+
+def _routing_unit(task):
+    """Oracle routing of one decode (sequence, KV head) unit against the GPU's
+    selection (a process-pool worker): regenerates the unit's stored inputs with
+    the counter-based generator (the same bytes make_inputs gives), builds the
+    summaries, routes both levels and checks the GPU's chunk and group ids.
+    Returns the number of near-tie differences it excused."""
+    from threadpoolctl import threadpool_limits
+    wl, seed, b, h, pos_last, gpu_chunks, gpu_groups = task
+    g = wl.gqa
+    prm = params_of(wl)
+    with threadpool_limits(limits=1):
+        q1 = S.query_slice(wl, seed, b, 1)
+        k = S.widen(S.key_slice(wl, seed, b, h, q1), wl.dtype)
+        q = S.widen(q1[h * g:(h + 1) * g], wl.dtype)
+        cs, gs = O.build_summaries(k, prm, n_valid=pos_last + 1)
+        cur = pos_last // wl.chunk
+        qbar = O.routing_query(q[:, 0:1])
+        cidx, ccand, cscore = O.route_chunks(qbar, cs, cur, prm)
+        scale = float(np.linalg.norm(qbar)) * max([float(np.linalg.norm(cs[c])) for c in ccand] or [1.0])
+        excused = 0
+        same = check_selection(gpu_chunks, cidx, ccand, cscore, wl.topk_chunks, scale,
+                               f"chunks b{b} h{h}")
+        chosen = cidx if same else [int(c) for c in gpu_chunks]
+        excused += 0 if same else 1
+        gidx, gcand, gscore = O.route_groups(qbar, gs, chosen, prm)
+        gscale = float(np.linalg.norm(qbar)) * max(
+            [float(np.linalg.norm(gs[i // prm.groups_per_chunk, i % prm.groups_per_chunk]))
+             for i in gcand] or [1.0])
+        if not check_selection(gpu_groups, gidx, gcand, gscore, wl.topk_groups, gscale,
+                               f"groups b{b} h{h}"):
+            excused += 1
+    return excused
+
+
+def compare_routing_all(wl: S.Workload, seed: int, res: dict, pos=None, procs: int | None = None):
+    """Routed ids of EVERY (sequence, KV head) unit of a decode step against the
+    oracle's routing (summaries and both top-k's; no attention), in parallel over
+    the host's cores (spawned processes, one unit each).  Returns the number of
+    near-tie differences excused."""
+    import multiprocessing as mp
+    import os
+    pos = np.full(wl.batch, wl.context - 1) if pos is None else np.asarray(pos)
+    tasks = [(wl, seed, b, h, int(pos[b]), [int(c) for c in res["chunk_idx"][b, h, 0]],
+              [int(i) for i in res["group_idx"][b, h, 0]])
+             for b in range(wl.batch) for h in range(wl.heads_kv)]
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    procs = procs or max(1, min(cores, 32 if wl.context <= 65536 else 16, len(tasks)))
+    with mp.get_context("spawn").Pool(procs) as pool:
+        return sum(pool.map(_routing_unit, tasks, chunksize=1))
+
+
+def compare_prefill_routing_all(wl: S.Workload, x: dict, res: dict, b: int, h: int) -> int:
+    """Routed ids of EVERY query block of one (sequence, KV head) of a prefill
+    against the oracle's routing; returns the near-tie differences excused."""
+    prm = params_of(wl)
+    g, c = wl.gqa, wl.chunk
+    k = S.widen(x["k"][b, h], wl.dtype)
+    pos_last = int(x["pos"][b])
+    q_len = x["q"].shape[2]
+    first = pos_last - q_len + 1
+    cs, gs = O.build_summaries(k, prm, n_valid=pos_last + 1)
+    qh = S.widen(x["q"][b, h * g:(h + 1) * g], wl.dtype)
+    excused = 0
+    for blk in range(q_len // c):
+        cur = (first + blk * c) // c
+        qbar = O.routing_query(qh[:, blk * c:(blk + 1) * c])
+        cidx, ccand, cscore = O.route_chunks(qbar, cs, cur, prm)
+        scale = float(np.linalg.norm(qbar)) * max([float(np.linalg.norm(cs[j])) for j in ccand] or [1.0])
+        same = check_selection(res["chunk_idx"][b, h, blk], cidx, ccand, cscore, wl.topk_chunks,
+                               scale, f"prefill chunks b{b} h{h} blk{blk}")
+        excused += 0 if same else 1
+        chosen = cidx if same else list(res["chunk_idx"][b, h, blk])
+        gidx, gcand, gscore = O.route_groups(qbar, gs, chosen, prm)
+        gscale = float(np.linalg.norm(qbar)) * max(
+            [float(np.linalg.norm(gs[i // prm.groups_per_chunk, i % prm.groups_per_chunk]))
+             for i in gcand] or [1.0])
+        if not check_selection(res["group_idx"][b, h, blk], gidx, gcand, gscore, wl.topk_groups,
+                               gscale, f"prefill groups b{b} h{h} blk{blk}"):
+            excused += 1
+    return excused
+
+
+def sample_units(wl: S.Workload, n: int, seed: int = 0):
+    """n distinct (sequence, KV head) units, always including the first and the last."""
+    rng = np.random.default_rng(seed)
+    units = [(b, h) for b in range(wl.batch) for h in range(wl.heads_kv)]
+    pick = {0, len(units) - 1} | set(int(i) for i in rng.permutation(len(units))[:max(0, n - 2)])
+    return [units[i] for i in sorted(pick)][:max(n, 2)]

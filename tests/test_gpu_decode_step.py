@@ -21,7 +21,8 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():  # pragma: no cover - collected on CPU too
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from gpu_harness import compare_head, layer_of, to_device  # noqa: E402
+from gpu_harness import (compare_head, compare_routing_all, layer_of, sample_units,  # noqa: E402
+                         to_device)
 from hierarchical_sparse_attention_hga_b200 import binding as B  # noqa: E402
 
 
@@ -123,7 +124,8 @@ def test_decode_step_llama3_8b_32k_batch16_full_size():
     x = S.make_inputs(wl, S.seed_for(1))
     sep, fus = run_both(wl, x, out_dtype=B.HGA_BF16)
     check_same_routing_close_output(sep, fus, 1e-2)
-    for b, h in ((0, 0), (7, 3), (15, 7)):
+    compare_routing_all(wl, S.seed_for(1), fus)   # all 128 units
+    for b, h in sample_units(wl, 16, seed=2):
         compare_head(wl, x, fus, b, h)
     for b in range(wl.batch):
         for h in range(wl.heads_kv):

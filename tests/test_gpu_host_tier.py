@@ -16,7 +16,8 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():  # pragma: no cover - collected on CPU too
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from gpu_harness import compare_head, layer_of, to_device  # noqa: E402
+from gpu_harness import (compare_head, compare_routing_all, layer_of, sample_units,  # noqa: E402
+                         to_device)
 from hierarchical_sparse_attention_hga_b200 import binding as B  # noqa: E402
 
 
@@ -125,5 +126,6 @@ def test_host_tier_decode_128k_batch8_full_size():
     res = dict(chunk_idx=r.ci.cpu().numpy().reshape(8, 8, 1, -1), group_idx=gi.reshape(8, 8, 1, -1),
                out=out, lse=lse)
     assert np.isfinite(out).all()
-    for b, h in ((0, 0), (5, 4), (7, 7)):
+    compare_routing_all(wl, S.seed_for(3), res)   # all 64 units
+    for b, h in sample_units(wl, 16):
         compare_head(wl, x, res, b, h)

@@ -54,6 +54,10 @@ def parse():
     ap.add_argument("--layers", type=int, default=0,
                     help="attention layers per decode step (0: 4, or 1 for the host tier)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    ap.add_argument("--warm-slots", type=int, default=0,
+                    help="warm-tier group slots per (sequence, KV head) (0: 4 x topk_groups)")
+    ap.add_argument("--warm-steps", type=int, default=64,
+                    help="consecutive decode steps of the warm-tier runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the other workloads' sub-records")
@@ -567,6 +571,7 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
     }
     if hot:
         rec["host_link"] = host_link_report(wl, ms, dev)
+        rec["warm_tier"] = warm_tier_report(args, wl, layer, L_[0], flush, stream)
     del L_, graphs
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
@@ -596,6 +601,105 @@ def host_link_report(wl: S.Workload, ms: dict, dev) -> dict:
     return {"bytes_per_step": routed + window, "routed_bytes": routed, "window_bytes": window,
             "gather_us": ms["gather"] * 1e3, "achieved_gbs": gbs, "h2d_copy_probe_gbs": best,
             "frac_of_probe": gbs / best}
+
+
+def warm_tier_report(args, wl: S.Workload, layer, d: dict, flush, stream) -> dict:
+    """The warm tier in front of the host tier, against the cold host tier.
+
+    T consecutive decode steps at positions n-T .. n-1 (every sequence), each
+    with its own query: q_t = rho q_{t-1} + sqrt(1 - rho^2) z_t drawn on the
+    device (a stationary AR(1) walk from the workload's query, stored bf16), so
+    that consecutive steps route to overlapping groups.  Each arm runs one
+    untimed step at n-T-1 that fills the windows (and, warm, the table after a
+    reset), then the T steps: the summary append, routing, the gather (warm:
+    hga_gather_warm, cold: hga_gather_host; both copy only the newest window
+    row, the previous step having been at the position before) and the
+    attention (warm: hga_attend_warm), all on the launch stream.  CUDA events around every step
+    and around its gather, L2 flushed before each step."""
+    import torch
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+
+    dev = d["q"].device
+    sh = stream.cuda_stream
+    n, T = wl.context, args.warm_steps
+    M = args.warm_slots or 4 * wl.topk_groups
+    bh = wl.batch * wl.heads_kv
+    group_bytes = wl.group * wl.head_dim * 2 * 2      # K and V rows of one group, bf16
+    rows = B.hga_warm_rows(layer, M)
+    kw = torch.empty(bh, rows, wl.head_dim, dtype=torch.bfloat16, device=dev)
+    vw = torch.empty_like(kw)
+    tags = torch.empty(bh, M, dtype=torch.int32, device=dev)
+    stamps = torch.empty_like(tags)
+    smap = torch.empty(bh, wl.topk_groups, dtype=torch.int32, device=dev)
+    counters = torch.zeros(2, dtype=torch.int64, device=dev)
+    pos_all = torch.arange(n - T - 1, n, device=dev).repeat_interleave(wl.batch).view(T + 1, wl.batch)
+
+    def queries(rho):
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(int(rho * 1000))
+        cur = d["q"].float()
+        out = [cur.to(torch.bfloat16)]
+        c = (1.0 - rho * rho) ** 0.5
+        for _ in range(T):
+            cur = rho * cur + c * torch.randn(cur.shape, generator=gen, device=dev)
+            out.append(cur.to(torch.bfloat16))
+        return out
+
+    def run(qs, warm):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(T)]
+        if warm:
+            B.hga_warm_reset(layer, M, tags, stamps, stream=sh)
+        for t in range(T + 1):
+            pos = pos_all[t]
+            p = n - T - 1 + t
+            if t:
+                flush()
+                ev[t - 1][0].record(stream)
+            B.hga_build_summaries(layer, d["k_host"], n, p, p + 1, d["cs"], d["gs"], stream=sh)
+            B.hga_route(layer, qs[t], 1, pos, d["cs"], d["gs"], n, d["ci"], d["gi"], stream=sh)
+            if t:
+                ev[t - 1][1].record(stream)
+            if warm:
+                B.hga_gather_warm(layer, d["k_host"], d["v_host"], n, pos, d["gi"], M, tags,
+                                  stamps, smap, kw, vw, refresh_window=1 if t == 0 else 2,
+                                  counters=counters if t else None, stream=sh)
+            else:
+                B.hga_gather_host(layer, d["k_host"], d["v_host"], n, pos, d["gi"], d["k_work"],
+                                  d["v_work"], refresh_window=1 if t == 0 else 2, stream=sh)
+            if t:
+                ev[t - 1][2].record(stream)
+            if warm:
+                B.hga_attend_warm(layer, qs[t], pos, kw, vw, n, d["gi"], smap, M, d["out"],
+                                  d["lse"], stream=sh)
+            else:
+                B.hga_attend(layer, qs[t], 1, pos, d["k_work"], d["v_work"], n, d["gi"],
+                             d["out"], d["lse"], stream=sh)
+            if t:
+                ev[t - 1][3].record(stream)
+        torch.cuda.synchronize()
+        assert B.hga_device_status(sh) == 0
+        step = sum(e[0].elapsed_time(e[3]) for e in ev) / T
+        gather = sum(e[1].elapsed_time(e[2]) for e in ev) / T
+        return step * 1e3, gather * 1e3
+
+    runs = []
+    for rho in (0.9, 0.95, 0.99):
+        qs = queries(rho)
+        counters.zero_()
+        w_step, w_gather = run(qs, True)
+        hits, misses = (int(v) for v in counters.cpu())
+        c_step, c_gather = run(qs, False)
+        runs.append({"rho": rho, "hit_rate": hits / max(1, hits + misses),
+                     "routed_host_bytes_per_step": {"warm": misses * group_bytes / T,
+                                                    "cold": (hits + misses) * group_bytes / T},
+                     "step_us": {"warm": w_step, "cold": c_step},
+                     "gather_us": {"warm": w_gather, "cold": c_gather}})
+    return {"slots_per_kv_head": M, "steps": T,
+            "hbm_bytes": 2 * bh * rows * wl.head_dim * 2 + 2 * tags.numel() * 4,
+            "timing": ("CUDA events around each of T direct-launch steps (summary append, route, "
+                       "gather, attention) on the launch stream, L2 flushed before each; one "
+                       "untimed step fills the windows first"),
+            "runs": runs}
 
 
 # ------------------------------------------------------------------ prefill

@@ -20,7 +20,7 @@ from dataclasses import dataclass, replace
 import numpy as np
 
 # tensor ids of the sub-streams
-_Q, _K, _V, _NEEDLE, _LOGNORM = 0, 1, 2, 3, 4
+_Q, _K, _V, _NEEDLE, _LOGNORM, _DRIFT, _REQ = 0, 1, 2, 3, 4, 5, 6
 
 
 @dataclass(frozen=True)
@@ -192,6 +192,55 @@ def make_inputs(wl: Workload, seed: int, q_len: int | None = None) -> dict:
                   for b in range(wl.batch)])
     pos = np.full(wl.batch, wl.context - 1, dtype=np.int64)
     return dict(q=np.stack(qs), k=k, v=v, pos=pos)
+
+
+def drifting_queries(wl: Workload, seed: int, steps: int, rho: float) -> np.ndarray:
+    """Stored decode queries of `steps` consecutive steps: [steps, B, Hq, 1, D].
+
+    Step 0 is query_slice's query; every next one keeps a share rho of the last:
+    q_t = rho * q_{t-1} + sqrt(1 - rho^2) * z_t, z_t ~ N(0,1) (a stationary
+    AR(1) walk, drawn in float64 and stored once per step), so that
+    consecutive decode steps route to overlapping groups as a real decode
+    does."""
+    out = np.empty((steps, wl.batch, wl.heads_q, 1, wl.head_dim),
+                   dtype=np.uint16 if wl.dtype == "bf16" else np.float32)
+    c = math.sqrt(max(0.0, 1.0 - rho * rho))
+    for b in range(wl.batch):
+        cur = widen(query_slice(wl, seed, b, 1), wl.dtype)
+        out[0, b] = store(cur, wl.dtype)
+        rng = _rng(seed, _DRIFT, b)
+        for t in range(1, steps):
+            cur = rho * cur + c * rng.standard_normal(cur.shape)
+            out[t, b] = store(cur, wl.dtype)
+    return out
+
+
+def group_requests(wl: Workload, seed: int, steps: int, pos: np.ndarray, keep: float,
+                   kg: int | None = None) -> np.ndarray:
+    """Synthetic level-2 selections for the warm tier: [steps, B, Hkv, kg] int32.
+
+    Every row holds kg distinct groups of candidate chunks of pos[b] (chunk c
+    with sink <= c < pos[b] // C - local), ascending, padded with -1 when fewer
+    exist; from one step to the next each group stays with probability `keep`
+    and the others are drawn afresh from the candidates."""
+    kg = wl.topk_groups if kg is None else kg
+    gpc = wl.chunk // wl.group
+    out = np.full((steps, wl.batch, wl.heads_kv, kg), -1, dtype=np.int32)
+    for b in range(wl.batch):
+        lo, hi = wl.sink * gpc, max(wl.sink, int(pos[b]) // wl.chunk - wl.local) * gpc
+        cand = np.arange(lo, hi)
+        n = min(kg, len(cand))
+        for h in range(wl.heads_kv):
+            rng = _rng(seed, _REQ, b, h)
+            cur = np.sort(rng.choice(cand, n, replace=False)) if n else cand[:0]
+            for t in range(steps):
+                if t:
+                    stay = cur[rng.random(len(cur)) < keep]
+                    pool = np.setdiff1d(cand, stay)
+                    cur = np.sort(np.concatenate([stay, rng.choice(pool, n - len(stay),
+                                                                   replace=False)]))
+                out[t, b, h, :n] = cur
+    return out
 
 
 def seed_for(index: int) -> int:

@@ -26,7 +26,8 @@ SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device
            "hga_debug_inject",
            "hga_workspace_size", "hga_build_summaries", "hga_route_chunks", "hga_route_groups",
            "hga_route", "hga_hot_rows", "hga_gather_host", "hga_attend", "hga_decode_step",
-           "hga_decode_step_launches", "hga_attend_noalloc")
+           "hga_decode_step_launches", "hga_attend_noalloc", "hga_warm_rows", "hga_warm_reset",
+           "hga_gather_warm", "hga_attend_warm")
 
 
 class HGAConfig(ctypes.Structure):
@@ -79,6 +80,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_debug_inject": (I32, [I32]),
         "hga_decode_step_launches": (ctypes.c_int, [C, I64, ctypes.POINTER(I32)]),
         "hga_attend_noalloc": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P]),
+        "hga_warm_rows": (ctypes.c_int, [C, I32, ctypes.POINTER(I64)]),
+        "hga_warm_reset": (ctypes.c_int, [C, I32, P, P, I32, P]),
+        "hga_gather_warm": (ctypes.c_int, [C, P, P, I64, P, P, I32, P, P, P, P, P, I32, P, P]),
+        "hga_attend_warm": (ctypes.c_int, [C, P, P, P, P, I64, P, P, I32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -208,12 +213,47 @@ def hga_decode_step_launches(cfg, n_alloc: int) -> int:
 
 
 def hga_gather_host(cfg, k_host, v_host, n_alloc: int, pos, group_idx, k_work, v_work,
-                    refresh_window: bool = False, stream=None) -> None:
-    """Host tier: stage the routed groups (and window rows) from pinned host K/V."""
+                    refresh_window: int = 0, stream=None) -> None:
+    """Host tier: stage the routed groups and window rows (refresh_window 0: the current
+    chunk up to pos, 1: the whole window, 2: the row at pos only) from pinned host K/V."""
     _check(load_library().hga_gather_host(ctypes.byref(_cfg(cfg)), _ptr(k_host), _ptr(v_host),
                                           n_alloc, _ptr(pos), _ptr(group_idx), _ptr(k_work),
-                                          _ptr(v_work), 1 if refresh_window else 0,
+                                          _ptr(v_work), int(refresh_window),
                                           _stream(stream)), "hga_gather_host")
+
+
+def hga_warm_rows(cfg, warm_groups: int) -> int:
+    """Rows per (sequence, KV head) of the warm tier's device working buffers."""
+    out = ctypes.c_int64(0)
+    _check(load_library().hga_warm_rows(ctypes.byref(_cfg(cfg)), warm_groups, ctypes.byref(out)),
+           "hga_warm_rows")
+    return out.value
+
+
+def hga_warm_reset(cfg, warm_groups: int, tags, stamps, seq: int = -1, stream=None) -> None:
+    """Empty the warm tables of one sequence (or of all, seq=-1)."""
+    _check(load_library().hga_warm_reset(ctypes.byref(_cfg(cfg)), warm_groups, _ptr(tags),
+                                         _ptr(stamps), seq, _stream(stream)), "hga_warm_reset")
+
+
+def hga_gather_warm(cfg, k_host, v_host, n_alloc: int, pos, group_idx, warm_groups: int, tags,
+                    stamps, slot_map, k_work, v_work, refresh_window: int = 0, counters=None,
+                    stream=None) -> None:
+    """Warm tier step: LRU lookup/eviction, then only the missed groups from host K/V."""
+    _check(load_library().hga_gather_warm(ctypes.byref(_cfg(cfg)), _ptr(k_host), _ptr(v_host),
+                                          n_alloc, _ptr(pos), _ptr(group_idx), warm_groups,
+                                          _ptr(tags), _ptr(stamps), _ptr(slot_map), _ptr(k_work),
+                                          _ptr(v_work), int(refresh_window),
+                                          _ptr(counters), _stream(stream)), "hga_gather_warm")
+
+
+def hga_attend_warm(cfg, q, pos, k_work, v_work, n_alloc: int, group_idx, slot_map,
+                    warm_groups: int, out, lse=None, stream=None) -> None:
+    """Decode attention over the warm working buffers (routed groups via slot_map)."""
+    _check(load_library().hga_attend_warm(ctypes.byref(_cfg(cfg)), _ptr(q), _ptr(pos),
+                                          _ptr(k_work), _ptr(v_work), n_alloc, _ptr(group_idx),
+                                          _ptr(slot_map), warm_groups, _ptr(out), _ptr(lse),
+                                          _stream(stream)), "hga_attend_warm")
 
 
 def hga_attend(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse=None,

@@ -254,11 +254,93 @@ hga_status hga_gather_host(const hga_config* cfg, const void* k_host, const void
   if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
   if (!k_host || !v_host || !pos || !group_idx || !k_work || !v_work)
     return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (refresh_window < 0 || refresh_window > 2)
+    return fail(HGA_ERR_INVALID_ARG, "refresh_window %d is not 0, 1 or 2", refresh_window);
   unsigned* err = nullptr;
   if ((st = device_error_ptr(&err)) != HGA_OK) return st;
   cudaError_t e = launch_gather_host(p, k_host, v_host, pos, group_idx, k_work, v_work,
-                                     refresh_window ? 1 : 0, err, static_cast<cudaStream_t>(stream));
+                                     refresh_window, err, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_gather_host");
+}
+
+static hga_status check_warm(const LayerParams& p, int32_t warm_groups) {
+  if (warm_groups < p.kg || warm_groups > kWarmMax)
+    return fail(HGA_ERR_INVALID_ARG, "warm_groups %d outside [topk_groups %d, %d]", warm_groups,
+                p.kg, kWarmMax);
+  return HGA_OK;
+}
+
+hga_status hga_warm_rows(const hga_config* cfg, int32_t warm_groups, int64_t* rows) {
+  if (!rows) return fail(HGA_ERR_INVALID_ARG, "rows is NULL");
+  LayerParams p;
+  hga_status st = make_params(cfg, cfg ? cfg->chunk : 0, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_warm(p, warm_groups)) != HGA_OK) return st;
+  *rows = hot_rows(p, warm_groups);
+  return HGA_OK;
+}
+
+hga_status hga_warm_reset(const hga_config* cfg, int32_t warm_groups, int32_t* tags,
+                          int32_t* stamps, int32_t seq, void* stream) {
+  Range nvtx_range("hga_warm_reset");
+  LayerParams p;
+  hga_status st = make_params(cfg, cfg ? cfg->chunk : 0, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_warm(p, warm_groups)) != HGA_OK) return st;
+  if (!tags || !stamps) return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (seq < -1 || seq >= p.B) return fail(HGA_ERR_INVALID_ARG, "seq %d outside [-1, %d)", seq, p.B);
+  const size_t per_seq = static_cast<size_t>(p.Hkv) * warm_groups;
+  const size_t off = seq < 0 ? 0 : static_cast<size_t>(seq) * per_seq;
+  const size_t count = seq < 0 ? per_seq * p.B : per_seq;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(tags + off, 0xff, count * sizeof(int32_t), s);  // -1: empty
+  if (e == cudaSuccess) e = cudaMemsetAsync(stamps + off, 0, count * sizeof(int32_t), s);
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_warm_reset");
+}
+
+hga_status hga_gather_warm(const hga_config* cfg, const void* k_host, const void* v_host,
+                           int64_t n_alloc, const int64_t* pos, const int32_t* group_idx,
+                           int32_t warm_groups, int32_t* tags, int32_t* stamps, int32_t* slot_map,
+                           void* k_work, void* v_work, int32_t refresh_window, uint64_t* counters,
+                           void* stream) {
+  Range nvtx_range("hga_gather_warm");
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+  if ((st = check_warm(p, warm_groups)) != HGA_OK) return st;
+  if (!k_host || !v_host || !pos || !group_idx || !tags || !stamps || !slot_map || !k_work ||
+      !v_work)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (refresh_window < 0 || refresh_window > 2)
+    return fail(HGA_ERR_INVALID_ARG, "refresh_window %d is not 0, 1 or 2", refresh_window);
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_gather_warm(p, k_host, v_host, pos, group_idx, warm_groups, tags, stamps,
+                                     slot_map, k_work, v_work, refresh_window,
+                                     reinterpret_cast<unsigned long long*>(counters), err,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_gather_warm");
+}
+
+hga_status hga_attend_warm(const hga_config* cfg, const void* q, const int64_t* pos,
+                           const void* k_work, const void* v_work, int64_t n_alloc,
+                           const int32_t* group_idx, const int32_t* slot_map, int32_t warm_groups,
+                           void* out, float* lse, void* stream) {
+  Range nvtx_range("hga_attend_warm");
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+  if ((st = check_warm(p, warm_groups)) != HGA_OK) return st;
+  if (!q || !pos || !k_work || !v_work || !group_idx || !slot_map || !out)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_attend_decode_bf16(p, cfg->out_dtype, q, pos, k_work, v_work, group_idx,
+                                            out, lse, err, 1, static_cast<cudaStream_t>(stream),
+                                            slot_map, warm_groups);
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attend_warm");
 }
 
 hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const int64_t* pos,

@@ -57,6 +57,8 @@ struct DecodeArgs {
   int nsplit;   // warp-splits per (sequence, KV head) = kWarps * cluster size
   int hot;      // K/V are the host tier's device working buffers (see host_tier.cu)
   int64_t rows; // rows per (sequence, KV head) of k / v: n_alloc, or the working-buffer rows
+  const int32_t* slot_map;  // warm tier: cached slot of every group_idx entry, or null
+  int slots;                // warm tier: cached group slots per (sequence, KV head)
 };
 
 template <typename TO>
@@ -157,6 +159,20 @@ attend_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
       n = warp_keep_ascending(
           gl, p.kg, [&](int gid) { return gid / p.Ng >= p.sink && gid / p.Ng < cur - p.local; },
           s_gl, &bad, s_slot);
+      if (a.slot_map) {  // warm tier: the kept entries' cached slots
+        __syncwarp();
+        const int32_t* sm = a.slot_map + static_cast<size_t>(bh) * p.kg;
+        bool bad_slot = false;
+        for (int i = lane; i < n; i += 32) {
+          int s = sm[s_slot[i]];
+          if (s < 0 || s >= a.slots) {
+            bad_slot = true;
+            s = 0;
+          }
+          s_slot[i] = s;
+        }
+        bad |= __any_sync(0xffffffffu, bad_slot);
+      }
     }
     if (lane == 0) {
       s_ng = n;
@@ -230,7 +246,8 @@ int cluster_size(const LayerParams& p) {
 template <typename TO>
 cudaError_t launch_t(const LayerParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                      const void* q, const int64_t* pos, const int32_t* group_idx, void* out,
-                     float* lse, unsigned* err, int hot, int64_t rows, cudaStream_t s) {
+                     float* lse, unsigned* err, int hot, int64_t rows, const int32_t* slot_map,
+                     int slots, cudaStream_t s) {
   const int cl = cluster_size(p);
   DecodeArgs<TO> a;
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -243,6 +260,8 @@ cudaError_t launch_t(const LayerParams& p, const CUtensorMap& tk, const CUtensor
   a.units_per_split = (max_units(p) + a.nsplit - 1) / a.nsplit;
   a.hot = hot;
   a.rows = rows;
+  a.slot_map = slot_map;
+  a.slots = slots;
   cudaError_t e = ensure_smem<attend_decode_bf16_kernel<TO>>(kSmemBytes);
   if (e != cudaSuccess) return e;
   // Programmatic launch (the prologue and the forced units' loads overlap the
@@ -264,16 +283,19 @@ bool decode_fast_path(const LayerParams& p, int dtype) {
 cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const void* q,
                                       const int64_t* pos, const void* k, const void* v,
                                       const int32_t* group_idx, void* out, float* lse,
-                                      unsigned* err, int hot, cudaStream_t s) {
+                                      unsigned* err, int hot, cudaStream_t s,
+                                      const int32_t* slot_map, int slots) {
   CUtensorMap tk, tv;
-  const int64_t rows = hot ? hot_rows(p) : p.n_alloc;
+  const int64_t rows = hot ? hot_rows(p, slot_map ? slots : 0) : p.n_alloc;
   const int64_t all_rows = static_cast<int64_t>(p.B) * p.Hkv * rows;
   cudaError_t e = make_bf16_map(&tk, k, all_rows, kUnit);
   if (e == cudaSuccess) e = make_bf16_map(&tv, v, all_rows, kUnit);
   if (e != cudaSuccess) return e;
   return out_dtype == 0
-             ? launch_t<float>(p, tk, tv, q, pos, group_idx, out, lse, err, hot, rows, s)
-             : launch_t<__nv_bfloat16>(p, tk, tv, q, pos, group_idx, out, lse, err, hot, rows, s);
+             ? launch_t<float>(p, tk, tv, q, pos, group_idx, out, lse, err, hot, rows,
+                                             slot_map, slots, s)
+             : launch_t<__nv_bfloat16>(p, tk, tv, q, pos, group_idx, out, lse, err, hot,
+                                                     rows, slot_map, slots, s);
 }
 
 }  // namespace hga

@@ -136,21 +136,37 @@ size_t attend_workspace_bytes(const LayerParams& p, int dtype);
 // The bf16, D = 128 decode kernel (TMA + mma.sync, in-cluster merge, no
 // workspace) applies to p.
 bool decode_fast_path(const LayerParams& p, int dtype);
-// hot != 0: k / v are the host tier's device working buffers (hot_rows(p)
-// rows per (sequence, KV head)) instead of the device cache.
+// hot != 0: k / v are the host tier's device working buffers (hot_rows(p,
+// slots) rows per (sequence, KV head)) instead of the device cache.  With
+// slot_map (warm tier) routed entry j sits at cached slot slot_map[j] of
+// `slots`; without, at slot j.
 cudaError_t launch_attend_decode_bf16(const LayerParams& p, int out_dtype, const void* q,
                                       const int64_t* pos, const void* k, const void* v,
                                       const int32_t* group_idx, void* out, float* lse,
-                                      unsigned* err, int hot, cudaStream_t s);
+                                      unsigned* err, int hot, cudaStream_t s,
+                                      const int32_t* slot_map = nullptr, int slots = 0);
 
 // Host tier: rows per (sequence, KV head) of the device working buffers:
-// sink chunks, a ring of local+1 chunks, and kg routed groups.
-__host__ __device__ inline int64_t hot_rows(const LayerParams& p) {
-  return static_cast<int64_t>(p.sink + p.local + 1) * p.C + static_cast<int64_t>(p.kg) * p.g;
+// sink chunks, a ring of local+1 chunks, and kg routed groups (or, with the
+// warm tier, `slots` cached groups).
+__host__ __device__ inline int64_t hot_rows(const LayerParams& p, int slots = 0) {
+  return static_cast<int64_t>(p.sink + p.local + 1) * p.C +
+         static_cast<int64_t>(slots > 0 ? slots : p.kg) * p.g;
 }
 cudaError_t launch_gather_host(const LayerParams& p, const void* k_host, const void* v_host,
                                const int64_t* pos, const int32_t* group_idx, void* k_work,
                                void* v_work, int refresh_window, unsigned* err, cudaStream_t s);
+
+// Warm tier: at most kWarmMax cached groups per (sequence, KV head).
+constexpr int kWarmMax = 2048;
+// One step of the warm tier (host_tier.cu): LRU lookup and eviction in
+// tags / stamps [B*Hkv][slots], slot_map [B*Hkv][kg] written, misses and the
+// window rows copied from the host cache.  counters (hits, misses) may be null.
+cudaError_t launch_gather_warm(const LayerParams& p, const void* k_host, const void* v_host,
+                               const int64_t* pos, const int32_t* group_idx, int slots,
+                               int32_t* tags, int32_t* stamps, int32_t* slot_map, void* k_work,
+                               void* v_work, int refresh_window, unsigned long long* counters,
+                               unsigned* err, cudaStream_t s);
 
 // The bf16, D = 128 prefill kernel (64-query blocks on tcgen05 / TMEM) applies to p.
 bool prefill_tc_path(const LayerParams& p, int dtype);

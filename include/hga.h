@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define HGA_ABI_VERSION 2
+#define HGA_ABI_VERSION 3
 
 typedef enum hga_status {
   HGA_OK = 0,
@@ -237,11 +237,15 @@ hga_status hga_hot_rows(const hga_config* cfg, int64_t* rows);
 /*
  * Fills the working buffers for one decode step at pos (host tier): copies from
  * the pinned host cache the routed groups of group_idx (as hga_route_groups
- * or hga_route wrote it; the same groups hga_attend keeps) and the current
- * chunk's rows up to pos; with refresh_window != 0 also the sink and local
- * chunks (after a prefill, or whenever the window is stale: a decode loop that
- * calls this at every consecutive position keeps it current; after positions
- * are skipped, pass refresh_window).  The copy is a
+ * or hga_route wrote it; the same groups hga_attend keeps) and window rows,
+ * by refresh_window:
+ *   0  the current chunk's rows up to pos (a decode loop that calls this at
+ *      every consecutive position keeps the whole window current);
+ *   1  those and the sink and local chunks (after a prefill, or after
+ *      positions are skipped);
+ *   2  the row at pos only: valid when the previous call for every sequence
+ *      was at pos - 1 (a consecutive decode loop after one call with 1).
+ * Any other value is HGA_ERR_INVALID_ARG.  The copy is a
  * kernel reading host memory directly (zero-copy 16-byte loads over the host
  * link); nothing is allocated.
  *   k_host, v_host  pinned host [B, Hkv, n_alloc, 128] bf16
@@ -250,6 +254,72 @@ hga_status hga_hot_rows(const hga_config* cfg, int64_t* rows);
 hga_status hga_gather_host(const hga_config* cfg, const void* k_host, const void* v_host,
                            int64_t n_alloc, const int64_t* pos, const int32_t* group_idx,
                            void* k_work, void* v_work, int32_t refresh_window, void* stream);
+
+/*
+ * Warm tier (HGA technical summary, "Architettura della Memoria": a bounded
+ * LRU cache in VRAM of recently routed spans, between the VRAM hot tier and
+ * the host RAM history).  The cached unit is a routed group.  Per (sequence,
+ * KV head) the working buffer's routed region holds warm_groups group slots
+ * (topk_groups <= warm_groups <= 2048), described by a table in device memory:
+ *   tags    int32 [B, Hkv, warm_groups]: group id held by each slot, -1 empty
+ *   stamps  int32 [B, Hkv, warm_groups]: decode step of last use, 0 empty
+ * A step's requests are the groups hga_attend keeps from group_idx (valid,
+ * in a candidate chunk, strictly ascending).  The step clock of a (sequence,
+ * KV head) is one more than its largest stamp; hits take it as stamp; the
+ * misses, ascending, replace empty slots (by slot index) first, then the
+ * least recently used (stamp, then group id, ascending), never a slot hit in
+ * the same step.  A cached group's rows are copies of the host cache: when a
+ * sequence's history changes (a new sequence in that batch slot, positions
+ * moving backwards, K/V rewritten), reset its table.
+ *
+ * Rows per (sequence, KV head) of the warm working buffers:
+ *   [sink chunks | ring of local+1 chunks | warm_groups cached groups].
+ */
+hga_status hga_warm_rows(const hga_config* cfg, int32_t warm_groups, int64_t* rows);
+
+/*
+ * Empties the warm tables of sequence seq (seq == -1: every sequence):
+ * tags = -1, stamps = 0, with two memsets on stream.  Call once before the
+ * first hga_gather_warm and whenever a sequence's history changes.
+ */
+hga_status hga_warm_reset(const hga_config* cfg, int32_t warm_groups, int32_t* tags,
+                          int32_t* stamps, int32_t seq, void* stream);
+
+/*
+ * One decode step of the warm tier: for every (sequence, KV head), one CTA
+ * looks its routed groups up in the table, assigns the misses their slots,
+ * writes the table and slot_map, and copies from the pinned host cache only
+ * the missed groups' rows, plus the window rows that refresh_window (0, 1 or
+ * 2) names, as hga_gather_host does.
+ *   k_host, v_host  pinned host [B, Hkv, n_alloc, 128] bf16
+ *   group_idx       device int32 [B, Hkv, topk_groups] from the routing
+ *   tags, stamps    the table above (read and written)
+ *   slot_map        device int32 [B, Hkv, topk_groups], written: the slot of
+ *                   every group_idx entry, -1 where the entry is not kept
+ *   k_work, v_work  device [B, Hkv, hga_warm_rows(), 128] bf16; cached slots
+ *                   keep their rows from step to step
+ *   counters        optional device uint64 [2]: hits and misses added
+ * Nothing is allocated.  Built for bf16, head_dim 128 decode.
+ */
+hga_status hga_gather_warm(const hga_config* cfg, const void* k_host, const void* v_host,
+                           int64_t n_alloc, const int64_t* pos, const int32_t* group_idx,
+                           int32_t warm_groups, int32_t* tags, int32_t* stamps, int32_t* slot_map,
+                           void* k_work, void* v_work, int32_t refresh_window, uint64_t* counters,
+                           void* stream);
+
+/*
+ * The exact attention of hga_attend (decode) over the warm working buffers:
+ * routed entry j of group_idx is read from cached slot slot_map[j] (as
+ * hga_gather_warm wrote it for the same group_idx).  Same units in the same
+ * order as the device-resident and host-tier paths, so the same bits.  A kept
+ * entry whose slot is outside [0, warm_groups) reads slot 0 and is flagged
+ * (HGA_ERR_DEVICE_CHECK from hga_device_status).
+ *   out  device [B, Hq, 1, 128] of cfg->out_dtype;  lse optional float32 [B, Hq, 1]
+ */
+hga_status hga_attend_warm(const hga_config* cfg, const void* q, const int64_t* pos,
+                           const void* k_work, const void* v_work, int64_t n_alloc,
+                           const int32_t* group_idx, const int32_t* slot_map, int32_t warm_groups,
+                           void* out, float* lse, void* stream);
 
 /*
  * Steps 4-5 - gather of the selected tokens' original K/V and exact softmax

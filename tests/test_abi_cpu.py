@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     from hierarchical_sparse_attention_hga_b200 import binding as B
-    assert B.hga_abi_version() == 2
+    assert B.hga_abi_version() == 3
     assert B.hga_status_string(0) == "HGA_OK"
     assert B.hga_status_string(6) == "HGA_ERR_DEVICE_CHECK"
     assert B.hga_status_string(99) == "HGA_ERR_UNKNOWN"
@@ -134,3 +134,37 @@ def test_decode_step_rejects_what_it_does_not_fuse(lib):
     with pytest.raises(B.HGAError) as e:
         B.hga_decode_step(host, 16, 16, 16, 16, 4096, 16, 16, 16, 16, 16, stream=0)
     assert e.value.status == 3
+
+
+def test_warm_tier_sizes_and_refusals(lib):
+    """hga_warm_rows: the window rows plus warm_groups groups; warm_groups below
+    topk_groups or above 2048, and null tables, are refused on the host."""
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    layer = B.Layer(batch=2, heads_q=32, heads_kv=8, head_dim=128)
+    window = (layer.sink_chunks + layer.local_chunks + 1) * layer.chunk
+    assert B.hga_hot_rows(layer) == window + layer.topk_groups * layer.group
+    for m in (layer.topk_groups, 100, 2048):
+        assert B.hga_warm_rows(layer, m) == window + m * layer.group
+    for m in (layer.topk_groups - 1, 2049, -1):
+        with pytest.raises(B.HGAError) as e:
+            B.hga_warm_rows(layer, m)
+        assert e.value.status == 1
+    with pytest.raises(B.HGAError) as e:
+        B.hga_warm_reset(layer, 64, None, 16, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(B.HGAError) as e:
+        B.hga_warm_reset(layer, 64, 16, 16, seq=2, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(B.HGAError) as e:
+        B.hga_gather_warm(layer, 16, 16, 4096, 16, 16, 64, 16, 16, None, 16, 16, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(B.HGAError) as e:
+        B.hga_attend_warm(layer, 16, 16, 16, 16, 4096, 16, 16, 16, 16, stream=0)
+    assert e.value.status == 1   # warm_groups 16 < topk_groups
+    for fn in (lambda: B.hga_gather_host(layer, 16, 16, 4096, 16, 16, 16, 16, refresh_window=3,
+                                         stream=0),
+               lambda: B.hga_gather_warm(layer, 16, 16, 4096, 16, 16, 64, 16, 16, 16, 16, 16,
+                                         refresh_window=-1, stream=0)):
+        with pytest.raises(B.HGAError) as e:
+            fn()
+        assert e.value.status == 1   # window modes are 0, 1 and 2

@@ -89,9 +89,11 @@ def test_host_tier_decode_matches_oracle():
             compare_head(wl, x, res, b, h)
 
 
-def test_host_tier_equals_device_path_step_by_step():
+@pytest.mark.parametrize("mode", [0, 2])
+def test_host_tier_equals_device_path_step_by_step(mode):
     """Decode steps across chunk boundaries: the window ring and the staged groups
-    give the same bits as the device-resident cache."""
+    give the same bits as the device-resident cache (window mode 0: the current
+    chunk re-copied each step; 2: only the newest row)."""
     wl = S.workload("host_tier_decode_128k", batch=2, context=4096, heads_q=8, heads_kv=2)
     x = S.make_inputs(wl, 42)
     r = Runner(wl, x)
@@ -101,7 +103,7 @@ def test_host_tier_equals_device_path_step_by_step():
         pos = np.array([p, p - 3], dtype=np.int64)
         r.summaries(p, p + 1, host=False)
         dev_out, dev_lse, dev_gi = r.step(pos, host=False)
-        host_out, host_lse, host_gi = r.step(pos, host=True, refresh=(step == 0))
+        host_out, host_lse, host_gi = r.step(pos, host=True, refresh=1 if step == 0 else mode)
         assert np.array_equal(dev_gi, host_gi)
         assert np.array_equal(dev_out, host_out), f"step at {p}"
         assert np.array_equal(dev_lse, host_lse)

@@ -27,7 +27,8 @@ SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device
            "hga_workspace_size", "hga_build_summaries", "hga_route_chunks", "hga_route_groups",
            "hga_route", "hga_hot_rows", "hga_gather_host", "hga_attend", "hga_decode_step",
            "hga_decode_step_launches", "hga_attend_noalloc", "hga_warm_rows", "hga_warm_reset",
-           "hga_gather_warm", "hga_attend_warm")
+           "hga_gather_warm", "hga_attend_warm", "hga_build_summaries_paged",
+           "hga_decode_step_paged")
 
 
 class HGAConfig(ctypes.Structure):
@@ -41,6 +42,13 @@ class HGAConfig(ctypes.Structure):
                 ("n_high_pairs", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("out_dtype", ctypes.c_int32), ("kv_loc", ctypes.c_int32),
                 ("rope_theta", ctypes.c_double)]
+
+
+class HGAKvPages(ctypes.Structure):
+    """Mirror of struct hga_kv_pages (a paged K/V pool's block table)."""
+
+    _fields_ = [("block_table", ctypes.c_void_p), ("n_pages", ctypes.c_int64),
+                ("page_size", ctypes.c_int32), ("max_pages", ctypes.c_int32)]
 
 
 class HGAError(RuntimeError):
@@ -63,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     C = ctypes.POINTER(HGAConfig)
+    KV = ctypes.POINTER(HGAKvPages)
     sig = {
         "hga_abi_version": (I32, []),
         "hga_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -84,6 +93,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_warm_reset": (ctypes.c_int, [C, I32, P, P, I32, P]),
         "hga_gather_warm": (ctypes.c_int, [C, P, P, I64, P, P, I32, P, P, P, P, P, I32, P, P]),
         "hga_attend_warm": (ctypes.c_int, [C, P, P, P, P, I64, P, P, I32, P, P, P]),
+        "hga_build_summaries_paged": (ctypes.c_int, [C, P, KV, P, P, P, P]),
+        "hga_decode_step_paged": (ctypes.c_int, [C, P, P, P, P, P, P, KV, P, P, P, P, P, P, I32,
+                                                 P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -274,6 +286,33 @@ def hga_decode_step(cfg, q, pos, chunk_sum, group_sum, n_alloc: int, k, v, chunk
                                           _ptr(group_idx), _ptr(group_score), _ptr(out),
                                           _ptr(lse), 1 if append else 0, _stream(stream)),
            "hga_decode_step")
+
+
+def kv_pages(block_table, n_pages: int, page_size: int, max_pages: int) -> HGAKvPages:
+    """A paged pool's description: block_table (device int32 [B, max_pages]) and sizes."""
+    return HGAKvPages(_ptr(block_table), n_pages, page_size, max_pages)
+
+
+def hga_build_summaries_paged(cfg, k_pages, kv: HGAKvPages, seq_len, chunk_sum, group_sum,
+                              stream=None) -> None:
+    """Summaries of a ragged batch over a paged pool: sequence b's rows up to seq_len[b]."""
+    _check(load_library().hga_build_summaries_paged(ctypes.byref(_cfg(cfg)), _ptr(k_pages),
+                                                    ctypes.byref(kv), _ptr(seq_len),
+                                                    _ptr(chunk_sum), _ptr(group_sum),
+                                                    _stream(stream)), "hga_build_summaries_paged")
+
+
+def hga_decode_step_paged(cfg, q, pos, chunk_sum, group_sum, k_pages, v_pages, kv: HGAKvPages,
+                          chunk_idx, group_idx, out, lse=None, chunk_score=None, group_score=None,
+                          append: bool = False, stream=None) -> None:
+    """hga_decode_step over a paged pool (one launch)."""
+    _check(load_library().hga_decode_step_paged(ctypes.byref(_cfg(cfg)), _ptr(q), _ptr(pos),
+                                                _ptr(chunk_sum), _ptr(group_sum), _ptr(k_pages),
+                                                _ptr(v_pages), ctypes.byref(kv), _ptr(chunk_idx),
+                                                _ptr(chunk_score), _ptr(group_idx),
+                                                _ptr(group_score), _ptr(out), _ptr(lse),
+                                                1 if append else 0, _stream(stream)),
+           "hga_decode_step_paged")
 
 
 def hga_debug_inject(flags: int) -> int:

@@ -404,4 +404,66 @@ hga_status hga_decode_step_launches(const hga_config* cfg, int64_t n_alloc, int3
   return HGA_OK;
 }
 
+// Checks a paged pool and derives p for n_alloc = max_pages * page_size.
+static hga_status paged_params(const hga_config* cfg, const hga_kv_pages* kv, LayerParams* p,
+                               KvPages* out) {
+  if (!kv || !kv->block_table) return fail(HGA_ERR_INVALID_ARG, "null block table");
+  if (kv->page_size <= 0 || kv->page_size % 16 != 0)
+    return fail(HGA_ERR_INVALID_ARG, "page_size %d is not a positive multiple of 16", kv->page_size);
+  if (kv->max_pages <= 0 || kv->n_pages <= 0)
+    return fail(HGA_ERR_INVALID_ARG, "max_pages and n_pages must be positive");
+  const int64_t n_alloc = static_cast<int64_t>(kv->max_pages) * kv->page_size;
+  hga_status st = make_params(cfg, n_alloc, 1, p);
+  if (st != HGA_OK) return st;
+  if (kv->n_pages * p->Hkv * kv->page_size >= (static_cast<int64_t>(1) << 31))
+    return fail(HGA_ERR_UNSUPPORTED, "the pool has 2^31 rows or more");
+  *out = KvPages{kv->block_table, kv->page_size, kv->max_pages, kv->n_pages};
+  return HGA_OK;
+}
+
+hga_status hga_build_summaries_paged(const hga_config* cfg, const void* k_pages,
+                                     const hga_kv_pages* kv, const int64_t* seq_len,
+                                     float* chunk_sum, float* group_sum, void* stream) {
+  Range nvtx_range("hga_build_summaries_paged");
+  LayerParams p;
+  KvPages pages;
+  hga_status st = paged_params(cfg, kv, &p, &pages);
+  if (st != HGA_OK) return st;
+  if (!k_pages || !seq_len || !chunk_sum || !group_sum)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_summaries_paged(p, cfg->dtype, k_pages, pages, seq_len, chunk_sum,
+                                         group_sum, err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_build_summaries_paged");
+}
+
+hga_status hga_decode_step_paged(const hga_config* cfg, const void* q, const int64_t* pos,
+                                 float* chunk_sum, float* group_sum, const void* k_pages,
+                                 const void* v_pages, const hga_kv_pages* kv, int32_t* chunk_idx,
+                                 float* chunk_score, int32_t* group_idx, float* group_score,
+                                 void* out, float* lse, int32_t append, void* stream) {
+  Range nvtx_range("hga_decode_step_paged");
+  LayerParams p;
+  KvPages pages;
+  hga_status st = paged_params(cfg, kv, &p, &pages);
+  if (st != HGA_OK) return st;
+  if (!q || !pos || !chunk_sum || !group_sum || !k_pages || !v_pages || !chunk_idx ||
+      !group_idx || !out)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (cfg->kv_loc != HGA_KV_DEVICE || !decode_fast_path(p, cfg->dtype) ||
+      !decode_item_path(p, pages.max_pages))
+    return fail(HGA_ERR_UNSUPPORTED,
+                "hga_decode_step_paged is one launch of the decode-step kernel: bf16, head_dim "
+                "128, group 16, top-k within its limits and a block-table row that fits in "
+                "shared memory");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_decode_step(p, cfg->out_dtype, q, pos, chunk_sum, group_sum, k_pages,
+                                     v_pages, chunk_idx, chunk_score, group_idx, group_score,
+                                     out, lse, append != 0, err,
+                                     static_cast<cudaStream_t>(stream), pages);
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_decode_step_paged");
+}
+
 }  // extern "C"

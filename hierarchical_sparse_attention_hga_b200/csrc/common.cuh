@@ -15,6 +15,7 @@ enum DeviceErr : unsigned {
   kErrChunkIdx = 1u << 2,     // chunk_idx entry not a complete candidate chunk / not ascending
   kErrGroupIdx = 1u << 3,     // group_idx entry not a group of a candidate chunk
   kErrTimeout = 1u << 4,      // a bounded wait gave up
+  kErrPage = 1u << 5,         // a block-table entry a step needs is not a page of the pool
 };
 
 // Layer parameters as the kernels see them (derived from hga_config).
@@ -29,6 +30,25 @@ struct LayerParams {
   double theta;
   unsigned debug;             // test hooks (kDebug* bits); 0 in normal use
 };
+
+// Paged K/V: k and v are pools [n_pages][Hkv][page_size][D]; token t of
+// sequence b lives in page block_table[b * max_pages + t / page_size], row
+// t % page_size.  page_size is a multiple of 16, so a group (and every 16-row
+// tile the kernels move) never straddles two pages.  block_table == nullptr:
+// the dense layout [B][Hkv][n_alloc][D].
+struct KvPages {
+  const int32_t* block_table;
+  int page_size;
+  int max_pages;   // entries per sequence; n_alloc = max_pages * page_size
+  int64_t n_pages;
+};
+
+// Row of token t of (b, h) in the [rows][D] view of a paged pool, given its
+// page (validated by the caller).
+__host__ __device__ __forceinline__ int64_t paged_row(const KvPages& kv, int Hkv, int h,
+                                                     int32_t page, int64_t t) {
+  return (static_cast<int64_t>(page) * Hkv + h) * kv.page_size + t % kv.page_size;
+}
 
 // Test hook of the one-launch decode step: warp 0 skips its first group-summary
 // copy of the first item of each CTA but still waits for it, so that bounded wait

@@ -221,7 +221,7 @@ __device__ __forceinline__ float score16(const float* rows, const float4 (&qv)[k
 constexpr int kL2Max = kKcMax * 8;  // level-2 candidates: chosen chunks x groups per chunk
 
 struct StepSmem {  // byte offsets into the dynamic shared memory (after alignment)
-  int W, n_tab;
+  int W, n_tab, n_pt;  // n_pt: block-table entries staged per item (paged pools), else 0
   __host__ __device__ size_t rings() const { return static_cast<size_t>(W) * kS * kStageBytes; }
   __host__ __device__ size_t o_union() const { return rings(); }                    // u64 [W][kKcMax]
   __host__ __device__ size_t o_ckey() const { return o_union() + static_cast<size_t>(W) * kKcMax * 8; }
@@ -232,7 +232,8 @@ struct StepSmem {  // byte offsets into the dynamic shared memory (after alignme
   __host__ __device__ size_t o_glist() const { return o_chunks() + kKcMax * 4; }    // int [kKgMax]
   __host__ __device__ size_t o_gsum() const { return o_glist() + kKgMax * 4; }      // float [8][kD]
   __host__ __device__ size_t o_tab() const { return o_gsum() + 8 * kD * 4; }        // float2 [n_tab]
-  __host__ __device__ size_t bytes() const { return 1024 + o_tab() + static_cast<size_t>(n_tab) * 8; }
+  __host__ __device__ size_t o_pages() const { return o_tab() + static_cast<size_t>(n_tab) * 8; }  // int [n_pt]
+  __host__ __device__ size_t bytes() const { return 1024 + o_pages() + static_cast<size_t>(n_pt) * 4; }
 };
 
 template <typename TO>
@@ -252,6 +253,7 @@ struct StepArgs {
   unsigned* err;
   int append;
   int n_items;
+  KvPages kv;               // paged pools (the PAGED kernels); block_table null otherwise
 };
 
 // 2 MB pages of each of the item's group-summary, K and V regions whose address
@@ -282,7 +284,12 @@ __device__ __forceinline__ int rank_among(const uint64_t* keys, int n, uint64_t 
 // current) loads right behind its own group-summary copies; they land while the
 // level-2 selection runs.
 
-template <int W, int R1, typename TO>
+// PAGED: k and v are page pools (KvPages); each item stages its sequence's
+// block-table row in shared memory (asynchronous copies issued at the item's
+// start, validated before the first barrier), and every K/V tile's row comes
+// from it.  An entry that is not a page of the pool is flagged and read as
+// zeros (its tiles start at a negative row, which the tensor copy fills).
+template <int W, int R1, typename TO, bool PAGED>
 __global__ void __launch_bounds__((W + 1) * 32, W == 7 ? 1 : 2)
 decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, StepArgs<TO> a, LayerParams p) {
@@ -294,7 +301,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;  // streaming threads: 0 .. W * 32 - 1
   uint8_t* base = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
-  StepSmem L{W, summ::table_entries(p, kD)};
+  StepSmem L{W, summ::table_entries(p, kD), PAGED ? a.kv.max_pages : 0};
   uint64_t* s_union = reinterpret_cast<uint64_t*>(base + L.o_union());
   uint64_t* ckey = reinterpret_cast<uint64_t*>(base + L.o_ckey());  // chosen chunks' keys, rank order
   uint64_t* gkey = reinterpret_cast<uint64_t*>(base + L.o_gkey());
@@ -304,6 +311,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
   int* glist = reinterpret_cast<int*>(base + L.o_glist());    // routed groups, rank order
   float(*gsum)[kD] = reinterpret_cast<float(*)[kD]>(base + L.o_gsum());
   float2* tab = reinterpret_cast<float2*>(base + L.o_tab());
+  int* s_pages = reinterpret_cast<int*>(base + L.o_pages());  // PAGED: the item's block-table row
 
   if (threadIdx.x == 0) {
     ptx::prefetch_tensormap(&tm_k);
@@ -322,12 +330,20 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
       __syncwarp();
       pdl_wait();  // the rows read and written may belong to the kernel just before
       for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
-        const int64_t pb = a.pos[item / p.Hkv];
+        const int b = item / p.Hkv, h = item % p.Hkv;
+        const int64_t pb = a.pos[b];
         if (pb < 0 || pb >= p.n_alloc) continue;
-        summ::append_closed_rows<__nv_bfloat16, kD>(
-            a.k + static_cast<size_t>(item) * p.n_alloc * kD,
-            a.chunk_sum + static_cast<size_t>(item) * p.n_chunks * kD,
+        auto group_rows = [&](int64_t g0) -> const __nv_bfloat16* {
+          if (!PAGED) return a.k + (static_cast<size_t>(item) * p.n_alloc + g0) * kD;
+          const int32_t pg = __ldg(a.kv.block_table + static_cast<size_t>(b) * a.kv.max_pages +
+                                   g0 / a.kv.page_size);
+          if (pg < 0 || pg >= a.kv.n_pages) return nullptr;
+          return a.k + static_cast<size_t>(paged_row(a.kv, p.Hkv, h, pg, g0)) * kD;
+        };
+        const bool rows_ok = summ::append_closed_rows<__nv_bfloat16, kD>(
+            group_rows, a.chunk_sum + static_cast<size_t>(item) * p.n_chunks * kD,
             a.group_sum + static_cast<size_t>(item) * p.n_chunks * p.Ng * kD, p, pb, tab, gsum);
+        if (!rows_ok && lane == 0) flag_error(a.err, kErrPage);
       }
     }
     cta_sync();
@@ -368,6 +384,15 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
     const float* cbase = a.chunk_sum + (static_cast<size_t>(item) * p.n_chunks + p.sink) * kD;
     const float* gbase = a.group_sum + static_cast<size_t>(item) * p.n_chunks * p.Ng * kD;
     const int64_t row_base = static_cast<int64_t>(item) * p.n_alloc;
+    if (PAGED) {  // the sequence's block-table row, landing while the scan runs
+      const int32_t* bt = a.kv.block_table + static_cast<size_t>(b) * a.kv.max_pages;
+      for (int i = tid; i < a.kv.max_pages; i += W * 32) ptx::cp_async4(s_pages + i, bt + i);
+    }
+    // row of token t of this item in the [rows][D] view of k / v
+    auto kv_row = [&](int64_t t) -> int32_t {
+      if (!PAGED) return static_cast<int32_t>(row_base + t);
+      return static_cast<int32_t>(paged_row(a.kv, p.Hkv, h, s_pages[t / a.kv.page_size], t));
+    };
 
     // 1. position, routing query and Q fragments: independent loads, issued first so
     //    that they do not queue behind the bulk copies below
@@ -386,7 +411,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
     load_q_frags(a.q, p, b, h, qa);
     // warm the address translation of the item's group-summary and K/V regions
     // (read later at scattered places) while the scan runs
-    if (warp == 0 && lane < 3 * kTlbPages) {
+    if (warp == 0 && lane < (PAGED ? 1 : 3) * kTlbPages) {
       const int which = lane / kTlbPages, page = lane % kTlbPages;
       const size_t span = which == 0 ? static_cast<size_t>(p.n_chunks) * p.Ng * kD * 4
                                      : static_cast<size_t>(p.n_alloc) * kD * 2;
@@ -472,11 +497,10 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
                                static_cast<uint32_t>(p.Ng) * kRowBytes, bar);
             }
           } else if (i < e_rt) {
-            issue_unit(&tm_k, &tm_v, st, bar,
-                       static_cast<int32_t>(row_base + forced_token(warp + (i - e_fw) * W)));
+            issue_unit(&tm_k, &tm_v, st, bar, kv_row(forced_token(warp + (i - e_fw) * W)));
           } else {
             issue_unit(&tm_k, &tm_v, st, bar,
-                       static_cast<int32_t>(row_base + static_cast<int64_t>(glist[warp + (i - e_rt) * W]) * kUnit));
+                       kv_row(static_cast<int64_t>(glist[warp + (i - e_rt) * W]) * kUnit));
           }
         }
         ++issued;
@@ -517,6 +541,17 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
     for (int r = 0; r < R1; ++r)
       if (r * 32 + lane < p.kc) s_union[warp * p.kc + r * 32 + lane] = l1[r];
+    if (PAGED) {  // this thread's block-table copies: landed; the entries the item reads, checked
+      ptx::cp_async_wait_all();
+      const int last = ok ? static_cast<int>(pb / a.kv.page_size) : -1;
+      for (int i = tid; i <= last; i += W * 32) {
+        const int pg = s_pages[i];
+        if (pg < 0 || pg >= a.kv.n_pages) {
+          flag_error(a.err, kErrPage);
+          s_pages[i] = -1;
+        }
+      }
+    }
     named_sync(kBarStream, W * 32);  // B1
 
     // ---- level 1: the kc best of the W lists, by rank, into chunks (rank order)
@@ -689,38 +724,45 @@ StepShape step_shape(const LayerParams& p) {
   return s;
 }
 
-size_t step_smem_bytes(const LayerParams& p, int W) {
-  return StepSmem{W, summ::table_entries(p, kD)}.bytes();
+size_t step_smem_bytes(const LayerParams& p, int W, int n_pt) {
+  return StepSmem{W, summ::table_entries(p, kD), n_pt}.bytes();
 }
 
-template <int W, int R1, typename TO>
+template <int W, int R1, typename TO, bool PAGED>
 cudaError_t launch_t(const LayerParams& p, int grid, const CUtensorMap& tk, const CUtensorMap& tv,
                      const StepArgs<TO>& a, cudaStream_t s) {
-  const size_t smem = step_smem_bytes(p, W);
-  cudaError_t e = ensure_smem<decode_step_kernel<W, R1, TO>>(smem);
+  const size_t smem = step_smem_bytes(p, W, PAGED ? a.kv.max_pages : 0);
+  cudaError_t e = ensure_smem<decode_step_kernel<W, R1, TO, PAGED>>(smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_step_kernel<W, R1, TO>, dim3(grid), dim3((W + 1) * 32), smem, s, 1,
-                    tk, tv, a, p);
+  return launch_pdl(decode_step_kernel<W, R1, TO, PAGED>, dim3(grid), dim3((W + 1) * 32), smem, s,
+                    1, tk, tv, a, p);
 }
 
-template <typename TO>
+template <typename TO, bool PAGED>
 cudaError_t dispatch(const LayerParams& p, const StepShape& sh, const CUtensorMap& tk,
                      const CUtensorMap& tv, const StepArgs<TO>& a, cudaStream_t s) {
   if (sh.W == 7)
-    return sh.R1 == 1 ? launch_t<7, 1, TO>(p, sh.grid, tk, tv, a, s)
-                      : launch_t<7, 2, TO>(p, sh.grid, tk, tv, a, s);
-  return sh.R1 == 1 ? launch_t<3, 1, TO>(p, sh.grid, tk, tv, a, s)
-                    : launch_t<3, 2, TO>(p, sh.grid, tk, tv, a, s);
+    return sh.R1 == 1 ? launch_t<7, 1, TO, PAGED>(p, sh.grid, tk, tv, a, s)
+                      : launch_t<7, 2, TO, PAGED>(p, sh.grid, tk, tv, a, s);
+  return sh.R1 == 1 ? launch_t<3, 1, TO, PAGED>(p, sh.grid, tk, tv, a, s)
+                    : launch_t<3, 2, TO, PAGED>(p, sh.grid, tk, tv, a, s);
+}
+
+template <typename TO>
+cudaError_t dispatch_kv(const LayerParams& p, const StepShape& sh, const CUtensorMap& tk,
+                        const CUtensorMap& tv, const StepArgs<TO>& a, cudaStream_t s) {
+  return a.kv.block_table ? dispatch<TO, true>(p, sh, tk, tv, a, s)
+                          : dispatch<TO, false>(p, sh, tk, tv, a, s);
 }
 
 }  // namespace
 
-bool decode_item_path(const LayerParams& p) {
+bool decode_item_path(const LayerParams& p, int n_pt) {
   const StepShape sh = step_shape(p);
   // dynamic shared memory: one CTA per SM may take 225 KB, two per SM 112 KB each
   const size_t limit = sh.W == 7 ? 225 * 1024 : 112 * 1024;
   return p.kc <= kKcMax && p.kg <= kKgMax && p.Ng <= 8 &&
-         kRows % p.Ng == 0 && step_smem_bytes(p, sh.W) <= limit;
+         kRows % p.Ng == 0 && step_smem_bytes(p, sh.W, n_pt) <= limit;
 }
 
 bool decode_step_path(const LayerParams& p, int dtype) {
@@ -732,8 +774,13 @@ cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* 
                                const int64_t* pos, float* chunk_sum, float* group_sum,
                                const void* k, const void* v, int32_t* chunk_idx,
                                float* chunk_score, int32_t* group_idx, float* group_score,
-                               void* out, float* lse, int append, unsigned* err, cudaStream_t s) {
-  if (!decode_item_path(p)) {  // the summary append, the routing kernel, then the attention kernel
+                               void* out, float* lse, int append, unsigned* err, cudaStream_t s,
+                               const KvPages& kv) {
+  const bool paged = kv.block_table != nullptr;
+  if (!decode_item_path(p, paged ? kv.max_pages : 0)) {
+    // the summary append, the routing kernel, then the attention kernel (dense
+    // caches only: the caller checks that a paged step fits the one launch)
+    if (paged) return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (append) e = launch_append_per_sequence(p, 1, k, pos, chunk_sum, group_sum, s);
     if (e == cudaSuccess)
@@ -743,7 +790,8 @@ cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* 
     return launch_attend_decode_bf16(p, out_dtype, q, pos, k, v, group_idx, out, lse, err, 0, s);
   }
   CUtensorMap tk, tv;
-  const int64_t all_rows = static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc;
+  const int64_t all_rows = paged ? kv.n_pages * p.Hkv * kv.page_size
+                                 : static_cast<int64_t>(p.B) * p.Hkv * p.n_alloc;
   cudaError_t e = make_bf16_map(&tk, k, all_rows, kUnit);
   if (e == cudaSuccess) e = make_bf16_map(&tv, v, all_rows, kUnit);
   if (e != cudaSuccess) return e;
@@ -753,13 +801,13 @@ cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* 
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
   if (out_dtype == 0) {
     StepArgs<float> a{qb, pos, kb, static_cast<const __nv_bfloat16*>(v), chunk_sum, group_sum, chunk_idx, chunk_score, group_idx,
-                      group_score, static_cast<float*>(out), lse, err, append, n_items};
-    return dispatch<float>(p, sh, tk, tv, a, s);
+                      group_score, static_cast<float*>(out), lse, err, append, n_items, kv};
+    return dispatch_kv<float>(p, sh, tk, tv, a, s);
   }
   StepArgs<__nv_bfloat16> a{qb, pos, kb, static_cast<const __nv_bfloat16*>(v), chunk_sum, group_sum, chunk_idx, chunk_score, group_idx,
                             group_score, static_cast<__nv_bfloat16*>(out), lse, err, append,
-                            n_items};
-  return dispatch<__nv_bfloat16>(p, sh, tk, tv, a, s);
+                            n_items, kv};
+  return dispatch_kv<__nv_bfloat16>(p, sh, tk, tv, a, s);
 }
 
 }  // namespace hga

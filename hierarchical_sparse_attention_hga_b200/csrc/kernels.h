@@ -114,15 +114,24 @@ cudaError_t launch_route_decode(const LayerParams& p, int dtype, bool level1, bo
 
 // One decode step (optional summary append + routing + attention): one launch of
 // decode_step_kernel when decode_item_path (kc <= 64, kg <= 128 and the shared
-// memory fits), else the append, routing and attention kernels; applies when
-// decode_step_path (bf16, D = 128 decode, device-resident K/V).
-bool decode_item_path(const LayerParams& p);
+// memory fits, with n_pt block-table entries staged per item for a paged pool),
+// else the append, routing and attention kernels; applies when
+// decode_step_path (bf16, D = 128 decode, device-resident K/V).  With
+// kv.block_table, k and v are page pools and only the one launch is taken.
+bool decode_item_path(const LayerParams& p, int n_pt = 0);
 bool decode_step_path(const LayerParams& p, int dtype);
 cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* q,
                                const int64_t* pos, float* chunk_sum, float* group_sum,
                                const void* k, const void* v, int32_t* chunk_idx,
                                float* chunk_score, int32_t* group_idx, float* group_score,
-                               void* out, float* lse, int append, unsigned* err, cudaStream_t s);
+                               void* out, float* lse, int append, unsigned* err, cudaStream_t s,
+                               const KvPages& kv = KvPages{nullptr, 0, 0, 0});
+
+// Summaries of paged pools: every group and chunk row that ends before
+// seq_len[b], per sequence (summaries.cu).
+cudaError_t launch_summaries_paged(const LayerParams& p, int dtype, const void* k_pages,
+                                   const KvPages& kv, const int64_t* seq_len, float* chunk_sum,
+                                   float* group_sum, unsigned* err, cudaStream_t s);
 
 // The summary rows each sequence's token pos[b] closes (one warp per (sequence,
 // KV head) item; the rows hga_build_summaries(pos, pos + 1) writes, per sequence).

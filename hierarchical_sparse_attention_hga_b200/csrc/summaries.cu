@@ -29,19 +29,38 @@ namespace {
 using summ::PairLoad;
 using summ::kGroup;
 
-template <typename T, int D, bool PRELOAD>
+// Paged pools (PAGED): sequence b's rows past seq_len[b] are never read (their
+// pages need not exist), and a group whose block-table entry is not a page of
+// the pool is skipped and flagged, with the chunk row it belongs to.
+template <typename T, int D, bool PRELOAD, bool PAGED>
 __global__ void __launch_bounds__(256)
 summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_t t_end,
                  int c_first, int c_count, float* __restrict__ chunk_sum,
-                 float* __restrict__ group_sum) {
+                 float* __restrict__ group_sum, KvPages kv, const int64_t* __restrict__ seq_len,
+                 unsigned* err) {
   constexpr int P = D / 2;
   constexpr int PPL = P / 32;
   extern __shared__ float2 smem_tab[];
   __shared__ float s_gsum[8][D];             // raw group sums of one chunk
+  __shared__ int s_missing[2];               // a group of the chunk had no page (by iteration parity)
   const int n_lo = P - p.n_high;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  const T* kb = k + static_cast<size_t>(bh) * p.n_alloc * D;
+  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  if (PAGED) {  // this sequence's rows end at seq_len[b]
+    const int64_t len = seq_len[b];
+    t_end = min(t_end, max(static_cast<int64_t>(0), len));
+  }
+  // key row g0 of a group (its rows follow contiguously), or null
+  auto group_rows = [&](int64_t g0) -> const T* {
+    if (!PAGED) return k + (static_cast<size_t>(bh) * p.n_alloc + g0) * D;
+    const int32_t pg = __ldg(kv.block_table + static_cast<size_t>(b) * kv.max_pages + g0 / kv.page_size);
+    if (pg < 0 || pg >= kv.n_pages) {
+      if (lane == 0) flag_error(err, kErrPage);
+      return nullptr;
+    }
+    return k + static_cast<size_t>(paged_row(kv, p.Hkv, h, pg, g0)) * D;
+  };
   // With PRELOAD (each CTA finishes one chunk: a decode append), the chunk's key
   // rows are loaded before the tables are built (k is never written by this
   // library), so their latency overlaps the table setup.
@@ -55,22 +74,30 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   }
   if (pre) {
     const int64_t g0 = static_cast<int64_t>(c_first + blockIdx.x) * p.C + static_cast<int64_t>(warp) * kGroup;
+    const T* grp = group_rows(g0);
+    pre = grp != nullptr;
+    if (pre) {
 #pragma unroll
-    for (int o = 0; o < kGroup; ++o) {
-      const T* row = kb + (g0 + o) * D + lane * PPL;
-      PairLoad<T, PPL>::run(row, x0[o]);
-      PairLoad<T, PPL>::run(row + P, y0[o]);
+      for (int o = 0; o < kGroup; ++o) {
+        const T* row = grp + o * D + lane * PPL;
+        PairLoad<T, PPL>::run(row, x0[o]);
+        PairLoad<T, PPL>::run(row + P, y0[o]);
+      }
     }
   }
   float2* tab_g = smem_tab;                  // [g][n_lo]: rotation by (g-1)/2 - o
   float2* tab_s = smem_tab + kGroup * n_lo;  // [Ng][n_lo]: rotation by (C-g)/2 - w*g
   for (int idx = threadIdx.x; idx < summ::table_entries(p, D); idx += blockDim.x)
     smem_tab[idx] = summ::table_entry(p, D, idx);
+  if (threadIdx.x == 0) s_missing[0] = s_missing[1] = 0;
   __syncthreads();
   pdl_wait();
 
-  for (int ci = blockIdx.x; ci < c_count; ci += gridDim.x) {
+  for (int ci = blockIdx.x, it = 0; ci < c_count; ci += gridDim.x, ++it) {
     const int c = c_first + ci;
+    // the other flag was last read before the previous iteration's final barrier
+    // and is next written after this iteration's
+    if (threadIdx.x == 0) s_missing[(it + 1) & 1] = 0;
     const int64_t c0 = static_cast<int64_t>(c) * p.C;
     const bool fin_c = c0 + p.C - 1 >= t_begin && c0 + p.C - 1 < t_end;
     // warp w: group w of the chunk
@@ -80,7 +107,8 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
       if (fin_c || fin_g) {
         float gx[PPL], gy[PPL];
         float x[kGroup][PPL], y[kGroup][PPL];
-        if (PRELOAD && ci == static_cast<int>(blockIdx.x)) {
+        bool have = true;
+        if (PRELOAD && pre && ci == static_cast<int>(blockIdx.x)) {
 #pragma unroll
           for (int o = 0; o < kGroup; ++o)
 #pragma unroll
@@ -89,13 +117,20 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
               y[o][u] = y0[o][u];
             }
         } else {
+          const T* grp = group_rows(g0);
+          have = grp != nullptr;
+          if (have) {
 #pragma unroll
-          for (int o = 0; o < kGroup; ++o) {
-            const T* row = kb + (g0 + o) * D + lane * PPL;
-            PairLoad<T, PPL>::run(row, x[o]);
-            PairLoad<T, PPL>::run(row + P, y[o]);
+            for (int o = 0; o < kGroup; ++o) {
+              const T* row = grp + o * D + lane * PPL;
+              PairLoad<T, PPL>::run(row, x[o]);
+              PairLoad<T, PPL>::run(row + P, y[o]);
+            }
+          } else if (lane == 0) {
+            s_missing[it & 1] = 1;
           }
         }
+        if (have) {
         summ::group_raw_sum<PPL>(x, y, tab_g, p.n_high, n_lo, lane, gx, gy);
         if (fin_g) {
           float* dst = group_sum + ((static_cast<size_t>(bh) * p.n_chunks + c) * p.Ng + warp) * D;
@@ -110,16 +145,19 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
           s_gsum[warp][lane * PPL + u] = gx[u];
           s_gsum[warp][P + lane * PPL + u] = gy[u];
         }
+        }
       }
     }
     if (fin_c) {  // uniform over the CTA
       __syncthreads();
       const float inv_c = 1.0f / p.C;
       float* dst = chunk_sum + (static_cast<size_t>(bh) * p.n_chunks + c) * D;
-      for (int i = threadIdx.x; i < P; i += blockDim.x) {
-        const float2 sc = summ::chunk_pair<D>(s_gsum, tab_s, p.Ng, p.n_high, n_lo, i);
-        dst[i] = __fmul_rn(sc.x, inv_c);
-        dst[P + i] = __fmul_rn(sc.y, inv_c);
+      if (!s_missing[it & 1]) {
+        for (int i = threadIdx.x; i < P; i += blockDim.x) {
+          const float2 sc = summ::chunk_pair<D>(s_gsum, tab_s, p.Ng, p.n_high, n_lo, i);
+          dst[i] = __fmul_rn(sc.x, inv_c);
+          dst[P + i] = __fmul_rn(sc.y, inv_c);
+        }
       }
     }
     __syncthreads();
@@ -127,9 +165,10 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   pdl_trigger();
 }
 
-template <typename T, int D>
+template <typename T, int D, bool PAGED>
 cudaError_t launch_summaries_t(const LayerParams& p, const void* k, int64_t t_begin, int64_t t_end,
-                               float* chunk_sum, float* group_sum, cudaStream_t stream) {
+                               float* chunk_sum, float* group_sum, const KvPages& kv,
+                               const int64_t* seq_len, unsigned* err, cudaStream_t stream) {
   // First group end at or after t_begin: nothing to do if it is past t_end.
   const int64_t first_g_end = (t_begin / p.g) * p.g + p.g - 1;
   if (t_end <= t_begin || first_g_end >= t_end) return cudaSuccess;
@@ -144,12 +183,12 @@ cudaError_t launch_summaries_t(const LayerParams& p, const void* k, int64_t t_be
   const int n_lo = D / 2 - p.n_high;
   const size_t smem = static_cast<size_t>(kGroup + p.Ng) * n_lo * sizeof(float2);
   if (c_count <= gx)  // one chunk per CTA
-    return launch_pdl(summaries_kernel<T, D, true>, grid, dim3(32 * p.Ng), smem, stream, 1,
+    return launch_pdl(summaries_kernel<T, D, true, PAGED>, grid, dim3(32 * p.Ng), smem, stream, 1,
                       static_cast<const T*>(k), p, t_begin, t_end, c_first, c_count, chunk_sum,
-                      group_sum);
-  return launch_pdl(summaries_kernel<T, D, false>, grid, dim3(32 * p.Ng), smem, stream, 1,
+                      group_sum, kv, seq_len, err);
+  return launch_pdl(summaries_kernel<T, D, false, PAGED>, grid, dim3(32 * p.Ng), smem, stream, 1,
                     static_cast<const T*>(k), p, t_begin, t_end, c_first, c_count, chunk_sum,
-                    group_sum);
+                    group_sum, kv, seq_len, err);
 }
 
 // Summary append of a decode step with per-sequence positions: one warp per
@@ -166,8 +205,9 @@ append_kernel(const T* __restrict__ k, const int64_t* __restrict__ pos, LayerPar
   pdl_wait();
   const int item = blockIdx.x;
   const int64_t pb = pos[item / p.Hkv];
+  const T* kb = k + static_cast<size_t>(item) * p.n_alloc * D;
   if (pb >= 0 && pb < p.n_alloc)
-    summ::append_closed_rows<T, D>(k + static_cast<size_t>(item) * p.n_alloc * D,
+    summ::append_closed_rows<T, D>([&](int64_t g0) { return kb + g0 * D; },
                                    chunk_sum + static_cast<size_t>(item) * p.n_chunks * D,
                                    group_sum + static_cast<size_t>(item) * p.n_chunks * p.Ng * D,
                                    p, pb, smem_tab, s_gsum);
@@ -196,13 +236,36 @@ cudaError_t launch_append_per_sequence(const LayerParams& p, int dtype, const vo
 
 cudaError_t launch_summaries(const LayerParams& p, int dtype, const void* k, int64_t t_begin,
                              int64_t t_end, float* chunk_sum, float* group_sum, cudaStream_t s) {
+  const KvPages dense{nullptr, 0, 0, 0};
   if (dtype == 0) {
-    return p.D == 64 ? launch_summaries_t<float, 64>(p, k, t_begin, t_end, chunk_sum, group_sum, s)
-                     : launch_summaries_t<float, 128>(p, k, t_begin, t_end, chunk_sum, group_sum, s);
+    return p.D == 64 ? launch_summaries_t<float, 64, false>(p, k, t_begin, t_end, chunk_sum,
+                                                           group_sum, dense, nullptr, nullptr, s)
+                     : launch_summaries_t<float, 128, false>(p, k, t_begin, t_end, chunk_sum,
+                                                            group_sum, dense, nullptr, nullptr, s);
   }
-  return p.D == 64
-             ? launch_summaries_t<__nv_bfloat16, 64>(p, k, t_begin, t_end, chunk_sum, group_sum, s)
-             : launch_summaries_t<__nv_bfloat16, 128>(p, k, t_begin, t_end, chunk_sum, group_sum, s);
+  return p.D == 64 ? launch_summaries_t<__nv_bfloat16, 64, false>(p, k, t_begin, t_end, chunk_sum,
+                                                                 group_sum, dense, nullptr,
+                                                                 nullptr, s)
+                   : launch_summaries_t<__nv_bfloat16, 128, false>(p, k, t_begin, t_end, chunk_sum,
+                                                                  group_sum, dense, nullptr,
+                                                                  nullptr, s);
+}
+
+cudaError_t launch_summaries_paged(const LayerParams& p, int dtype, const void* k_pages,
+                                   const KvPages& kv, const int64_t* seq_len, float* chunk_sum,
+                                   float* group_sum, unsigned* err, cudaStream_t s) {
+  if (dtype == 0) {
+    return p.D == 64 ? launch_summaries_t<float, 64, true>(p, k_pages, 0, p.n_alloc, chunk_sum,
+                                                          group_sum, kv, seq_len, err, s)
+                     : launch_summaries_t<float, 128, true>(p, k_pages, 0, p.n_alloc, chunk_sum,
+                                                           group_sum, kv, seq_len, err, s);
+  }
+  return p.D == 64 ? launch_summaries_t<__nv_bfloat16, 64, true>(p, k_pages, 0, p.n_alloc,
+                                                                chunk_sum, group_sum, kv, seq_len,
+                                                                err, s)
+                   : launch_summaries_t<__nv_bfloat16, 128, true>(p, k_pages, 0, p.n_alloc,
+                                                                 chunk_sum, group_sum, kv, seq_len,
+                                                                 err, s);
 }
 
 }  // namespace hga

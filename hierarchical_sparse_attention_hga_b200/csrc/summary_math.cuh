@@ -114,15 +114,17 @@ template <> struct PairLoad<__nv_bfloat16, 1> {
 // The summary rows of one (sequence, KV head) item whose last token is pb: the
 // group that pb ends, and the chunk when pb ends it too (a chunk row needs the
 // raw sums of all its groups, recomputed here from the cache).  One warp;
-// kb is the item's key rows, chunk_sum / group_sum its tables, tab the full
-// rotation table, gsum [Ng][D] scratch.  Nothing is written unless pb ends a
-// group.
-template <typename T, int D>
-__device__ void append_closed_rows(const T* kb, float* chunk_sum, float* group_sum,
+// group_rows(t0) gives the item's key row t0 of a group start t0 (the group's
+// rows follow it contiguously), or null when that group is not available;
+// chunk_sum / group_sum are the item's tables, tab the full rotation table,
+// gsum [Ng][D] scratch.  Nothing is written unless pb ends a group; false
+// (and nothing written) when a group the rows need is not available.
+template <typename T, int D, typename GroupRows>
+__device__ bool append_closed_rows(GroupRows group_rows, float* chunk_sum, float* group_sum,
                                    const LayerParams& p, int64_t pb, const float2* tab,
                                    float (*gsum)[D]) {
   constexpr int P = D / 2, PPL = P / 32;
-  if ((pb + 1) % kGroup != 0) return;
+  if ((pb + 1) % kGroup != 0) return true;
   const int lane = threadIdx.x & 31;
   const int n_lo = P - p.n_high;
   const int c = static_cast<int>(pb / p.C);
@@ -130,10 +132,12 @@ __device__ void append_closed_rows(const T* kb, float* chunk_sum, float* group_s
   const int w_close = static_cast<int>(pb % p.C) / kGroup;
   for (int w = closes_chunk ? 0 : w_close; w <= w_close; ++w) {
     const int64_t g0 = static_cast<int64_t>(c) * p.C + static_cast<int64_t>(w) * kGroup;
+    const T* grp = group_rows(g0);
+    if (grp == nullptr) return false;
     float x[kGroup][PPL], y[kGroup][PPL];
 #pragma unroll
     for (int o = 0; o < kGroup; ++o) {
-      const T* row = kb + (g0 + o) * D + lane * PPL;
+      const T* row = grp + o * D + lane * PPL;
       PairLoad<T, PPL>::run(row, x[o]);
       PairLoad<T, PPL>::run(row + P, y[o]);
     }
@@ -164,6 +168,7 @@ __device__ void append_closed_rows(const T* kb, float* chunk_sum, float* group_s
     }
   }
   __syncwarp();
+  return true;
 }
 
 }  // namespace summ

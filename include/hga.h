@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define HGA_ABI_VERSION 3
+#define HGA_ABI_VERSION 4
 
 typedef enum hga_status {
   HGA_OK = 0,
@@ -86,6 +86,22 @@ typedef struct hga_config {
   int32_t kv_loc;         /* hga_kv_loc of k and v (HGA_KV_DEVICE for the calls below) */
   double rope_theta;      /* RoPE base: omega_i = rope_theta^(-2i/D) */
 } hga_config;
+
+/*
+ * A paged K/V pool (hga_build_summaries_paged, hga_decode_step_paged), the
+ * block-table layout of serving engines: k and v are pools
+ * [n_pages, Hkv, page_size, D] (page-major, then KV head: one (page, head) is
+ * page_size contiguous rows), and token t of sequence b lives at row
+ * t % page_size of page block_table[b * max_pages + t / page_size].  Entries
+ * past a sequence's last token are never read (they may be -1).  Summary
+ * tables stay dense per sequence, with max_pages * page_size rows of capacity.
+ */
+typedef struct hga_kv_pages {
+  const int32_t* block_table; /* device int32 [B, max_pages] */
+  int64_t n_pages;            /* pages in each of the k and v pools */
+  int32_t page_size;          /* tokens per page: a positive multiple of 16 */
+  int32_t max_pages;          /* block-table entries per sequence */
+} hga_kv_pages;
 
 /* Version of this ABI (HGA_ABI_VERSION of the built library). */
 int32_t hga_abi_version(void);
@@ -394,6 +410,38 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q, const int64_t* 
  * hga_decode_step does not take.
  */
 hga_status hga_decode_step_launches(const hga_config* cfg, int64_t n_alloc, int32_t* launches);
+
+/*
+ * Ragged serving batch over a paged pool: hga_build_summaries for every
+ * sequence b over its own tokens [0, seq_len[b]) (device int64 [B]), reading
+ * k_pages through kv->block_table.  chunk_sum / group_sum are dense per
+ * sequence, [B, Hkv, n_alloc / C, D] and [B, Hkv, n_alloc / C, C / g, D] with
+ * n_alloc = kv->max_pages * kv->page_size (a multiple of C).  A block-table
+ * entry the build needs that is not a page of the pool ([0, n_pages)) skips
+ * its group (and chunk) and sets the device error word
+ * (HGA_ERR_DEVICE_CHECK from hga_device_status).
+ */
+hga_status hga_build_summaries_paged(const hga_config* cfg, const void* k_pages,
+                                     const hga_kv_pages* kv, const int64_t* seq_len,
+                                     float* chunk_sum, float* group_sum, void* stream);
+
+/*
+ * hga_decode_step over a paged pool: the same outputs, bit for bit, as
+ * hga_decode_step on a dense cache holding the same rows (per-sequence
+ * positions pos[b] < n_alloc = kv->max_pages * kv->page_size; the summary
+ * append reads the closed group's rows through the block table).  One launch
+ * of the decode-step kernel, which stages each sequence's block-table row in
+ * shared memory; shapes it cannot take (hga_decode_step_launches would say 2,
+ * or the block-table row does not fit beside the kernel's buffers) return
+ * HGA_ERR_UNSUPPORTED.  An entry a step needs that is not a page of the pool
+ * sets the device error word; its tiles read as zeros (never outside the pool).
+ *   k_pages, v_pages  device bf16 pools [n_pages, Hkv, page_size, 128]
+ */
+hga_status hga_decode_step_paged(const hga_config* cfg, const void* q, const int64_t* pos,
+                                 float* chunk_sum, float* group_sum, const void* k_pages,
+                                 const void* v_pages, const hga_kv_pages* kv, int32_t* chunk_idx,
+                                 float* chunk_score, int32_t* group_idx, float* group_score,
+                                 void* out, float* lse, int32_t append, void* stream);
 
 /*
  * hga_attend for callers that cannot allocate device memory.  The paper has no

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     from hierarchical_sparse_attention_hga_b200 import binding as B
-    assert B.hga_abi_version() == 3
+    assert B.hga_abi_version() == 4
     assert B.hga_status_string(0) == "HGA_OK"
     assert B.hga_status_string(6) == "HGA_ERR_DEVICE_CHECK"
     assert B.hga_status_string(99) == "HGA_ERR_UNKNOWN"
@@ -168,3 +168,25 @@ def test_warm_tier_sizes_and_refusals(lib):
         with pytest.raises(B.HGAError) as e:
             fn()
         assert e.value.status == 1   # window modes are 0, 1 and 2
+
+
+def test_paged_pool_refusals(lib):
+    """Paged calls check the block-table description on the host: a page size that
+    is not a positive multiple of 16, a null table, non-positive sizes, a capacity
+    that is not whole chunks, a pool of 2^31 rows or more."""
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    layer = B.Layer(batch=2, heads_q=32, heads_kv=8, head_dim=128)
+    cases = [(B.kv_pages(16, 100, 8, 64), 1), (B.kv_pages(None, 100, 64, 64), 1),
+             (B.kv_pages(16, 0, 64, 64), 1), (B.kv_pages(16, 100, 64, 0), 1),
+             (B.kv_pages(16, 100, 48, 5), 2), (B.kv_pages(16, 1 << 24, 256, 64), 3)]
+    for kv, status in cases:
+        with pytest.raises(B.HGAError) as e:
+            B.hga_decode_step_paged(layer, 16, 16, 16, 16, 16, 16, kv, 16, 16, 16, stream=0)
+        assert e.value.status == status, (kv.page_size, kv.n_pages, kv.max_pages)
+        with pytest.raises(B.HGAError) as e:
+            B.hga_build_summaries_paged(layer, 16, kv, 16, 16, 16, stream=0)
+        assert e.value.status == status
+    with pytest.raises(B.HGAError) as e:   # null pointers after a valid description
+        B.hga_decode_step_paged(layer, None, 16, 16, 16, 16, 16, B.kv_pages(16, 100, 64, 64), 16,
+                                16, 16, stream=0)
+    assert e.value.status == 1

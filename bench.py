@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=0,
                     help="attention layers per decode step (0: 4, or 1 for the host tier)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    ap.add_argument("--sub", default=None,
+                    help="run one of the additional workloads alone (its record is printed)")
     ap.add_argument("--warm-slots", type=int, default=0,
                     help="warm-tier group slots per (sequence, KV head) (0: 4 x topk_groups)")
     ap.add_argument("--warm-steps", type=int, default=64,
@@ -104,40 +106,52 @@ def peaks():
 
 # ---------------------------------------------------------------- byte counts
 
-def step_bytes(wl: S.Workload) -> dict:
+def step_bytes(wl: S.Workload, positions=None) -> dict:
     """Algorithmic HBM bytes of one decode step per kernel (whole batch).
 
     route_chunks: the candidate chunk-summary rows (fp32) + the G query rows;
     route_groups: the groups of the kc selected chunks + query rows + chunk ids;
     attend: K and V rows of the T routed tokens + query rows + output (fp32);
     summaries: the closing chunk's and group's key rows + the rows written.
+    positions: each sequence's query position (default: the last row, context-1);
+    "tokens" is T of the first sequence.
     """
     e = 2 if wl.dtype == "bf16" else 4
     d, g = wl.head_dim, wl.gqa
-    p = wl.context - 1
-    cur = p // wl.chunk
-    n_cand = max(0, cur - wl.local - wl.sink)
-    kc = min(wl.topk_chunks, n_cand)
     ng = wl.chunk // wl.group
-    kg = min(wl.topk_groups, kc * ng)
-    forced = (min(wl.sink, max(0, cur - wl.local)) * wl.chunk + (p - max(0, cur - wl.local) * wl.chunk + 1))
-    t = forced + kg * wl.group
-    units = wl.batch * wl.heads_kv
     qrow = g * d * e
-    closes_chunk = (p + 1) % wl.chunk == 0
-    closes_group = (p + 1) % wl.group == 0
-    summ = 0
-    if closes_chunk:
-        summ = wl.chunk * d * e + (d + ng * d) * 4
-    elif closes_group:
-        summ = wl.group * d * e + d * 4
-    return dict(
-        summaries=units * summ,
-        route_chunks=units * (n_cand * d * 4 + qrow),
-        route_groups=units * (kc * ng * d * 4 + qrow + wl.topk_chunks * 4),
-        attend=units * (t * d * e * 2 + qrow + g * d * 4 + wl.topk_groups * 4),
-        tokens=t,
-    )
+    positions = [wl.context - 1] * wl.batch if positions is None else [int(x) for x in positions]
+    tot = dict(summaries=0, route_chunks=0, route_groups=0, attend=0)
+    first_t = None
+    for p in positions:
+        cur = p // wl.chunk
+        n_cand = max(0, cur - wl.local - wl.sink)
+        kc = min(wl.topk_chunks, n_cand)
+        kg = min(wl.topk_groups, kc * ng)
+        forced = (min(wl.sink, max(0, cur - wl.local)) * wl.chunk +
+                  (p - max(0, cur - wl.local) * wl.chunk + 1))
+        t = forced + kg * wl.group
+        first_t = t if first_t is None else first_t
+        summ = 0
+        if (p + 1) % wl.chunk == 0:
+            summ = wl.chunk * d * e + (d + ng * d) * 4
+        elif (p + 1) % wl.group == 0:
+            summ = wl.group * d * e + d * 4
+        tot["summaries"] += wl.heads_kv * summ
+        tot["route_chunks"] += wl.heads_kv * (n_cand * d * 4 + qrow)
+        tot["route_groups"] += wl.heads_kv * (kc * ng * d * 4 + qrow + wl.topk_chunks * 4)
+        tot["attend"] += wl.heads_kv * (t * d * e * 2 + qrow + g * d * 4 + wl.topk_groups * 4)
+    tot["tokens"] = first_t
+    return tot
+
+
+def decode_step_bytes(wl: S.Workload, positions=None) -> int:
+    """Bytes of the one-launch decode step: append + routing + attention, less the
+    query rows the routing and the attention would each read again."""
+    nb = step_bytes(wl, positions)
+    e = 2 if wl.dtype == "bf16" else 4
+    return (nb["summaries"] + nb["route_chunks"] + nb["route_groups"] + nb["attend"] -
+            2 * wl.batch * wl.heads_kv * wl.gqa * wl.head_dim * e)
 
 
 # ------------------------------------------------------------------ clocks
@@ -469,8 +483,7 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
     # (the host enqueues them while the flush runs, so the events bracket GPU work)
     nb = step_bytes(wl)
     nb["route"] = nb["route_chunks"] + nb["route_groups"]
-    nb["decode_step"] = nb["summaries"] + nb["route"] + nb["attend"] - \
-        2 * bh * wl.gqa * wl.head_dim * (2 if wl.dtype == "bf16" else 4)
+    nb["decode_step"] = decode_step_bytes(wl)
     one_launch = not hot and B.hga_decode_step_launches(layer, n) == 1
     if one_launch:
         kern = "decode_step"
@@ -573,6 +586,179 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
         rec["host_link"] = host_link_report(wl, ms, dev)
         rec["warm_tier"] = warm_tier_report(args, wl, layer, L_[0], flush, stream)
     del L_, graphs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def ragged_positions(wl: S.Workload, seed: int) -> np.ndarray:
+    """A serving batch's mix of context lengths: each sequence's position drawn
+    log-uniform in [2048, context), seeded."""
+    rng = np.random.default_rng([seed, 77])
+    return np.exp(rng.uniform(np.log(2048), np.log(wl.context), wl.batch)).astype(np.int64)
+
+
+def make_pool(k, v, pos: np.ndarray, page: int, seed: int):
+    """Scatter each sequence's pages up to its position into a shuffled page pool
+    (the layout a serving engine's allocator leaves): pools [n_pages, Hkv, page,
+    D] and the block table [B, context/page], -1 past each sequence's last page."""
+    import torch
+    b_, h, n, d = k.shape
+    mp = n // page
+    need = pos // page + 1
+    total = int(need.sum())
+    perm = torch.randperm(total, generator=torch.Generator().manual_seed(seed))
+    bt = torch.full((b_, mp), -1, dtype=torch.int32)
+    kp = torch.empty(total, h, page, d, dtype=k.dtype, device=k.device)
+    vp = torch.empty_like(kp)
+    kb, vb = k.view(b_, h, mp, page, d), v.view(b_, h, mp, page, d)
+    at = 0
+    for b in range(b_):
+        m = int(need[b])
+        ids = perm[at:at + m]
+        at += m
+        bt[b, :m] = ids.to(torch.int32)
+        dst = ids.to(k.device)
+        kp[dst] = kb[b, :, :m].permute(1, 0, 2, 3)
+        vp[dst] = vb[b, :, :m].permute(1, 0, 2, 3)
+    return kp, vp, bt.to(k.device), total
+
+
+def paged_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, world: int, ranks,
+                 seed: int, pages=(16, 64, 256)) -> dict:
+    """A ragged serving batch over paged K/V: every sequence at its own position
+    (ragged_positions), the pages of every layer scattered through a shuffled
+    pool, the one-launch paged decode step of `layers` layers back to back (each
+    its own pool and tables) against the dense one-launch step on the same rows
+    and positions.  Same timing method as the decode records; the headline is
+    the first page size, the others are reported beside it; outputs of every
+    arm checked bit for bit against the dense step."""
+    import torch
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+
+    dev = torch.device("cuda")
+    n = wl.context
+    pos_np = ragged_positions(wl, seed)
+    pos = torch.as_tensor(pos_np, device=dev)
+    layer = make_layer(B, wl, B.HGA_F32)
+    bh = wl.batch * wl.heads_kv
+    nc, ng = n // wl.chunk, wl.chunk // wl.group
+    flush = Flush(dev)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def tables():
+        return dict(cs=torch.zeros(bh, nc, wl.head_dim, device=dev),
+                    gs=torch.zeros(bh, nc, ng, wl.head_dim, device=dev),
+                    ci=torch.empty(bh, wl.topk_chunks, dtype=torch.int32, device=dev),
+                    gi=torch.empty(bh, wl.topk_groups, dtype=torch.int32, device=dev),
+                    out=torch.empty(wl.batch, wl.heads_q, 1, wl.head_dim, device=dev),
+                    lse=torch.empty(wl.batch, wl.heads_q, 1, device=dev))
+
+    L_ = []
+    for li in range(layers):
+        q, k, v, _ = device_inputs(wl, seed + li, dev)
+        d = dict(q=q, k=k, v=v, dense=tables())
+        B.hga_build_summaries(layer, k, n, 0, n, d["dense"]["cs"], d["dense"]["gs"], stream=sh)
+        L_.append(d)
+
+    def run(d, page, st):
+        t = d[page]
+        if page == "dense":
+            B.hga_decode_step(layer, d["q"], pos, t["cs"], t["gs"], n, d["k"], d["v"], t["ci"],
+                              t["gi"], t["out"], t["lse"], append=True, stream=st)
+        else:
+            B.hga_decode_step_paged(layer, d["q"], pos, t["cs"], t["gs"], t["kp"], t["vp"],
+                                    t["kv"], t["ci"], t["gi"], t["out"], t["lse"], append=True,
+                                    stream=st)
+
+    def graph_of(page):
+        for _ in range(max(1, warmup)):
+            for d in L_:
+                run(d, page, sh)
+        torch.cuda.synchronize()
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_):
+            cs_ = torch.cuda.current_stream().cuda_stream
+            for d in L_:
+                run(d, page, cs_)
+        torch.cuda.synchronize()
+        assert B.hga_device_status(sh) == 0
+        return g_
+
+    g_dense = graph_of("dense")
+    ms_dense = timed_graph(g_dense, steps, flush, stream)
+    del g_dense
+    hbm, peak_kind = peaks()
+    arms = {}
+    for i, page in enumerate(pages):
+        for li, d in enumerate(L_):
+            kp, vp, bt, n_pages = make_pool(d["k"], d["v"], pos_np, page, seed + li)
+            t = dict(tables(), kp=kp, vp=vp, bt=bt, kv=B.kv_pages(bt, n_pages, page, n // page))
+            B.hga_build_summaries_paged(layer, kp, t["kv"], pos, t["cs"], t["gs"], stream=sh)
+            d[page] = t
+        g_ = graph_of(page)
+        for d in L_:   # same routing and the same output bits as the dense step
+            assert torch.equal(d["dense"]["gi"], d[page]["gi"])
+            assert torch.equal(d["dense"]["out"].view(torch.int32), d[page]["out"].view(torch.int32))
+        for _ in range(warmup):
+            flush()
+            g_.replay()
+        ranks.barrier()
+        torch.cuda.synchronize()
+        if i == 0:
+            with ClockSampler(torch.cuda.current_device()) as clk:
+                ms = timed_graph(g_, steps, flush, stream)
+        else:
+            ms = timed_graph(g_, steps, flush, stream)
+        ranks.barrier()
+        ms = ranks.max(ms)
+        # roofline: events around the layers' direct launches, queued behind the flush
+        n_side = min(steps, 100)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_side)]
+        for a_, b_ in ev:
+            flush()
+            a_.record(stream)
+            for d in L_:
+                run(d, page, sh)
+            b_.record(stream)
+        torch.cuda.synchronize()
+        assert B.hga_device_status(sh) == 0
+        kern_ms = ranks.max(sum(a_.elapsed_time(b_) for a_, b_ in ev) / n_side / layers)
+        nbytes = decode_step_bytes(wl, pos_np) + bh * (n // page) * 4   # + the block-table rows
+        arms[page] = dict(ms=ms, kern_ms=kern_ms, nbytes=nbytes)
+        del g_
+        for d in L_:
+            del d[page]
+        torch.cuda.empty_cache()
+
+    head = arms[pages[0]]
+    achieved = head["nbytes"] / (head["kern_ms"] * 1e-3) / 1e9
+    per_layer = head["ms"] / layers
+    unit = "decode tokens/s (one attention layer)"
+    rec = {
+        "value": job_rate(wl.batch, world, per_layer), "unit": unit, "ms_per_step": head["ms"],
+        "attn_us_per_layer": per_layer * 1e3, "dense_us_per_layer": ms_dense / layers * 1e3,
+        "page_sizes_us_per_layer": {str(pg): a["ms"] / layers * 1e3 for pg, a in arms.items()},
+        "layers_per_step": layers,
+        "data": "synthetic (N(0,1) q/k/v drawn on the device; pages shuffled through the pool)",
+        "config": {"workload": "paged_ragged_decode", "batch_per_gpu": wl.batch,
+                   "capacity": n, "page_size": pages[0], "positions": {
+                       "min": int(pos_np.min()), "median": int(np.median(pos_np)),
+                       "max": int(pos_np.max()), "recipe": "log-uniform in [2048, capacity)"},
+                   "heads_q": wl.heads_q, "heads_kv": wl.heads_kv, "head_dim": wl.head_dim,
+                   "topk_chunks": wl.topk_chunks, "topk_groups": wl.topk_groups,
+                   "l2": L2_NOTE},
+        "roofline": {"kernel": "decode_step_kernel (paged)", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "algorithmic_bytes": head["nbytes"],
+                     "kernel_us": head["kern_ms"] * 1e3},
+        "gpu_launches": layers * steps,
+        "parity": "every arm's routed ids and outputs equal the dense step's bit for bit (checked here)",
+        "clocks": clk.report(),
+    }
+    del L_
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return rec
@@ -1025,6 +1211,7 @@ SUB_WORKLOADS = (
     ("host_tier_decode_128k_b8", S.workload("host_tier_decode_128k"), 1),
     ("llama3_8b_decode_32k_b4", S.workload("llama3_8b_decode_32k", batch=4, needles=0), 4),
     ("llama3_8b_decode_32k_b1", S.workload("llama3_8b_decode_32k", batch=1, needles=0), 4),
+    ("paged_ragged_decode_32k_b16", S.workload("llama3_8b_decode_32k", needles=0), 4),
 )
 
 
@@ -1048,6 +1235,20 @@ def main():
     B.load_library()
     dev = torch.device("cuda")
     ranks = Ranks(world, dev)
+    if args.sub:
+        name, swl, layers = next(t for t in SUB_WORKLOADS if t[0] == args.sub)
+        seed = rank_seed(swl.name, rank)
+        if swl.prefill:
+            r = prefill_record(args, swl, args.steps, args.warmup, world, ranks, seed)
+        elif name.startswith("paged"):
+            r = paged_record(args, swl, layers, args.steps, args.warmup, world, ranks, seed)
+        else:
+            r = decode_record(args, swl, layers, args.steps, args.warmup, world, ranks, seed,
+                              compare=False)
+        if rank == 0:
+            print(json.dumps({"workload": name, "n_gpus": world, "steps": args.steps,
+                              "warmup": args.warmup, **r}))
+        return
     wl = workload_of(args)
     seed = rank_seed(args.workload, rank)
     x = S.make_inputs(wl, seed)
@@ -1073,11 +1274,13 @@ def main():
             sseed = rank_seed(swl.name, 0) + 17 * (i + 1)
             if swl.prefill:
                 r = prefill_record(args, swl, sub_steps, args.warmup, world, ranks, sseed)
+            elif name.startswith("paged"):
+                r = paged_record(args, swl, layers, sub_steps, args.warmup, world, ranks, sseed)
             else:
                 r = decode_record(args, swl, layers, sub_steps, args.warmup, world, ranks, sseed,
                                   compare=False)
             r["steps"] = sub_steps
-            if not args.no_cpu_baseline:
+            if not args.no_cpu_baseline and not name.startswith("paged"):
                 r["cpu_baseline"] = cpu_baseline(swl, sseed, 3.0, r["unit"])
             subs[name] = r
         line["workloads"] = subs

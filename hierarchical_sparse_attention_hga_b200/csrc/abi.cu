@@ -415,9 +415,13 @@ static hga_status paged_params(const hga_config* cfg, const hga_kv_pages* kv, La
   const int64_t n_alloc = static_cast<int64_t>(kv->max_pages) * kv->page_size;
   hga_status st = make_params(cfg, n_alloc, 1, p);
   if (st != HGA_OK) return st;
-  if (kv->n_pages * p->Hkv * kv->page_size >= (static_cast<int64_t>(1) << 31))
-    return fail(HGA_ERR_UNSUPPORTED, "the pool has 2^31 rows or more");
-  *out = KvPages{kv->block_table, kv->page_size, kv->max_pages, kv->n_pages};
+  if (kv->n_pages * p->Hkv * kv->page_size >= (static_cast<int64_t>(1) << 31) ||
+      n_alloc >= (static_cast<int64_t>(1) << 31))
+    return fail(HGA_ERR_UNSUPPORTED, "the pool, or a sequence's capacity, has 2^31 rows or more");
+  int shift = -1;
+  for (int s = 0; s < 31; ++s)
+    if ((1 << s) == kv->page_size) shift = s;
+  *out = KvPages{kv->block_table, kv->page_size, kv->max_pages, kv->n_pages, shift};
   return HGA_OK;
 }
 

@@ -39,15 +39,23 @@ struct LayerParams {
 struct KvPages {
   const int32_t* block_table;
   int page_size;
-  int max_pages;   // entries per sequence; n_alloc = max_pages * page_size
+  int max_pages;   // entries per sequence; n_alloc = max_pages * page_size < 2^31
   int64_t n_pages;
+  int page_shift;  // log2(page_size) when it is a power of two, else -1
 };
+
+// Block-table index of token t (t < 2^31).
+__host__ __device__ __forceinline__ uint32_t page_index(const KvPages& kv, uint32_t t) {
+  return kv.page_shift >= 0 ? t >> kv.page_shift : t / static_cast<uint32_t>(kv.page_size);
+}
 
 // Row of token t of (b, h) in the [rows][D] view of a paged pool, given its
 // page (validated by the caller).
 __host__ __device__ __forceinline__ int64_t paged_row(const KvPages& kv, int Hkv, int h,
                                                      int32_t page, int64_t t) {
-  return (static_cast<int64_t>(page) * Hkv + h) * kv.page_size + t % kv.page_size;
+  const uint32_t tt = static_cast<uint32_t>(t);
+  return (static_cast<int64_t>(page) * Hkv + h) * kv.page_size +
+         (tt - page_index(kv, tt) * static_cast<uint32_t>(kv.page_size));
 }
 
 // Test hook of the one-launch decode step: warp 0 skips its first group-summary

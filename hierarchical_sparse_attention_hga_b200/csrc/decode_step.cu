@@ -232,7 +232,9 @@ struct StepSmem {  // byte offsets into the dynamic shared memory (after alignme
   __host__ __device__ size_t o_glist() const { return o_chunks() + kKcMax * 4; }    // int [kKgMax]
   __host__ __device__ size_t o_gsum() const { return o_glist() + kKgMax * 4; }      // float [8][kD]
   __host__ __device__ size_t o_tab() const { return o_gsum() + 8 * kD * 4; }        // float2 [n_tab]
-  __host__ __device__ size_t o_pages() const { return o_tab() + static_cast<size_t>(n_tab) * 8; }  // int [n_pt]
+  __host__ __device__ size_t o_pages() const {  // int [n_pt], 16-byte aligned
+    return (o_tab() + static_cast<size_t>(n_tab) * 8 + 15) & ~static_cast<size_t>(15);
+  }
   __host__ __device__ size_t bytes() const { return 1024 + o_pages() + static_cast<size_t>(n_pt) * 4; }
 };
 
@@ -336,7 +338,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
         auto group_rows = [&](int64_t g0) -> const __nv_bfloat16* {
           if (!PAGED) return a.k + (static_cast<size_t>(item) * p.n_alloc + g0) * kD;
           const int32_t pg = __ldg(a.kv.block_table + static_cast<size_t>(b) * a.kv.max_pages +
-                                   g0 / a.kv.page_size);
+                                   page_index(a.kv, static_cast<uint32_t>(g0)));
           if (pg < 0 || pg >= a.kv.n_pages) return nullptr;
           return a.k + static_cast<size_t>(paged_row(a.kv, p.Hkv, h, pg, g0)) * kD;
         };
@@ -386,12 +388,18 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int64_t row_base = static_cast<int64_t>(item) * p.n_alloc;
     if (PAGED) {  // the sequence's block-table row, landing while the scan runs
       const int32_t* bt = a.kv.block_table + static_cast<size_t>(b) * a.kv.max_pages;
-      for (int i = tid; i < a.kv.max_pages; i += W * 32) ptx::cp_async4(s_pages + i, bt + i);
+      if (a.kv.max_pages % 4 == 0 && (reinterpret_cast<uintptr_t>(a.kv.block_table) & 15) == 0) {
+        for (int i = 4 * tid; i < a.kv.max_pages; i += 4 * W * 32) ptx::cp_async16(s_pages + i, bt + i);
+      } else {
+        for (int i = tid; i < a.kv.max_pages; i += W * 32) ptx::cp_async4(s_pages + i, bt + i);
+      }
     }
     // row of token t of this item in the [rows][D] view of k / v
     auto kv_row = [&](int64_t t) -> int32_t {
       if (!PAGED) return static_cast<int32_t>(row_base + t);
-      return static_cast<int32_t>(paged_row(a.kv, p.Hkv, h, s_pages[t / a.kv.page_size], t));
+      const uint32_t tt = static_cast<uint32_t>(t);
+      const uint32_t j = page_index(a.kv, tt);
+      return (s_pages[j] * p.Hkv + h) * a.kv.page_size + static_cast<int32_t>(tt - j * a.kv.page_size);
     };
 
     // 1. position, routing query and Q fragments: independent loads, issued first so
@@ -544,13 +552,16 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (PAGED) {  // this thread's block-table copies: landed; the entries the item reads, checked
       ptx::cp_async_wait_all();
       const int last = ok ? static_cast<int>(pb / a.kv.page_size) : -1;
-      for (int i = tid; i <= last; i += W * 32) {
-        const int pg = s_pages[i];
-        if (pg < 0 || pg >= a.kv.n_pages) {
-          flag_error(a.err, kErrPage);
-          s_pages[i] = -1;
+      const bool wide = a.kv.max_pages % 4 == 0 && (reinterpret_cast<uintptr_t>(a.kv.block_table) & 15) == 0;
+      const int step = wide ? 4 : 1;  // entries per copy of this thread
+      for (int i0 = step * tid; i0 <= last; i0 += step * W * 32)
+        for (int i = i0; i < i0 + step && i <= last; ++i) {
+          const int pg = s_pages[i];
+          if (pg < 0 || pg >= a.kv.n_pages) {
+            flag_error(a.err, kErrPage);
+            s_pages[i] = -1;
+          }
         }
-      }
     }
     named_sync(kBarStream, W * 32);  // B1
 

@@ -125,7 +125,7 @@ cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* 
                                const void* k, const void* v, int32_t* chunk_idx,
                                float* chunk_score, int32_t* group_idx, float* group_score,
                                void* out, float* lse, int append, unsigned* err, cudaStream_t s,
-                               const KvPages& kv = KvPages{nullptr, 0, 0, 0});
+                               const KvPages& kv = KvPages{nullptr, 0, 0, 0, -1});
 
 // Summaries of paged pools: every group and chunk row that ends before
 // seq_len[b], per sequence (summaries.cu).

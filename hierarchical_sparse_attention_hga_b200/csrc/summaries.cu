@@ -54,7 +54,7 @@ summaries_kernel(const T* __restrict__ k, LayerParams p, int64_t t_begin, int64_
   // key row g0 of a group (its rows follow contiguously), or null
   auto group_rows = [&](int64_t g0) -> const T* {
     if (!PAGED) return k + (static_cast<size_t>(bh) * p.n_alloc + g0) * D;
-    const int32_t pg = __ldg(kv.block_table + static_cast<size_t>(b) * kv.max_pages + g0 / kv.page_size);
+    const int32_t pg = __ldg(kv.block_table + static_cast<size_t>(b) * kv.max_pages + page_index(kv, static_cast<uint32_t>(g0)));
     if (pg < 0 || pg >= kv.n_pages) {
       if (lane == 0) flag_error(err, kErrPage);
       return nullptr;
@@ -236,7 +236,7 @@ cudaError_t launch_append_per_sequence(const LayerParams& p, int dtype, const vo
 
 cudaError_t launch_summaries(const LayerParams& p, int dtype, const void* k, int64_t t_begin,
                              int64_t t_end, float* chunk_sum, float* group_sum, cudaStream_t s) {
-  const KvPages dense{nullptr, 0, 0, 0};
+  const KvPages dense{nullptr, 0, 0, 0, -1};
   if (dtype == 0) {
     return p.D == 64 ? launch_summaries_t<float, 64, false>(p, k, t_begin, t_end, chunk_sum,
                                                            group_sum, dense, nullptr, nullptr, s)

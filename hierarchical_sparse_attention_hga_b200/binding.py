@@ -28,7 +28,7 @@ SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device
            "hga_route", "hga_hot_rows", "hga_gather_host", "hga_attend", "hga_decode_step",
            "hga_decode_step_launches", "hga_attend_noalloc", "hga_warm_rows", "hga_warm_reset",
            "hga_gather_warm", "hga_attend_warm", "hga_build_summaries_paged",
-           "hga_decode_step_paged")
+           "hga_decode_step_paged", "hga_attend_backward_workspace_size", "hga_attend_backward")
 
 
 class HGAConfig(ctypes.Structure):
@@ -96,6 +96,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_build_summaries_paged": (ctypes.c_int, [C, P, KV, P, P, P, P]),
         "hga_decode_step_paged": (ctypes.c_int, [C, P, P, P, P, P, P, KV, P, P, P, P, P, P, I32,
                                                  P]),
+        "hga_attend_backward_workspace_size": (ctypes.c_int, [C, I64, I32, ctypes.POINTER(SZ)]),
+        "hga_attend_backward": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, P, P, P, P,
+                                               SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -313,6 +316,25 @@ def hga_decode_step_paged(cfg, q, pos, chunk_sum, group_sum, k_pages, v_pages, k
                                                 _ptr(group_score), _ptr(out), _ptr(lse),
                                                 1 if append else 0, _stream(stream)),
            "hga_decode_step_paged")
+
+
+def hga_attend_backward_workspace_size(cfg, n_alloc: int, q_len: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().hga_attend_backward_workspace_size(ctypes.byref(_cfg(cfg)), n_alloc,
+                                                             q_len, ctypes.byref(out)),
+           "hga_attend_backward_workspace_size")
+    return out.value
+
+
+def hga_attend_backward(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, out, lse, d_out,
+                        dq, dk, dv, workspace, workspace_bytes: int, stream=None) -> None:
+    """dQ, dK, dV of a prefill attention over its routed index sets."""
+    _check(load_library().hga_attend_backward(ctypes.byref(_cfg(cfg)), _ptr(q), q_len, _ptr(pos),
+                                              _ptr(k), _ptr(v), n_alloc, _ptr(group_idx),
+                                              _ptr(out), _ptr(lse), _ptr(d_out), _ptr(dq),
+                                              _ptr(dk), _ptr(dv), _ptr(workspace),
+                                              workspace_bytes, _stream(stream)),
+           "hga_attend_backward")
 
 
 def hga_debug_inject(flags: int) -> int:

@@ -470,4 +470,42 @@ hga_status hga_decode_step_paged(const hga_config* cfg, const void* q, const int
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_decode_step_paged");
 }
 
+hga_status hga_attend_backward_workspace_size(const hga_config* cfg, int64_t n_alloc,
+                                              int32_t q_len, size_t* bytes) {
+  if (!bytes) return fail(HGA_ERR_INVALID_ARG, "bytes is NULL");
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, q_len, &p);
+  if (st != HGA_OK) return st;
+  if (!backward_path(p, cfg->dtype))
+    return fail(HGA_ERR_UNSUPPORTED,
+                "the backward pass is built for bf16, head_dim 128, group 16 prefill of whole "
+                "chunks, G <= 16, topk_groups <= 128");
+  *bytes = backward_workspace_bytes(p);
+  return HGA_OK;
+}
+
+hga_status hga_attend_backward(const hga_config* cfg, const void* q, int32_t q_len,
+                               const int64_t* pos, const void* k, const void* v, int64_t n_alloc,
+                               const int32_t* group_idx, const void* out, const float* lse,
+                               const void* d_out, float* dq, float* dk, float* dv,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  Range nvtx_range("hga_attend_backward");
+  size_t need = 0;
+  hga_status st = hga_attend_backward_workspace_size(cfg, n_alloc, q_len, &need);
+  if (st != HGA_OK) return st;
+  if (!q || !pos || !k || !v || !group_idx || !out || !lse || !d_out || !dq || !dk || !dv)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (!workspace || workspace_bytes < need)
+    return fail(HGA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                workspace_bytes);
+  LayerParams p;
+  make_params(cfg, n_alloc, q_len, &p);
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_attend_backward(p, q, k, v, out, cfg->out_dtype == HGA_F32 ? 1 : 0, lse,
+                                         d_out, pos, group_idx, dq, dk, dv, workspace, err,
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attend_backward");
+}
+
 }  // extern "C"

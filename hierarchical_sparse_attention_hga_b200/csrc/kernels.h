@@ -127,6 +127,16 @@ cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* 
                                void* out, float* lse, int append, unsigned* err, cudaStream_t s,
                                const KvPages& kv = KvPages{nullptr, 0, 0, 0, -1});
 
+// Backward pass of the prefill attention over the routed index sets
+// (attend_backward.cu): bf16, D = 128, group 16, whole aligned query chunks.
+bool backward_path(const LayerParams& p, int dtype);
+size_t backward_workspace_bytes(const LayerParams& p);
+cudaError_t launch_attend_backward(const LayerParams& p, const void* q, const void* k,
+                                   const void* v, const void* out, int out_f32, const float* lse,
+                                   const void* d_out, const int64_t* pos, const int32_t* group_idx,
+                                   float* dq, float* dk, float* dv, void* workspace,
+                                   unsigned* err, cudaStream_t s);
+
 // Summaries of paged pools: every group and chunk row that ends before
 // seq_len[b], per sequence (summaries.cu).
 cudaError_t launch_summaries_paged(const LayerParams& p, int dtype, const void* k_pages,

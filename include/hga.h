@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define HGA_ABI_VERSION 4
+#define HGA_ABI_VERSION 5
 
 typedef enum hga_status {
   HGA_OK = 0,
@@ -410,6 +410,39 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q, const int64_t* 
  * hga_decode_step does not take.
  */
 hga_status hga_decode_step_launches(const hga_config* cfg, int64_t n_alloc, int32_t* launches);
+
+/*
+ * Backward pass of a prefill call of hga_attend (HGA technical summary,
+ * "Risultati Sperimentali": the method is trained and fine-tuned end to end;
+ * "Metodologia -> Meccanismo Core", item 4: the output is an exact softmax
+ * attention over the selected tokens).  The routing is a selection, so no
+ * gradient flows through it or through the summaries: with the forward's token
+ * sets held fixed (forced chunks, the block's own chunk causally, and the kept
+ * groups of group_idx), for P = exp(S - lse), S = Q K^T / sqrt(D) and
+ * Delta = rowsum(dO * O):
+ *   dV = P^T dO,  dS = P * (dO V^T - Delta),  dQ = dS K / sqrt(D),
+ *   dK = dS^T Q / sqrt(D),
+ * accumulated over the G query heads of each KV head and every query row.
+ *   q, d_out   device bf16 [B, Hq, q_len, 128]; q_len whole aligned chunks
+ *              ending at pos[b] (as the forward)
+ *   k, v       device bf16 [B, Hkv, n_alloc, 128]
+ *   group_idx  the forward's routing, device int32 [B, Hkv, q_len / C, kg]
+ *   out, lse   the forward's output (cfg->out_dtype) and natural-log LSE
+ *   dq         device float32 [B, Hq, q_len, 128] (written)
+ *   dk, dv     device float32 [B, Hkv, n_alloc, 128] (every row written; rows
+ *              no query sees are zero)
+ *   workspace  device scratch of hga_attend_backward_workspace_size() bytes
+ * The sums run in a fixed order (no atomics): the result does not depend on
+ * scheduling.  Built for bf16, head_dim 128, group 16, G <= 16,
+ * topk_groups <= 128.
+ */
+hga_status hga_attend_backward_workspace_size(const hga_config* cfg, int64_t n_alloc,
+                                              int32_t q_len, size_t* bytes);
+hga_status hga_attend_backward(const hga_config* cfg, const void* q, int32_t q_len,
+                               const int64_t* pos, const void* k, const void* v, int64_t n_alloc,
+                               const int32_t* group_idx, const void* out, const float* lse,
+                               const void* d_out, float* dq, float* dk, float* dv,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Ragged serving batch over a paged pool: hga_build_summaries for every

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     from hierarchical_sparse_attention_hga_b200 import binding as B
-    assert B.hga_abi_version() == 4
+    assert B.hga_abi_version() == 5
     assert B.hga_status_string(0) == "HGA_OK"
     assert B.hga_status_string(6) == "HGA_ERR_DEVICE_CHECK"
     assert B.hga_status_string(99) == "HGA_ERR_UNKNOWN"
@@ -190,3 +190,27 @@ def test_paged_pool_refusals(lib):
         B.hga_decode_step_paged(layer, None, 16, 16, 16, 16, 16, B.kv_pages(16, 100, 64, 64), 16,
                                 16, 16, stream=0)
     assert e.value.status == 1
+
+
+def test_backward_workspace_and_refusals(lib):
+    """The backward pass sizes its workspace on the host and refuses decode shapes,
+    fp32 K/V, null pointers and a short workspace before any CUDA call."""
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+    layer = B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128)
+    small = B.hga_attend_backward_workspace_size(layer, 8192, 8192)
+    big = B.hga_attend_backward_workspace_size(layer, 65536, 65536)
+    assert 0 < small < big
+    for args, status in (((layer, 8192, 1), 3),
+                         ((B.Layer(batch=1, heads_q=32, heads_kv=8, head_dim=128, dtype=B.HGA_F32),
+                           8192, 8192), 3)):
+        with pytest.raises(B.HGAError) as e:
+            B.hga_attend_backward_workspace_size(*args)
+        assert e.value.status == status
+    with pytest.raises(B.HGAError) as e:
+        B.hga_attend_backward(layer, None, 8192, 16, 16, 16, 8192, 16, 16, 16, 16, 16, 16, 16, 16,
+                              small, stream=0)
+    assert e.value.status == 1
+    with pytest.raises(B.HGAError) as e:
+        B.hga_attend_backward(layer, 16, 8192, 16, 16, 16, 8192, 16, 16, 16, 16, 16, 16, 16, 16,
+                              small - 1, stream=0)
+    assert e.value.status == 7

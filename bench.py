@@ -764,6 +764,102 @@ def paged_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wor
     return rec
 
 
+def training_record(args, wl: S.Workload, steps: int, warmup: int, world: int, ranks,
+                    seed: int) -> dict:
+    """One training step of one attention layer at the prefill shape: the forward
+    (summaries, routing of every 64-query block, attention) and the backward over
+    the forward's index sets (hga_attend_backward: dQ, dK, dV) for a synthetic
+    upstream gradient.  Same timing method as the prefill record."""
+    import torch
+    from hierarchical_sparse_attention_hga_b200 import binding as B
+
+    dev = torch.device("cuda")
+    n = wl.context
+    nblk = n // wl.chunk
+    q, k, v, pos = device_inputs(wl, seed, dev)
+    layer = make_layer(B, wl, B.HGA_BF16)
+    bh = wl.batch * wl.heads_kv
+    cs = torch.empty(bh, n // wl.chunk, wl.head_dim, device=dev)
+    gs = torch.empty(bh, n // wl.chunk, wl.chunk // wl.group, wl.head_dim, device=dev)
+    ci = torch.empty(bh, nblk, wl.topk_chunks, dtype=torch.int32, device=dev)
+    gi = torch.empty(bh, nblk, wl.topk_groups, dtype=torch.int32, device=dev)
+    out = torch.empty(wl.batch, wl.heads_q, n, wl.head_dim, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(wl.batch, wl.heads_q, n, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed + 1)
+    dout = torch.randn(out.shape, generator=gen, device=dev).to(torch.bfloat16)
+    dq = torch.empty(out.shape, device=dev)
+    dk = torch.empty(k.shape, device=dev)
+    dv = torch.empty(v.shape, device=dev)
+    bwb = B.hga_attend_backward_workspace_size(layer, n, n)
+    bws = torch.empty(bwb, dtype=torch.uint8, device=dev)
+    flush = Flush(dev)
+    parts = {
+        "forward": lambda: (B.hga_build_summaries(layer, k, n, 0, n, cs, gs),
+                            B.hga_route(layer, q, n, pos, cs, gs, n, ci, gi),
+                            B.hga_attend(layer, q, n, pos, k, v, n, gi, out, lse)),
+        "backward": lambda: B.hga_attend_backward(layer, q, n, pos, k, v, n, gi, out, lse, dout,
+                                                  dq, dk, dv, bws, bwb),
+    }
+
+    def step():
+        for fn in parts.values():
+            fn()
+
+    for _ in range(max(1, warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert B.hga_device_status() == 0
+    graphs = {}
+    for name, fn in list(parts.items()) + [("step", step)]:
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_):
+            fn()
+        graphs[name] = g_
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms_step = timed_graph(graphs["step"], steps, flush, stream)
+    ranks.barrier()
+    ms_step = ranks.max(ms_step)
+    ms = {name: timed_graph(graphs[name], max(3, min(steps, 20)), flush, stream) for name in parts}
+    assert B.hga_device_status() == 0
+    assert bool(torch.isfinite(dq).all()) and bool(torch.isfinite(dk).all())
+    # algorithmic flops per visible (query row, key) pair: forward 4D (S, PV);
+    # backward 14D (dQ pass: S, dP, dS K; dK/dV pass: S, dP, P^T dO, dS^T Q)
+    fwd_flops = prefill_flops(wl)
+    bwd_flops = fwd_flops * 14 / 4
+    peak, peak_kind = tensor_peak()
+    achieved = bwd_flops / (ms["backward"] * 1e-3) / 1e12
+    tokens = wl.batch * n
+    rec = {
+        "value": job_rate(tokens, world, ms_step),
+        "unit": "training tokens/s (one attention layer, forward + backward)",
+        "ms_per_step": ms_step, "forward_ms": ms["forward"], "backward_ms": ms["backward"],
+        "layers_per_step": 1,
+        "dtype": "bf16 q/k/v/dO, fp32 accumulation and gradients",
+        "data": "synthetic (N(0,1) q/k/v and upstream gradient drawn on the device)",
+        "config": {"workload": wl.name + " (training step)", "batch_per_gpu": wl.batch,
+                   "context": n, "heads_q": wl.heads_q, "heads_kv": wl.heads_kv,
+                   "head_dim": wl.head_dim, "chunk": wl.chunk, "topk_chunks": wl.topk_chunks,
+                   "topk_groups": wl.topk_groups, "l2": L2_NOTE},
+        "roofline": {"kernel": "hga_attend_backward (dq_kernel + dkdv_kernel + helpers)",
+                     "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "algorithmic_flops": bwd_flops,
+                     "kernel_us": ms["backward"] * 1e3,
+                     "note": "mma.sync m16n8k16 kernels; timed as the whole backward call"},
+        "gpu_launches": steps * (3 + 5),
+        "clocks": clk.report(),
+    }
+    del q, k, v, dq, dk, dv, bws, graphs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
 def host_link_report(wl: S.Workload, ms: dict, dev) -> dict:
     """Host-tier traffic over the host link per step, against a pinned H2D copy probe."""
     import torch
@@ -1212,6 +1308,7 @@ SUB_WORKLOADS = (
     ("llama3_8b_decode_32k_b4", S.workload("llama3_8b_decode_32k", batch=4, needles=0), 4),
     ("llama3_8b_decode_32k_b1", S.workload("llama3_8b_decode_32k", batch=1, needles=0), 4),
     ("paged_ragged_decode_32k_b16", S.workload("llama3_8b_decode_32k", needles=0), 4),
+    ("training_step_64k", S.workload("llama3_8b_prefill_64k"), 1),
 )
 
 
@@ -1237,8 +1334,14 @@ def main():
     ranks = Ranks(world, dev)
     if args.sub:
         name, swl, layers = next(t for t in SUB_WORKLOADS if t[0] == args.sub)
+        if args.batch:
+            swl = swl.with_(batch=args.batch)
+        if args.context:
+            swl = swl.with_(context=args.context)
         seed = rank_seed(swl.name, rank)
-        if swl.prefill:
+        if name.startswith("training"):
+            r = training_record(args, swl, args.steps, args.warmup, world, ranks, seed)
+        elif swl.prefill:
             r = prefill_record(args, swl, args.steps, args.warmup, world, ranks, seed)
         elif name.startswith("paged"):
             r = paged_record(args, swl, layers, args.steps, args.warmup, world, ranks, seed)
@@ -1272,7 +1375,9 @@ def main():
         sub_steps = max(3, min(args.steps, 20))
         for i, (name, swl, layers) in enumerate(SUB_WORKLOADS):
             sseed = rank_seed(swl.name, 0) + 17 * (i + 1)
-            if swl.prefill:
+            if name.startswith("training"):
+                r = training_record(args, swl, sub_steps, args.warmup, world, ranks, sseed)
+            elif swl.prefill:
                 r = prefill_record(args, swl, sub_steps, args.warmup, world, ranks, sseed)
             elif name.startswith("paged"):
                 r = paged_record(args, swl, layers, sub_steps, args.warmup, world, ranks, sseed)
@@ -1280,7 +1385,7 @@ def main():
                 r = decode_record(args, swl, layers, sub_steps, args.warmup, world, ranks, sseed,
                                   compare=False)
             r["steps"] = sub_steps
-            if not args.no_cpu_baseline and not name.startswith("paged"):
+            if not args.no_cpu_baseline and not name.startswith(("paged", "training")):
                 r["cpu_baseline"] = cpu_baseline(swl, sseed, 3.0, r["unit"])
             subs[name] = r
         line["workloads"] = subs

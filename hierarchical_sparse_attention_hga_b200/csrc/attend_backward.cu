@@ -145,31 +145,41 @@ __device__ __forceinline__ void load_a_rows(const __nv_bfloat16* r0, const __nv_
   }
 }
 
-// acc[2][4] += A (registers, rows g / g+8) x B^T, B = the 16 rows of tile `bt`
-// (rows are the n index): S = A B^T over the 128 columns.
-__device__ __forceinline__ void mma_rows_t(float (&acc)[2][4], const uint32_t (&a)[8][4],
-                                           uint32_t bt) {
+// s[2][4] += A x K^T and dp[2][4] += A2 x V^T with A, A2 in registers (rows g,
+// g + 8) and K, V the 16 rows of tiles kt, vt (rows are the n index), the four
+// accumulator chains interleaved.
+__device__ __forceinline__ void mma_rows_t2(float (&s)[2][4], float (&dp)[2][4],
+                                            const uint32_t (&a)[8][4], const uint32_t (&a2)[8][4],
+                                            uint32_t kt, uint32_t vt) {
   const int lane = threadIdx.x & 31, mi = lane >> 3, ri = lane & 7;
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    uint32_t r[4];
-    ptx::ldmatrix_x4(swz(bt, (mi >> 1) * 8 + ri, kk * 2 + (mi & 1)), r);
-    ptx::mma_bf16_16816(acc[0], a[kk], r[0], r[1]);
-    ptx::mma_bf16_16816(acc[1], a[kk], r[2], r[3]);
+    uint32_t rk[4], rv[4];
+    ptx::ldmatrix_x4(swz(kt, (mi >> 1) * 8 + ri, kk * 2 + (mi & 1)), rk);
+    ptx::ldmatrix_x4(swz(vt, (mi >> 1) * 8 + ri, kk * 2 + (mi & 1)), rv);
+    ptx::mma_bf16_16816_pure(s[0], a[kk], rk[0], rk[1]);
+    ptx::mma_bf16_16816_pure(s[1], a[kk], rk[2], rk[3]);
+    ptx::mma_bf16_16816_pure(dp[0], a2[kk], rv[0], rv[1]);
+    ptx::mma_bf16_16816_pure(dp[1], a2[kk], rv[2], rv[3]);
   }
 }
 
-// acc[2][4] += A x B^T with A = the 16 rows of tile `at` (rows are the m index)
-// and B = the 16 rows of tile `bt`.
-__device__ __forceinline__ void mma_tiles_t(float (&acc)[2][4], uint32_t at, uint32_t bt) {
+// st[2][4] += K Q^T and dpt[2][4] += V dO^T, with K, V (rows the m index) and Q,
+// dO (rows the n index) 16-row tiles; the four chains interleaved.
+__device__ __forceinline__ void mma_tiles_t2(float (&st)[2][4], float (&dpt)[2][4], uint32_t kt,
+                                             uint32_t qt, uint32_t vt, uint32_t dt) {
   const int lane = threadIdx.x & 31, mi = lane >> 3, ri = lane & 7;
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    uint32_t ra[4], rb[4];
-    ptx::ldmatrix_x4(swz(at, (mi & 1) * 8 + ri, kk * 2 + (mi >> 1)), ra);
-    ptx::ldmatrix_x4(swz(bt, (mi >> 1) * 8 + ri, kk * 2 + (mi & 1)), rb);
-    ptx::mma_bf16_16816(acc[0], ra, rb[0], rb[1]);
-    ptx::mma_bf16_16816(acc[1], ra, rb[2], rb[3]);
+    uint32_t ka[4], qb[4], va[4], db[4];
+    ptx::ldmatrix_x4(swz(kt, (mi & 1) * 8 + ri, kk * 2 + (mi >> 1)), ka);
+    ptx::ldmatrix_x4(swz(qt, (mi >> 1) * 8 + ri, kk * 2 + (mi & 1)), qb);
+    ptx::ldmatrix_x4(swz(vt, (mi & 1) * 8 + ri, kk * 2 + (mi >> 1)), va);
+    ptx::ldmatrix_x4(swz(dt, (mi >> 1) * 8 + ri, kk * 2 + (mi & 1)), db);
+    ptx::mma_bf16_16816_pure(st[0], ka, qb[0], qb[1]);
+    ptx::mma_bf16_16816_pure(st[1], ka, qb[2], qb[3]);
+    ptx::mma_bf16_16816_pure(dpt[0], va, db[0], db[1]);
+    ptx::mma_bf16_16816_pure(dpt[1], va, db[2], db[3]);
   }
 }
 
@@ -182,8 +192,8 @@ __device__ __forceinline__ void mma_into_rows(float (&acc)[16][4], const uint32_
   for (int nn = 0; nn < 8; ++nn) {
     uint32_t r[4];
     ptx::ldmatrix_x4_trans(swz(bt, (mi & 1) * 8 + ri, nn * 2 + (mi >> 1)), r);
-    ptx::mma_bf16_16816(acc[2 * nn], a, r[0], r[1]);
-    ptx::mma_bf16_16816(acc[2 * nn + 1], a, r[2], r[3]);
+    ptx::mma_bf16_16816_pure(acc[2 * nn], a, r[0], r[1]);
+    ptx::mma_bf16_16816_pure(acc[2 * nn + 1], a, r[2], r[3]);
   }
 }
 
@@ -422,8 +432,7 @@ __global__ void __launch_bounds__(kDqWarps * 32) dq_kernel(BwdArgs a, LayerParam
       const uint32_t kt = ptx::smem_u32(dsm + (u & 1) * 2 * kTile);
       const uint32_t vt = kt + kTile;
       float s[2][4] = {}, dp[2][4] = {};
-      mma_rows_t(s, qa, kt);
-      mma_rows_t(dp, da, vt);
+      mma_rows_t2(s, dp, qa, da, kt, vt);
       const bool causal = tk0 + 15 > tq0;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -556,8 +565,7 @@ __global__ void __launch_bounds__(kKvWarps * 32) dkdv_kernel(BwdArgs a, LayerPar
     const uint32_t qt = kt + 2 * kTile + stage * 2 * kTile, dt = qt + kTile;
     const float* ld = reinterpret_cast<const float*>(wsm + 6 * kTile) + stage * 32;
     float st[2][4] = {}, dpt[2][4] = {};
-    mma_tiles_t(st, kt, qt);   // S^T: keys x queries
-    mma_tiles_t(dpt, vt, dt);  // dP^T
+    mma_tiles_t2(st, dpt, kt, qt, vt, dt);  // S^T (keys x queries) and dP^T
     const int64_t tq0 = static_cast<int64_t>(jq) * p.C + r0;
     const bool causal = jq == c && tq0 < tk0 + 15;
     float pt[2][4];

@@ -58,6 +58,9 @@ def parse():
                     help="run one of the additional workloads alone (its record is printed)")
     ap.add_argument("--warm-slots", type=int, default=0,
                     help="warm-tier group slots per (sequence, KV head) (0: 4 x topk_groups)")
+    ap.add_argument("--cold-dir", default=None,
+                    help="directory of the cold tier's history file (default: the system's "
+                         "temporary directory)")
     ap.add_argument("--warm-steps", type=int, default=64,
                     help="consecutive decode steps of the warm-tier runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -976,12 +979,82 @@ def warm_tier_report(args, wl: S.Workload, layer, d: dict, flush, stream) -> dic
                                                     "cold": (hits + misses) * group_bytes / T},
                      "step_us": {"warm": w_step, "cold": c_step},
                      "gather_us": {"warm": w_gather, "cold": c_gather}})
-    return {"slots_per_kv_head": M, "steps": T,
+    # the cold tier: the same steps with the history in a file, read per step by
+    # host threads (plan on the GPU, stage on the host, fill on the GPU)
+    qs = queries(0.95)
+    cold = {}
+    try:
+        cold = cold_tier_run(args, B, wl, layer, d, qs, pos_all, M, tags, stamps, smap, kw, vw,
+                             counters, group_bytes, sh)
+    except (B.HGAError, OSError) as e:   # e.g. no room for the history file
+        cold = {"unavailable": str(e)}
+    return {"slots_per_kv_head": M, "steps": T, "cold_tier": cold,
             "hbm_bytes": 2 * bh * rows * wl.head_dim * 2 + 2 * tags.numel() * 4,
             "timing": ("CUDA events around each of T direct-launch steps (summary append, route, "
                        "gather, attention) on the launch stream, L2 flushed before each; one "
                        "untimed step fills the windows first"),
             "runs": runs}
+
+
+def cold_tier_run(args, B, wl, layer, d, qs, pos_all, M, tags, stamps, smap, kw, vw, counters,
+                  group_bytes, sh) -> dict:
+    """The warm-tier steps with the history in a file (the cold tier): plan on the
+    GPU, stage the misses and the newest window row from the file with host
+    threads, fill and attend on the GPU."""
+    import tempfile
+    import torch
+    n, T = wl.context, args.warm_steps
+    bh = wl.batch * wl.heads_kv
+    dev = d["q"].device
+    rho = 0.95
+    plan = torch.empty(bh, wl.topk_groups, 2, dtype=torch.int32, device=dev)
+    n_plan = torch.empty(bh, dtype=torch.int32, device=dev)
+    plan_h = torch.empty(plan.shape, dtype=torch.int32).pin_memory()
+    n_plan_h = torch.empty(n_plan.shape, dtype=torch.int32).pin_memory()
+    staging = torch.zeros(B.hga_cold_stage_bytes(layer), dtype=torch.uint8).pin_memory()
+    with tempfile.TemporaryDirectory(dir=args.cold_dir) as tmp:
+        with B.ColdStore(os.path.join(tmp, "kv.bin"), layer, n, create=True) as store:
+            store.write(d["k_host"], d["v_host"], 0, n, threads=16)
+            B.hga_warm_reset(layer, M, tags, stamps, stream=sh)
+            counters.zero_()
+            step_ms, stage_ms, groups = [], [], 0
+            for t in range(T + 1):
+                pos = pos_all[t]
+                p = n - T - 1 + t
+                mode = 1 if t == 0 else 2
+                torch.cuda.synchronize()
+                t0 = time.perf_counter()
+                B.hga_build_summaries(layer, d["k_host"], n, p, p + 1, d["cs"], d["gs"], stream=sh)
+                B.hga_route(layer, qs[t], 1, pos, d["cs"], d["gs"], n, d["ci"], d["gi"], stream=sh)
+                B.hga_warm_plan(layer, n, pos, d["gi"], M, tags, stamps, smap, plan, n_plan,
+                                counters=counters, stream=sh)
+                plan_h.copy_(plan, non_blocking=True)
+                n_plan_h.copy_(n_plan, non_blocking=True)
+                torch.cuda.synchronize()
+                s0 = time.perf_counter()
+                store.stage(layer, np.full(wl.batch, p, dtype=np.int64), plan_h.numpy(),
+                            n_plan_h.numpy(), mode, staging, threads=16)
+                s1 = time.perf_counter()
+                B.hga_warm_fill(layer, n, pos, staging, plan, n_plan, M, mode, kw, vw, stream=sh)
+                B.hga_attend_warm(layer, qs[t], pos, kw, vw, n, d["gi"], smap, M, d["out"],
+                                  d["lse"], stream=sh)
+                torch.cuda.synchronize()
+                t1 = time.perf_counter()
+                if t:
+                    step_ms.append((t1 - t0) * 1e3)
+                    stage_ms.append((s1 - s0) * 1e3)
+                    groups += int(n_plan_h.sum())
+            assert B.hga_device_status(sh) == 0
+            hits, misses = (int(v) for v in counters.cpu())
+            read = groups * group_bytes + T * bh * d["k_host"].shape[-1] * 2 * 2
+            return {"rho": rho, "hit_rate": hits / max(1, hits + misses),
+                    "file_bytes_read_per_step": read / T,
+                    "step_ms": sum(step_ms) / T, "stage_ms": sum(stage_ms) / T,
+                    "stage_gbs": read / (sum(stage_ms) * 1e-3) / 1e9,
+                    "timing": ("host wall clock around each step (the plan's device-to-host "
+                               "copy and the file reads make the step synchronous), 16 host "
+                               "threads; the file was just written, so the page cache may "
+                               "serve the reads")}
 
 
 # ------------------------------------------------------------------ prefill

@@ -28,7 +28,9 @@ SYMBOLS = ("hga_abi_version", "hga_status_string", "hga_last_error", "hga_device
            "hga_route", "hga_hot_rows", "hga_gather_host", "hga_attend", "hga_decode_step",
            "hga_decode_step_launches", "hga_attend_noalloc", "hga_warm_rows", "hga_warm_reset",
            "hga_gather_warm", "hga_attend_warm", "hga_build_summaries_paged",
-           "hga_decode_step_paged", "hga_attend_backward_workspace_size", "hga_attend_backward")
+           "hga_decode_step_paged", "hga_attend_backward_workspace_size", "hga_attend_backward",
+           "hga_cold_open", "hga_cold_close", "hga_cold_write", "hga_cold_stage_bytes",
+           "hga_warm_plan", "hga_cold_stage", "hga_warm_fill")
 
 
 class HGAConfig(ctypes.Structure):
@@ -99,6 +101,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "hga_attend_backward_workspace_size": (ctypes.c_int, [C, I64, I32, ctypes.POINTER(SZ)]),
         "hga_attend_backward": (ctypes.c_int, [C, P, I32, P, P, P, I64, P, P, P, P, P, P, P, P,
                                                SZ, P]),
+        "hga_cold_open": (ctypes.c_int, [ctypes.c_char_p, C, I64, I32, ctypes.POINTER(P)]),
+        "hga_cold_close": (ctypes.c_int, [P]),
+        "hga_cold_write": (ctypes.c_int, [P, P, P, I64, I64, I32]),
+        "hga_cold_stage_bytes": (ctypes.c_int, [C, ctypes.POINTER(SZ)]),
+        "hga_warm_plan": (ctypes.c_int, [C, I64, P, P, I32, P, P, P, P, P, P, P]),
+        "hga_cold_stage": (ctypes.c_int, [P, C, P, P, P, I32, P, I32]),
+        "hga_warm_fill": (ctypes.c_int, [C, I64, P, P, P, P, I32, I32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -118,7 +127,11 @@ def _ptr(x):
         return None
     if isinstance(x, int):
         return x
-    return x.data_ptr()
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if not x.flags["C_CONTIGUOUS"]:  # a numpy array (host-side calls)
+        raise ValueError("host arrays passed to the library must be C-contiguous")
+    return x.ctypes.data
 
 
 def _stream(stream):
@@ -335,6 +348,61 @@ def hga_attend_backward(cfg, q, q_len: int, pos, k, v, n_alloc: int, group_idx, 
                                               _ptr(dk), _ptr(dv), _ptr(workspace),
                                               workspace_bytes, _stream(stream)),
            "hga_attend_backward")
+
+
+class ColdStore:
+    """A file-backed K/V history (the cold tier); close() or use as a context manager."""
+
+    def __init__(self, path: str, cfg, n_alloc: int, create: bool = False):
+        self.handle = ctypes.c_void_p()
+        _check(load_library().hga_cold_open(str(path).encode(), ctypes.byref(_cfg(cfg)), n_alloc,
+                                            1 if create else 0, ctypes.byref(self.handle)),
+               "hga_cold_open")
+
+    def write(self, k, v, t0: int, t1: int, threads: int = 8) -> None:
+        _check(load_library().hga_cold_write(self.handle, _ptr(k), _ptr(v), t0, t1, threads),
+               "hga_cold_write")
+
+    def stage(self, cfg, pos, plan, n_plan, window_mode: int, staging, threads: int = 8) -> None:
+        _check(load_library().hga_cold_stage(self.handle, ctypes.byref(_cfg(cfg)), _ptr(pos),
+                                             _ptr(plan), _ptr(n_plan), window_mode, _ptr(staging),
+                                             threads), "hga_cold_stage")
+
+    def close(self) -> None:
+        if self.handle:
+            _check(load_library().hga_cold_close(self.handle), "hga_cold_close")
+            self.handle = ctypes.c_void_p()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+
+def hga_cold_stage_bytes(cfg) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().hga_cold_stage_bytes(ctypes.byref(_cfg(cfg)), ctypes.byref(out)),
+           "hga_cold_stage_bytes")
+    return out.value
+
+
+def hga_warm_plan(cfg, n_alloc: int, pos, group_idx, warm_groups: int, tags, stamps, slot_map,
+                  plan, n_plan, counters=None, stream=None) -> None:
+    """The warm tier's table update alone: misses as (group, slot) pairs for a cold store."""
+    _check(load_library().hga_warm_plan(ctypes.byref(_cfg(cfg)), n_alloc, _ptr(pos),
+                                        _ptr(group_idx), warm_groups, _ptr(tags), _ptr(stamps),
+                                        _ptr(slot_map), _ptr(plan), _ptr(n_plan), _ptr(counters),
+                                        _stream(stream)), "hga_warm_plan")
+
+
+def hga_warm_fill(cfg, n_alloc: int, pos, staging, plan, n_plan, warm_groups: int,
+                  window_mode: int, k_work, v_work, stream=None) -> None:
+    """Copies a cold store's staged rows into the warm working buffers."""
+    _check(load_library().hga_warm_fill(ctypes.byref(_cfg(cfg)), n_alloc, _ptr(pos),
+                                        _ptr(staging), _ptr(plan), _ptr(n_plan), warm_groups,
+                                        window_mode, _ptr(k_work), _ptr(v_work), _stream(stream)),
+           "hga_warm_fill")
 
 
 def hga_debug_inject(flags: int) -> int:

@@ -40,7 +40,7 @@ def _stale(target, deps):
 
 
 def _compile(src, verbose):
-    obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+    obj = os.path.join(OBJ, os.path.splitext(os.path.basename(src))[0] + ".o")
     if not _stale(obj, [src] + _headers()):
         return obj
     cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
@@ -62,7 +62,7 @@ def build(verbose: bool = False) -> str:
         objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
     if _stale(LIB, objs):
         tmp = LIB + ".tmp"
-        cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]
+        cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-pthread", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode:
             sys.stderr.write(r.stdout + r.stderr)

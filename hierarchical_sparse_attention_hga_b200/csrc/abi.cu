@@ -9,8 +9,11 @@
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
+#include <new>
+#include <string>
 
 #include "../../include/hga.h"
+#include "cold_tier.h"
 #include "kernels.h"
 
 namespace hga {
@@ -506,6 +509,126 @@ hga_status hga_attend_backward(const hga_config* cfg, const void* q, int32_t q_l
                                          d_out, pos, group_idx, dq, dk, dv, workspace, err,
                                          static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_attend_backward");
+}
+
+hga_status hga_warm_plan(const hga_config* cfg, int64_t n_alloc, const int64_t* pos,
+                         const int32_t* group_idx, int32_t warm_groups, int32_t* tags,
+                         int32_t* stamps, int32_t* slot_map, int32_t* plan, int32_t* n_plan,
+                         uint64_t* counters, void* stream) {
+  Range nvtx_range("hga_warm_plan");
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+  if ((st = check_warm(p, warm_groups)) != HGA_OK) return st;
+  if (!pos || !group_idx || !tags || !stamps || !slot_map || !plan || !n_plan)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_gather_warm(p, nullptr, nullptr, pos, group_idx, warm_groups, tags, stamps,
+                                     slot_map, nullptr, nullptr, 0,
+                                     reinterpret_cast<unsigned long long*>(counters), err,
+                                     static_cast<cudaStream_t>(stream),
+                                     reinterpret_cast<int2*>(plan), n_plan);
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_warm_plan");
+}
+
+hga_status hga_warm_fill(const hga_config* cfg, int64_t n_alloc, const int64_t* pos,
+                         const void* staging, const int32_t* plan, const int32_t* n_plan,
+                         int32_t warm_groups, int32_t window_mode, void* k_work, void* v_work,
+                         void* stream) {
+  Range nvtx_range("hga_warm_fill");
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+  if ((st = check_warm(p, warm_groups)) != HGA_OK) return st;
+  if (!pos || !staging || !plan || !n_plan || !k_work || !v_work)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (window_mode < 0 || window_mode > 2)
+    return fail(HGA_ERR_INVALID_ARG, "window_mode %d is not 0, 1 or 2", window_mode);
+  unsigned* err = nullptr;
+  if ((st = device_error_ptr(&err)) != HGA_OK) return st;
+  cudaError_t e = launch_warm_fill(p, staging, reinterpret_cast<const int2*>(plan), n_plan, pos,
+                                   warm_groups, window_mode, k_work, v_work, err,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "hga_warm_fill");
+}
+
+}  // extern "C"
+
+struct hga_cold_store {
+  hga::ColdStore s;
+  int32_t B, Hkv;
+};
+
+extern "C" {
+
+hga_status hga_cold_stage_bytes(const hga_config* cfg, size_t* bytes) {
+  if (!bytes) return fail(HGA_ERR_INVALID_ARG, "bytes is NULL");
+  LayerParams p;
+  hga_status st = make_params(cfg, cfg ? cfg->chunk : 0, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+  *bytes = static_cast<size_t>(p.B) * p.Hkv * cold_stage_unit_bytes(p);
+  return HGA_OK;
+}
+
+hga_status hga_cold_open(const char* path, const hga_config* cfg, int64_t n_alloc,
+                         int32_t create, hga_cold_store** store) {
+  if (!path || !store) return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  LayerParams p;
+  hga_status st = make_params(cfg, n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+  hga_cold_store* h = new (std::nothrow) hga_cold_store;
+  if (!h) return fail(HGA_ERR_INVALID_ARG, "out of host memory");
+  const std::string e = cold_open(path, static_cast<int64_t>(p.B) * p.Hkv, n_alloc, p.D * 2,
+                                  create != 0, &h->s);
+  if (!e.empty()) {
+    delete h;
+    return fail(HGA_ERR_INVALID_ARG, "hga_cold_open: %s", e.c_str());
+  }
+  h->B = p.B;
+  h->Hkv = p.Hkv;
+  *store = h;
+  return HGA_OK;
+}
+
+hga_status hga_cold_close(hga_cold_store* store) {
+  if (!store) return fail(HGA_ERR_INVALID_ARG, "store is NULL");
+  cold_close(&store->s);
+  delete store;
+  return HGA_OK;
+}
+
+hga_status hga_cold_write(hga_cold_store* store, const void* k, const void* v, int64_t t0,
+                          int64_t t1, int32_t threads) {
+  Range nvtx_range("hga_cold_write");
+  if (!store || !k || !v) return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  if (t0 < 0 || t1 < t0 || t1 > store->s.n_alloc)
+    return fail(HGA_ERR_INVALID_ARG, "need 0 <= t0 <= t1 <= n_alloc");
+  const std::string e = cold_write(store->s, k, v, t0, t1, threads);
+  return e.empty() ? HGA_OK : fail(HGA_ERR_INVALID_ARG, "hga_cold_write: %s", e.c_str());
+}
+
+hga_status hga_cold_stage(hga_cold_store* store, const hga_config* cfg, const int64_t* pos,
+                          const int32_t* plan, const int32_t* n_plan, int32_t window_mode,
+                          void* staging, int32_t threads) {
+  Range nvtx_range("hga_cold_stage");
+  if (!store || !pos || !plan || !n_plan || !staging)
+    return fail(HGA_ERR_INVALID_ARG, "null pointer");
+  LayerParams p;
+  hga_status st = make_params(cfg, store->s.n_alloc, 1, &p);
+  if (st != HGA_OK) return st;
+  if ((st = check_host_tier(cfg, p)) != HGA_OK) return st;
+  if (p.B != store->B || p.Hkv != store->Hkv)
+    return fail(HGA_ERR_SHAPE, "the store was opened for another batch or head count");
+  if (window_mode < 0 || window_mode > 2)
+    return fail(HGA_ERR_INVALID_ARG, "window_mode %d is not 0, 1 or 2", window_mode);
+  const std::string e = cold_stage(store->s, p, pos, reinterpret_cast<const int2*>(plan), n_plan,
+                                   window_mode, staging, threads);
+  return e.empty() ? HGA_OK : fail(HGA_ERR_INVALID_ARG, "hga_cold_stage: %s", e.c_str());
 }
 
 }  // extern "C"

@@ -175,7 +175,8 @@ gather_warm_kernel(const uint4* __restrict__ k_host, const uint4* __restrict__ v
                    LayerParams p, int M, int Mp, int32_t* __restrict__ tags,
                    int32_t* __restrict__ stamps, int32_t* __restrict__ slot_map, int refresh,
                    uint4* __restrict__ k_work, uint4* __restrict__ v_work,
-                   unsigned long long* __restrict__ counters, unsigned* err) {
+                   unsigned long long* __restrict__ counters, unsigned* err,
+                   int2* __restrict__ plan, int32_t* __restrict__ n_plan) {
   __shared__ unsigned long long s_key[kWarmMax];  // eviction order, then the miss list
   __shared__ short s_val[kWarmMax];               // slot of each key
   __shared__ int s_gid[1024], s_in[1024];         // kept groups, their group_idx positions
@@ -208,6 +209,7 @@ gather_warm_kernel(const uint4* __restrict__ k_host, const uint4* __restrict__ v
   int32_t* sm_row = slot_map + static_cast<size_t>(bh) * p.kg;
   if (!ok) {
     for (int j = tid; j < p.kg; j += kWarmThreads) sm_row[j] = -1;
+    if (plan && tid == 0) n_plan[bh] = 0;
     return;
   }
   const int n = s_n;
@@ -279,6 +281,16 @@ gather_warm_kernel(const uint4* __restrict__ k_host, const uint4* __restrict__ v
   }
   __syncthreads();
   for (int j = tid; j < p.kg; j += kWarmThreads) sm_row[j] = s_map[j];
+  if (plan) {  // decide only: the misses, for a cold store to stage
+    for (int r = tid; r < s_m; r += kWarmThreads) {
+      const unsigned long long mk = s_key[r];
+      plan[static_cast<size_t>(bh) * p.kg + r] =
+          make_int2(static_cast<int>(mk >> 32), static_cast<int>(mk & 0xffffffffu));
+    }
+    if (tid == 0) n_plan[bh] = s_m;
+    pdl_trigger();
+    return;
+  }
 
   const uint4* kh = k_host + static_cast<size_t>(bh) * p.n_alloc * kRowVec;
   const uint4* vh = v_host + static_cast<size_t>(bh) * p.n_alloc * kRowVec;
@@ -316,6 +328,56 @@ gather_warm_kernel(const uint4* __restrict__ k_host, const uint4* __restrict__ v
   pdl_trigger();
 }
 
+// Copies the rows a cold store staged for one warm step (see launch_warm_fill):
+// the missed groups into their slots, the window rows into the window.  One CTA
+// per (sequence, KV head), zero-copy 16-byte loads of the pinned staging.
+__global__ void __launch_bounds__(kWarmThreads)
+warm_fill_kernel(const uint4* __restrict__ staging, const int2* __restrict__ plan,
+                 const int32_t* __restrict__ n_plan, const int64_t* __restrict__ pos,
+                 LayerParams p, int M, int mode, uint4* __restrict__ k_work,
+                 uint4* __restrict__ v_work, unsigned* err) {
+  const int tid = threadIdx.x, bh = blockIdx.x, b = bh / p.Hkv;
+  const int64_t pb = pos[b];
+  const bool ok = valid_position(pb, p, tid == 0 ? err : nullptr);
+  pdl_wait();
+  if (!ok) return;
+  const int64_t WR = window_row_capacity(p);
+  const int64_t unit_vec = cold_stage_unit_bytes(p) / 16;
+  const uint4* sg = staging + static_cast<size_t>(bh) * unit_vec;   // [K|V][kg][16][16 vec]
+  const uint4* sw = sg + static_cast<size_t>(2) * p.kg * p.g * kRowVec;  // [K|V][WR][16 vec]
+  const int64_t R = hot_rows(p, M);
+  const int64_t W = static_cast<int64_t>(p.sink + p.local + 1) * p.C;
+  uint4* kw = k_work + static_cast<size_t>(bh) * R * kRowVec;
+  uint4* vw = v_work + static_cast<size_t>(bh) * R * kRowVec;
+  const int m = min(n_plan[bh], p.kg);
+  const int per = p.g * kRowVec;
+  const int64_t cur = pb / p.C, b0 = max(static_cast<int64_t>(0), cur - p.local);
+  const int64_t nw = window_row_count(p, pb, mode);
+  const int64_t total = static_cast<int64_t>(m) * per + nw * kRowVec;
+  for (int64_t e = tid; e < total; e += kWarmThreads) {
+    size_t src, dst;
+    if (e < static_cast<int64_t>(m) * per) {
+      const int r = static_cast<int>(e / per), w = static_cast<int>(e - static_cast<int64_t>(r) * per);
+      const int slot = plan[static_cast<size_t>(bh) * p.kg + r].y;
+      if (slot < 0 || slot >= M) continue;
+      src = static_cast<size_t>(r) * per + w;
+      dst = static_cast<size_t>(W + static_cast<int64_t>(slot) * p.g) * kRowVec + w;
+      kw[dst] = sg[src];
+      vw[dst] = sg[static_cast<size_t>(p.kg) * per + src];
+    } else {
+      const int64_t f = e - static_cast<int64_t>(m) * per;
+      const int64_t i = f / kRowVec, w = f - i * kRowVec;
+      const int64_t t = window_row_token(p, pb, mode, i);
+      const int64_t c = t / p.C;
+      const int64_t row = c < p.sink && c < b0 ? t : (p.sink + c % (p.local + 1)) * p.C + t % p.C;
+      dst = static_cast<size_t>(row * kRowVec + w);
+      kw[dst] = sw[i * kRowVec + w];
+      vw[dst] = sw[(WR + i) * kRowVec + w];
+    }
+  }
+  pdl_trigger();
+}
+
 }  // namespace
 
 cudaError_t launch_gather_host(const LayerParams& p, const void* k_host, const void* v_host,
@@ -335,13 +397,22 @@ cudaError_t launch_gather_warm(const LayerParams& p, const void* k_host, const v
                                const int64_t* pos, const int32_t* group_idx, int slots,
                                int32_t* tags, int32_t* stamps, int32_t* slot_map, void* k_work,
                                void* v_work, int refresh_window, unsigned long long* counters,
-                               unsigned* err, cudaStream_t s) {
+                               unsigned* err, cudaStream_t s, int2* plan, int32_t* n_plan) {
   int mp = 2;
   while (mp < slots) mp <<= 1;
   return launch_pdl(gather_warm_kernel, dim3(p.B * p.Hkv), dim3(kWarmThreads), 0, s, 1,
                     static_cast<const uint4*>(k_host), static_cast<const uint4*>(v_host), pos,
                     group_idx, p, slots, mp, tags, stamps, slot_map, refresh_window,
-                    static_cast<uint4*>(k_work), static_cast<uint4*>(v_work), counters, err);
+                    static_cast<uint4*>(k_work), static_cast<uint4*>(v_work), counters, err,
+                    plan, n_plan);
+}
+
+cudaError_t launch_warm_fill(const LayerParams& p, const void* staging, const int2* plan,
+                             const int32_t* n_plan, const int64_t* pos, int slots, int mode,
+                             void* k_work, void* v_work, unsigned* err, cudaStream_t s) {
+  return launch_pdl(warm_fill_kernel, dim3(p.B * p.Hkv), dim3(kWarmThreads), 0, s, 1,
+                    static_cast<const uint4*>(staging), plan, n_plan, pos, p, slots, mode,
+                    static_cast<uint4*>(k_work), static_cast<uint4*>(v_work), err);
 }
 
 }  // namespace hga

@@ -176,6 +176,30 @@ cudaError_t launch_gather_host(const LayerParams& p, const void* k_host, const v
                                const int64_t* pos, const int32_t* group_idx, void* k_work,
                                void* v_work, int refresh_window, unsigned* err, cudaStream_t s);
 
+// Window rows a host-tier step copies for a query at pb, in the order a cold
+// store stages them: with refresh mode 1 the sink chunks (c < min(sink, b0)),
+// then the local chunks [b0, cur); then the current chunk from its first row
+// (modes 0 and 1) or only the row at pb (mode 2), up to pb.
+__host__ __device__ inline int64_t window_row_count(const LayerParams& p, int64_t pb, int mode) {
+  const int64_t cur = pb / p.C, b0 = cur - p.local > 0 ? cur - p.local : 0;
+  const int64_t n_sink = mode == 1 ? (p.sink < b0 ? p.sink : b0) * p.C : 0;
+  const int64_t n_local = mode == 1 ? (cur - b0) * p.C : 0;
+  return n_sink + n_local + (pb - (mode == 2 ? pb : cur * p.C) + 1);
+}
+__host__ __device__ inline int64_t window_row_token(const LayerParams& p, int64_t pb, int mode,
+                                                    int64_t i) {
+  const int64_t cur = pb / p.C, b0 = cur - p.local > 0 ? cur - p.local : 0;
+  const int64_t n_sink = mode == 1 ? (p.sink < b0 ? p.sink : b0) * p.C : 0;
+  const int64_t n_local = mode == 1 ? (cur - b0) * p.C : 0;
+  if (i < n_sink) return i;
+  if (i < n_sink + n_local) return b0 * p.C + (i - n_sink);
+  return (mode == 2 ? pb : cur * p.C) + (i - n_sink - n_local);
+}
+// Rows per (sequence, KV head) of a cold store's window staging.
+__host__ __device__ inline int64_t window_row_capacity(const LayerParams& p) {
+  return static_cast<int64_t>(p.sink + p.local + 1) * p.C;
+}
+
 // Warm tier: at most kWarmMax cached groups per (sequence, KV head).
 constexpr int kWarmMax = 2048;
 // One step of the warm tier (host_tier.cu): LRU lookup and eviction in
@@ -185,7 +209,21 @@ cudaError_t launch_gather_warm(const LayerParams& p, const void* k_host, const v
                                const int64_t* pos, const int32_t* group_idx, int slots,
                                int32_t* tags, int32_t* stamps, int32_t* slot_map, void* k_work,
                                void* v_work, int refresh_window, unsigned long long* counters,
-                               unsigned* err, cudaStream_t s);
+                               unsigned* err, cudaStream_t s, int2* plan = nullptr,
+                               int32_t* n_plan = nullptr);
+// With plan / n_plan the warm step above only decides: the table and slot map
+// are written, and each (sequence, KV head)'s misses as (group, slot) pairs
+// [B*Hkv][kg] with their count [B*Hkv]; no row is copied.  launch_warm_fill then
+// copies the rows a cold store staged (pinned host memory, read in place):
+// staging per (sequence, KV head) = [K | V][kg][16 rows][128] of the misses in
+// plan order, then [K | V][window_row_capacity][128] of the window rows.
+cudaError_t launch_warm_fill(const LayerParams& p, const void* staging, const int2* plan,
+                             const int32_t* n_plan, const int64_t* pos, int slots, int mode,
+                             void* k_work, void* v_work, unsigned* err, cudaStream_t s);
+// Bytes of staging per (sequence, KV head).
+__host__ __device__ inline int64_t cold_stage_unit_bytes(const LayerParams& p) {
+  return 2 * (static_cast<int64_t>(p.kg) * 16 + window_row_capacity(p)) * p.D * 2;
+}
 
 // The bf16, D = 128 prefill kernel (64-query blocks on tcgen05 / TMEM) applies to p.
 bool prefill_tc_path(const LayerParams& p, int dtype);

@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define HGA_ABI_VERSION 5
+#define HGA_ABI_VERSION 6
 
 typedef enum hga_status {
   HGA_OK = 0,
@@ -410,6 +410,64 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q, const int64_t* 
  * hga_decode_step does not take.
  */
 hga_status hga_decode_step_launches(const hga_config* cfg, int64_t n_alloc, int32_t* launches);
+
+/*
+ * Cold tier (HGA technical summary, "Architettura della Memoria": the whole K/V
+ * history may live in host RAM or on NVMe; VRAM holds the summaries, the
+ * windows and the warm LRU of routed groups).  The history lives in a file, K
+ * then V, each [B, Hkv, n_alloc, 128] bf16 rows; a decode step with a cold
+ * store runs
+ *   hga_route -> hga_warm_plan -> (plan and counts to the host) ->
+ *   hga_cold_stage -> hga_warm_fill -> hga_attend_warm,
+ * so that only the warm tier's misses and the window rows are read from the
+ * file, by a pool of host threads, into pinned staging the fill kernel reads
+ * in place.  Staging per (sequence, KV head): [K | V][kg][16][128] of the
+ * misses in plan order, then [K | V][(sink + local + 1) * C][128] of the
+ * window rows (hga_cold_stage_bytes gives the whole size).
+ */
+typedef struct hga_cold_store hga_cold_store;
+
+/* Opens the history file at path (create != 0: created, or grown, to
+ * 2 * B * Hkv * n_alloc * 256 bytes).  A file shorter than that without create
+ * is HGA_ERR_INVALID_ARG.  Close with hga_cold_close. */
+hga_status hga_cold_open(const char* path, const hga_config* cfg, int64_t n_alloc,
+                         int32_t create, hga_cold_store** store);
+hga_status hga_cold_close(hga_cold_store* store);
+
+/* Writes rows [t0, t1) of every (sequence, KV head) from host k, v
+ * [B, Hkv, n_alloc, 128] bf16 (after a prefill; each decode step's new row
+ * before that step), with up to `threads` host threads.  Synchronous. */
+hga_status hga_cold_write(hga_cold_store* store, const void* k, const void* v, int64_t t0,
+                          int64_t t1, int32_t threads);
+
+/* Bytes of staging for one step of cfg's batch. */
+hga_status hga_cold_stage_bytes(const hga_config* cfg, size_t* bytes);
+
+/* The decision half of hga_gather_warm: the same table update and slot_map,
+ * and per (sequence, KV head) its misses as (group, slot) int32 pairs in plan
+ * [B, Hkv, kg, 2] with their count in n_plan [B, Hkv] (device); no row is
+ * copied. */
+hga_status hga_warm_plan(const hga_config* cfg, int64_t n_alloc, const int64_t* pos,
+                         const int32_t* group_idx, int32_t warm_groups, int32_t* tags,
+                         int32_t* stamps, int32_t* slot_map, int32_t* plan, int32_t* n_plan,
+                         uint64_t* counters, void* stream);
+
+/* Reads a step's rows from the file into staging (host memory, pinned for
+ * hga_warm_fill): the missed groups of plan / n_plan (host copies of
+ * hga_warm_plan's outputs) and the window rows of pos (host [B]) under
+ * window_mode (0, 1, 2 as in hga_gather_host).  Synchronous, `threads` host
+ * threads.  A group or position outside the history is HGA_ERR_INVALID_ARG. */
+hga_status hga_cold_stage(hga_cold_store* store, const hga_config* cfg, const int64_t* pos,
+                          const int32_t* plan, const int32_t* n_plan, int32_t window_mode,
+                          void* staging, int32_t threads);
+
+/* Copies the staged rows into the warm working buffers: the misses into the
+ * slots plan names, the window rows into the window (device pos, plan and
+ * n_plan; staging pinned host memory read in place over the host link). */
+hga_status hga_warm_fill(const hga_config* cfg, int64_t n_alloc, const int64_t* pos,
+                         const void* staging, const int32_t* plan, const int32_t* n_plan,
+                         int32_t warm_groups, int32_t window_mode, void* k_work, void* v_work,
+                         void* stream);
 
 /*
  * Backward pass of a prefill call of hga_attend (HGA technical summary,

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_abi_version_and_status_strings(lib):
     from hierarchical_sparse_attention_hga_b200 import binding as B
-    assert B.hga_abi_version() == 5
+    assert B.hga_abi_version() == 6
     assert B.hga_status_string(0) == "HGA_OK"
     assert B.hga_status_string(6) == "HGA_ERR_DEVICE_CHECK"
     assert B.hga_status_string(99) == "HGA_ERR_UNKNOWN"

@@ -262,3 +262,51 @@ def test_warm_attend_flags_a_slot_outside_the_table():
     assert B.hga_device_status() == 6
     assert torch.isfinite(out).all()
     assert B.hga_device_status() == 0
+
+
+def test_cold_tier_decode_loop_equals_device_path(tmp_path):
+    """The history in a file (the cold tier): each step plans on the GPU, stages the
+    misses and window rows from the file on the host, fills the warm buffers and
+    attends; 48 routed steps with drifting queries across chunk boundaries give the
+    device-resident path's bits, and only the misses are read."""
+    wl = _wl()
+    x = S.make_inputs(wl, 59)
+    slots = 64
+    w = Warm(wl, x, slots)
+    lay = w.host_layer
+    qs = S.drifting_queries(wl, 60, 48, 0.95)
+    plan = torch.empty(w.bh, wl.topk_groups, 2, dtype=torch.int32, device="cuda")
+    n_plan = torch.empty(w.bh, dtype=torch.int32, device="cuda")
+    plan_h = torch.empty(plan.shape, dtype=torch.int32).pin_memory()
+    n_plan_h = torch.empty(n_plan.shape, dtype=torch.int32).pin_memory()
+    staging = torch.zeros(B.hga_cold_stage_bytes(lay), dtype=torch.uint8).pin_memory()
+    start = 4000
+    B.hga_build_summaries(w.dev_layer, w.k, w.n, 0, start, w.cs, w.gs)
+    read_groups = 0
+    with B.ColdStore(tmp_path / "kv.bin", lay, w.n, create=True) as store:
+        store.write(w.k_host, w.v_host, 0, start)          # the prompt's history
+        for t, p in enumerate(range(start, start + 48)):
+            store.write(w.k_host, w.v_host, p, p + 1)       # the step's new row
+            pos = np.array([p, p - 3], dtype=np.int64)
+            pos_t = torch.as_tensor(pos, device="cuda")
+            q = to_device(qs[t], wl.dtype)
+            mode = 1 if t == 0 else 2
+            B.hga_build_summaries(w.dev_layer, w.k, w.n, p, p + 1, w.cs, w.gs)
+            B.hga_route(w.dev_layer, q, 1, pos_t, w.cs, w.gs, w.n, w.ci, w.gi)
+            B.hga_warm_plan(lay, w.n, pos_t, w.gi, slots, w.tags, w.stamps, w.slot_map, plan,
+                            n_plan, counters=w.counters)
+            plan_h.copy_(plan)
+            n_plan_h.copy_(n_plan)
+            torch.cuda.synchronize()
+            store.stage(lay, pos, plan_h.numpy(), n_plan_h.numpy(), mode, staging, threads=4)
+            B.hga_warm_fill(lay, w.n, pos_t, staging, plan, n_plan, slots, mode, w.k_work,
+                            w.v_work)
+            out_w, lse_w = w.attend(q, pos_t, warm=True)
+            out_d, lse_d = w.attend(q, pos_t, warm=False)
+            torch.cuda.synchronize()
+            assert B.hga_device_status() == 0
+            assert torch.equal(out_w.view(torch.int32), out_d.view(torch.int32)), f"step at {p}"
+            assert torch.equal(lse_w.view(torch.int32), lse_d.view(torch.int32))
+            read_groups += int(n_plan_h.sum())
+    hits, misses = w.counters.cpu().tolist()
+    assert misses == read_groups and hits > misses

@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b_decode_32k")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--context", type=int, default=None, help="override the context length")
+    ap.add_argument("--dtype", default=None, choices=["bf16", "f32"],
+                    help="override the K/V storage type (f32 runs the general attention kernels)")
     ap.add_argument("--layers", type=int, default=0,
                     help="attention layers per decode step (0: 4, or 1 for the host tier)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
@@ -400,6 +402,13 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
         B.hga_gather_host(layer, d["k_host"], d["v_host"], n, pos, d["gi"], d["k_work"],
                           d["v_work"], refresh_window=True, stream=sh)
 
+    # the one-call decode step takes bf16, D = 128; other shapes (fp32 caches, D = 64)
+    # run the append, routing and general attention calls
+    try:
+        fusable = not hot and B.hga_decode_step_launches(layer, n) >= 1
+    except B.HGAError:
+        fusable = False
+
     def parts_of(d):
         k_src, v_src = (d["k_host"], d["v_host"]) if hot else (d["k"], d["v"])
         k_att, v_att = (d["k_work"], d["v_work"]) if hot else (d["k"], d["v"])
@@ -418,7 +427,7 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
         if hot:
             pr["gather"] = lambda st: B.hga_gather_host(layer, d["k_host"], d["v_host"], n, pos,
                                                         d["gi"], d["k_work"], d["v_work"], stream=st)
-        else:
+        elif fusable:
             # the whole step in one call: summary append, routing and attention
             pr["decode_step"] = lambda st: B.hga_decode_step(layer, d["q"], pos, d["cs"], d["gs"], n,
                                                              d["k"], d["v"], d["ci"], d["gi"],
@@ -448,13 +457,20 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
         step = one_layer
         comparisons = {"four_call_step_us": chain_step(parts, ("route_chunks", "route_groups",
                                                                 "gather", "attend"))}
-    else:
+    elif fusable:
         def step(st):
             for pr in parts_l:
                 pr["decode_step"](st)
         comparisons = {"two_call_step_us": chain_step(parts, ("route", "attend")),
                        "four_call_step_us": chain_step(parts, ("route_chunks", "route_groups",
                                                                "attend"))} if compare else {}
+    else:
+        layer_steps = [chain_step(pr, ("route", "attend")) for pr in parts_l]
+
+        def step(st):
+            for ls in layer_steps:
+                ls(st)
+        comparisons = {}
 
     for _ in range(max(1, warmup)):
         step(sh)
@@ -487,13 +503,14 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
     nb = step_bytes(wl)
     nb["route"] = nb["route_chunks"] + nb["route_groups"]
     nb["decode_step"] = decode_step_bytes(wl)
-    one_launch = not hot and B.hga_decode_step_launches(layer, n) == 1
+    one_launch = fusable and B.hga_decode_step_launches(layer, n) == 1
     if one_launch:
         kern = "decode_step"
     else:
         kern = max(("route", "attend"), key=lambda kk: ms[kk])
     kernel_name = {"decode_step": "decode_step_kernel", "route": "route_decode_kernel",
-                   "attend": "attend_decode_bf16_kernel"}[kern]
+                   "attend": "attend_decode_bf16_kernel" if wl.dtype == "bf16" and
+                   wl.head_dim == 128 else "attend_kernel + combine_kernel"}[kern]
     lay = layers if kern == "decode_step" else 1
     ds = [torch.cuda.Event(enable_timing=True) for _ in range(n_side)]
     de = [torch.cuda.Event(enable_timing=True) for _ in range(n_side)]
@@ -515,7 +532,7 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
     for qh, d in zip(q_host, L_):
         qh.copy_(d["q"])
     kv_new = torch.empty(len(L_), 2, wl.batch, wl.heads_kv, wl.head_dim,
-                         dtype=torch.bfloat16).pin_memory()
+                         dtype=(L_[0]["k_host"] if hot else L_[0]["k"]).dtype).pin_memory()
     for li, d in enumerate(L_):
         kv_new[li, 0].copy_((d["k_host"] if hot else d["k"])[:, :, p].cpu())
         kv_new[li, 1].copy_((d["v_host"] if hot else d["v"])[:, :, p].cpu())
@@ -1339,6 +1356,8 @@ def workload_of(args) -> S.Workload:
         wl = wl.with_(batch=args.batch)
     if args.context:
         wl = wl.with_(context=args.context)
+    if args.dtype:
+        wl = wl.with_(dtype=args.dtype)
     return wl
 
 
@@ -1441,7 +1460,8 @@ def main():
             **rec}
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, seed, args.cpu_seconds, line["unit"])
-    default_run = args.workload == "llama3_8b_decode_32k" and not args.batch and not args.context
+    default_run = (args.workload == "llama3_8b_decode_32k" and not args.batch and not args.context
+                   and not args.dtype)
     if world == 1 and default_run and not args.no_workloads:
         del x
         subs = {}

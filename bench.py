@@ -369,16 +369,27 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
-    # every layer: its own caches, summaries, routing buffers and outputs
+    # every layer: its own caches, summaries, routing buffers and outputs; the layers'
+    # queries (and the new K/V rows, see e2e) share one device input buffer and their
+    # outputs one output buffer, so a step moves its inputs and results in one copy each
+    kv_dtype = k0.dtype
+    q_bytes = layers * q0.numel() * q0.element_size()
+    kv_bytes = 0 if hot else layers * 2 * wl.batch * wl.heads_kv * wl.head_dim * k0.element_size()
+    dev_in = torch.empty(q_bytes + kv_bytes, dtype=torch.uint8, device=dev)
+    qs_all = dev_in[:q_bytes].view(q0.dtype).view((layers,) + tuple(q0.shape))
+    kv_dev = None if hot else dev_in[q_bytes:].view(kv_dtype).view(
+        layers, 2, wl.batch, wl.heads_kv, wl.head_dim)
+    outs_all = torch.empty(layers, wl.batch, wl.heads_q, 1, wl.head_dim, device=dev)
     L_ = []
     for li in range(layers):
-        q, k, v = (q0, k0, v0) if li == 0 else (q0.clone(), k0.clone(), v0.clone())
-        d = dict(q=q, k=k, v=v,
+        k, v = (k0, v0) if li == 0 else (k0.clone(), v0.clone())
+        qs_all[li].copy_(q0)
+        d = dict(q=qs_all[li], k=k, v=v,
                  cs=torch.empty(bh, nc, wl.head_dim, device=dev),
                  gs=torch.empty(bh, nc, ng, wl.head_dim, device=dev),
                  ci=torch.empty(bh, wl.topk_chunks, dtype=torch.int32, device=dev),
                  gi=torch.empty(bh, wl.topk_groups, dtype=torch.int32, device=dev),
-                 out=torch.empty(wl.batch, wl.heads_q, 1, wl.head_dim, device=dev),
+                 out=outs_all[li],
                  lse=torch.empty(wl.batch, wl.heads_q, 1, device=dev))
         L_.append(d)
     del q0, k0, v0
@@ -527,40 +538,41 @@ def decode_record(args, wl: S.Workload, layers: int, steps: int, warmup: int, wo
     achieved = nb[kern] / (kern_ms * 1e-3) / 1e9
 
     # e2e: every step, the new token's q and K/V rows of every layer come in from
-    # pinned host memory and every layer's output goes back
-    q_host = [torch.empty(d["q"].shape, dtype=d["q"].dtype).pin_memory() for d in L_]
-    for qh, d in zip(q_host, L_):
-        qh.copy_(d["q"])
-    kv_new = torch.empty(len(L_), 2, wl.batch, wl.heads_kv, wl.head_dim,
-                         dtype=(L_[0]["k_host"] if hot else L_[0]["k"]).dtype).pin_memory()
+    # pinned host memory (one copy into the shared input buffer; the K/V rows then
+    # go to their cache rows on the device) and every layer's output goes back (one
+    # copy of the shared output buffer)
+    host_in = torch.empty(dev_in.shape, dtype=torch.uint8).pin_memory()
+    host_in.copy_(dev_in)
+    kv_new = None if hot else host_in[q_bytes:].view(kv_dtype).view(kv_dev.shape)
+    kv_rows = torch.empty(layers, 2, wl.batch, wl.heads_kv, wl.head_dim, dtype=kv_dtype)
     for li, d in enumerate(L_):
-        kv_new[li, 0].copy_((d["k_host"] if hot else d["k"])[:, :, p].cpu())
-        kv_new[li, 1].copy_((d["v_host"] if hot else d["v"])[:, :, p].cpu())
-    out_host = [torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory() for d in L_]
+        kv_rows[li, 0].copy_((d["k_host"] if hot else d["k"])[:, :, p].cpu())
+        kv_rows[li, 1].copy_((d["v_host"] if hot else d["v"])[:, :, p].cpu())
+    if not hot:
+        kv_new.copy_(kv_rows)
+    out_host = torch.empty(outs_all.shape, dtype=outs_all.dtype).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e = []
     for i in range(warmup + min(steps, 100)):
         flush()
         e0.record(stream)
+        dev_in.copy_(host_in, non_blocking=True)
         for li, d in enumerate(L_):
-            d["q"].copy_(q_host[li], non_blocking=True)
             if hot:  # the new token's K/V goes into the host cache, a host-side write
-                d["k_host"][:, :, p].copy_(kv_new[li, 0])
-                d["v_host"][:, :, p].copy_(kv_new[li, 1])
+                d["k_host"][:, :, p].copy_(kv_rows[li, 0])
+                d["v_host"][:, :, p].copy_(kv_rows[li, 1])
             else:
-                d["k"][:, :, p].copy_(kv_new[li, 0], non_blocking=True)
-                d["v"][:, :, p].copy_(kv_new[li, 1], non_blocking=True)
+                d["k"][:, :, p].copy_(kv_dev[li, 0])
+                d["v"][:, :, p].copy_(kv_dev[li, 1])
         graphs["step"].replay()
-        for li, d in enumerate(L_):
-            out_host[li].copy_(d["out"], non_blocking=True)
+        out_host.copy_(outs_all, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
         if i >= warmup:
             e2e.append(e0.elapsed_time(e1))
     ms_e2e = ranks.max(sum(e2e) / len(e2e))
-    h2d = sum(t.numel() * t.element_size() for t in q_host) + \
-        (0 if hot else kv_new.numel() * kv_new.element_size())
-    d2h = sum(t.numel() * t.element_size() for t in out_host)
+    h2d = q_bytes + kv_bytes
+    d2h = out_host.numel() * out_host.element_size()
 
     per_layer_ms = ms_step / layers
     total_bytes = nb["summaries"] + nb["route"] + nb["attend"]

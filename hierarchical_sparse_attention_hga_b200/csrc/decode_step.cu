@@ -20,17 +20,22 @@
 // (bf16, 128B-swizzled boxes).  So the whole item is a stream of equal units
 // spread over the warps, with up to 3 W units in flight.
 //
-//   scan:    candidate summary units, round-robin over all warps; each warp
-//            scores its rows with the routing kernel's arithmetic and keeps a
-//            running top-kc list in registers (a bitonic network over 64-bit
-//            keys: score order, then the lower chunk index), then publishes it;
-//   forced:  the sink, local and current chunks' K/V units, round-robin over
-//            warps 1..W-1, queued right behind their scan units (so their
-//            loads fill the gap while the routing finishes);
-//   route:   warp 0 merges the W lists (top-kc), streams the chosen chunks'
-//            group summaries through its ring and keeps a running top-kg list
-//            the same way, then publishes the routed group list;
-//   routed:  the routed groups' K/V units, round-robin over all warps;
+//   scan:    candidate summary units, round-robin over all warps (the first
+//            ones issued before the position is known); each warp scores its
+//            rows with the routing kernel's arithmetic and keeps a running
+//            top-kc list in registers (insertion by ballot and shuffle, or a
+//            bitonic merge for a unit with many winners: score order, then the
+//            lower chunk index), then publishes it;
+//   level 1: after a barrier, every thread ranks its share of the W lists'
+//            keys against all of them; the kc best are the chosen chunks;
+//   level 2: each warp streams its chosen chunks' group summaries, scores them,
+//            and, after a barrier, the kc * Ng keys are ranked the same way into
+//            the routed group list;
+//   forced:  each warp's share of the sink, local and current chunks' K/V units,
+//            queued right behind its group-summary copies (so their loads land
+//            while the level-2 selection runs);
+//   routed:  the routed groups' K/V units, round-robin over all warps; every K/V
+//            unit is attended as it lands (mma.sync, P in registers);
 //   merge:   the warps' (o, m, l) partials, by log-sum-exp in shared memory.
 //
 // The append warp meanwhile finalises the summary rows that the item's new

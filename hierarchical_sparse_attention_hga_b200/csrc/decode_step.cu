@@ -227,6 +227,7 @@ constexpr int kL2Max = kKcMax * 8;  // level-2 candidates: chosen chunks x group
 
 struct StepSmem {  // byte offsets into the dynamic shared memory (after alignment)
   int W, n_tab, n_pt;  // n_pt: block-table entries staged per item (paged pools), else 0
+  int peer_floats;     // clusters: the CTAs' partials gathered in rank 0, else 0
   __host__ __device__ size_t rings() const { return static_cast<size_t>(W) * kS * kStageBytes; }
   __host__ __device__ size_t o_union() const { return rings(); }                    // u64 [W][kKcMax]
   __host__ __device__ size_t o_ckey() const { return o_union() + static_cast<size_t>(W) * kKcMax * 8; }
@@ -240,7 +241,12 @@ struct StepSmem {  // byte offsets into the dynamic shared memory (after alignme
   __host__ __device__ size_t o_pages() const {  // int [n_pt], 16-byte aligned
     return (o_tab() + static_cast<size_t>(n_tab) * 8 + 15) & ~static_cast<size_t>(15);
   }
-  __host__ __device__ size_t bytes() const { return 1024 + o_pages() + static_cast<size_t>(n_pt) * 4; }
+  __host__ __device__ size_t o_peer() const {  // float [peer_floats], 16-byte aligned
+    return (o_pages() + static_cast<size_t>(n_pt) * 4 + 15) & ~static_cast<size_t>(15);
+  }
+  __host__ __device__ size_t bytes() const {
+    return 1024 + o_peer() + static_cast<size_t>(peer_floats) * 4;
+  }
 };
 
 template <typename TO>
@@ -296,7 +302,17 @@ __device__ __forceinline__ int rank_among(const uint64_t* keys, int n, uint64_t 
 // start, validated before the first barrier), and every K/V tile's row comes
 // from it.  An entry that is not a page of the pool is flagged and read as
 // zeros (its tiles start at a negative row, which the tensor copy fills).
-template <int W, int R1, typename TO, bool PAGED>
+//
+// NC > 1 (small batches, NC items' worth of SMs each): each item on a cluster of
+// NC CTAs, one per SM.  Every CTA scans a slice of the candidate summaries
+// (units round-robin over the cluster's NC x W warps), takes its slice's
+// top-kc and writes it into rank 0's shared memory (distributed shared memory,
+// then a remote mbarrier arrival); rank 0 selects the chunks among the NC lists,
+// runs level 2 and broadcasts the routed list the same way; every CTA attends
+// its share of the window units at once and of the routed units on arrival,
+// and sends its partial (o, m, l) to rank 0, which merges them and writes the
+// outputs.  Every wait on another CTA is bounded.
+template <int W, int R1, typename TO, bool PAGED, int NC>
 __global__ void __launch_bounds__((W + 1) * 32, W == 7 ? 1 : 2)
 decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, StepArgs<TO> a, LayerParams p) {
@@ -304,11 +320,22 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
   __shared__ uint64_t bars[W][kS];
   __shared__ float s_ml[W][16][2];
   __shared__ int s_abort;
+  __shared__ uint64_t s_l1all[NC > 1 ? NC : 1][kKcMax];  // rank 0: every CTA's slice top-kc
+  __shared__ uint64_t s_l1bar;   // rank 0: the NC slice lists arrived
+  __shared__ uint64_t s_hand;    // ranks > 0: the routed list arrived
+  __shared__ uint64_t s_peerbar; // rank 0: the NC - 1 partials arrived
+  __shared__ int s_ng_in;        // ranks > 0: routed groups in the list received
+  __shared__ int s_bad[2];       // rank 0: a wait of this item gave up (by item parity)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;  // streaming threads: 0 .. W * 32 - 1
   uint8_t* base = smem_raw + ((1024 - (ptx::smem_u32(smem_raw) & 1023)) & 1023);
-  StepSmem L{W, summ::table_entries(p, kD), PAGED ? a.kv.max_pages : 0};
+  StepSmem L{W, summ::table_entries(p, kD), PAGED ? a.kv.max_pages : 0,
+             NC > 1 ? NC * p.G * (kD + 2) : 0};
+  // clusters: this CTA's rank, and its warps' place among the cluster's NW warps
+  const int crank = NC > 1 ? static_cast<int>(ptx::cluster_ctarank()) : 0;
+  constexpr int NW = NC * W;
+  float* peer = reinterpret_cast<float*>(base + L.o_peer());  // rank 0: [NC][G][kD] o, [NC][G] (m, l)
   uint64_t* s_union = reinterpret_cast<uint64_t*>(base + L.o_union());
   uint64_t* ckey = reinterpret_cast<uint64_t*>(base + L.o_ckey());  // chosen chunks' keys, rank order
   uint64_t* gkey = reinterpret_cast<uint64_t*>(base + L.o_gkey());
@@ -325,10 +352,17 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
     ptx::prefetch_tensormap(&tm_v);
     for (int w = 0; w < W; ++w)
       for (int s = 0; s < kS; ++s) ptx::mbar_init(&bars[w][s], 1);
+    ptx::mbar_init(&s_l1bar, NC);
+    ptx::mbar_init(&s_hand, 1);
+    ptx::mbar_init(&s_peerbar, NC > 1 ? NC - 1 : 1);
     s_abort = 0;
+    s_bad[0] = s_bad[1] = 0;
     ptx::fence_barrier_init();
   }
   __syncthreads();
+  if (NC > 1) ptx::cluster_barrier();  // every CTA's barriers exist before any remote arrival
+  const int item0 = NC > 1 ? static_cast<int>(blockIdx.x) / NC : static_cast<int>(blockIdx.x);
+  const int istride = NC > 1 ? static_cast<int>(gridDim.x) / NC : static_cast<int>(gridDim.x);
 
   // ------------------------------------------------------------ append warp
   if (warp == W) {
@@ -336,7 +370,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
       for (int i = lane; i < L.n_tab; i += 32) tab[i] = summ::table_entry(p, kD, i);
       __syncwarp();
       pdl_wait();  // the rows read and written may belong to the kernel just before
-      for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+      for (int item = item0; item < a.n_items && crank == 0; item += istride) {
         const int b = item / p.Hkv, h = item % p.Hkv;
         const int64_t pb = a.pos[b];
         if (pb < 0 || pb >= p.n_alloc) continue;
@@ -354,6 +388,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
       }
     }
     cta_sync();
+    if (NC > 1) ptx::cluster_barrier();
     pdl_trigger();
     return;
   }
@@ -374,9 +409,9 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
   const int cpu = kRows / p.Ng;  // chosen chunks per group-summary unit
 
   pdl_wait();  // summaries may come from the kernel just before
-  for (int item = blockIdx.x; item < a.n_items; item += gridDim.x, ++item_no) {
+  for (int item = item0; item < a.n_items; item += istride, ++item_no) {
     const int b = item / p.Hkv, h = item % p.Hkv;
-    if (s_abort) {  // an earlier item of this CTA timed out: write the empty result, no waits
+    if (NC == 1 && s_abort) {  // an earlier item of this CTA timed out: write the empty result, no waits
       if (warp == 0) {
         for (int i = lane; i < p.kc; i += 32) a.chunk_idx[static_cast<size_t>(item) * p.kc + i] = -1;
         for (int i = lane; i < p.kg; i += 32) a.group_idx[static_cast<size_t>(item) * p.kg + i] = -1;
@@ -437,9 +472,10 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
 
     // 2. the warp's first scan units before the position is known: the rows that
     //    exist past the sink (the units beyond this item's candidates are dropped)
-    const int n_spec = min(kS, n_su_max > warp ? (n_su_max - warp + W - 1) / W : 0);
+    const int gw = crank * W + warp;  // this warp among the cluster's NW warps
+    const int n_spec = min(kS, n_su_max > gw ? (n_su_max - gw + NW - 1) / NW : 0);
     for (int i = 0; i < n_spec; ++i) {
-      const int su = warp + i * W;
+      const int su = gw + i * NW;
       if (lane == 0) {
         const int nr = min(kRows, rows_max - su * kRows);
         ptx::mbar_expect_tx(&wbar[issued % kS], static_cast<uint32_t>(nr) * kRowBytes);
@@ -471,15 +507,17 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int ns = min(p.kc, n_cand);       // chosen chunks
     const int n_l2 = ns * p.Ng;             // level-2 candidates
     const int ng = min(p.kg, n_l2);         // routed groups
-    auto count = [&](int n) { return n > warp ? (n - warp + W - 1) / W : 0; };  // i = warp + k W < n
+    auto count = [&](int n) { return n > gw ? (n - gw + NW - 1) / NW : 0; };  // i = gw + k NW < n
+    auto count_cta = [&](int n) { return n > warp ? (n - warp + W - 1) / W : 0; };
     const int n_head = max(count(n_su), n_spec);  // scan units (those past n_su are dropped)
-    const int n_mine = count(ns);                 // chosen chunks warp, warp + W, ...
+    const int n_mine = crank == 0 ? count_cta(ns) : 0;  // chosen chunks warp, warp + W, ... (rank 0)
     const int n_fw = count(n_forced);             // window units warp, warp + W, ...
     const int n_l2u = (n_mine + cpu - 1) / cpu;
     const int n_rw = count(ng);
     // stream index -> unit: [0, e_l2) scan; [e_l2, e_fw) group summaries; [e_fw, e_rt)
     // window; [e_rt, e_all) routed
-    const int e_l2 = n_head, e_fw = e_l2 + n_l2u, e_rt = e_fw + n_fw, e_all = e_rt + n_rw;
+    const int e_l2 = n_head, e_fw = e_l2 + n_l2u, e_rt = e_fw + n_fw;
+    int e_all = e_rt + n_rw;
     auto forced_token = [&](int f) -> int64_t {
       return static_cast<int64_t>(f < su_sink ? f : u_first_local + (f - su_sink)) * kUnit;
     };
@@ -492,7 +530,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
         uint64_t* bar = &wbar[issued % kS];
         if (lane == 0) {
           if (i < e_l2) {
-            const int su = warp + i * W;
+            const int su = gw + i * NW;
             const int nr = min(kRows, n_cand - su * kRows);
             ptx::mbar_expect_tx(bar, static_cast<uint32_t>(nr) * kRowBytes);
             ptx::bulk_load(st, cbase + static_cast<size_t>(su) * kRows * kD,
@@ -510,10 +548,10 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
                                static_cast<uint32_t>(p.Ng) * kRowBytes, bar);
             }
           } else if (i < e_rt) {
-            issue_unit(&tm_k, &tm_v, st, bar, kv_row(forced_token(warp + (i - e_fw) * W)));
+            issue_unit(&tm_k, &tm_v, st, bar, kv_row(forced_token(gw + (i - e_fw) * NW)));
           } else {
             issue_unit(&tm_k, &tm_v, st, bar,
-                       kv_row(static_cast<int64_t>(glist[warp + (i - e_rt) * W]) * kUnit));
+                       kv_row(static_cast<int64_t>(glist[gw + (i - e_rt) * NW]) * kUnit));
           }
         }
         ++issued;
@@ -544,8 +582,8 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
     for (int r = 0; r < R1; ++r) l1[r] = 0ull;
     consume(0, e_l2, e_l2, [&](int i, uint8_t* st) {
-      if (i * W + warp < n_su) {
-        const int su = warp + i * W;
+      if (i * NW + gw < n_su) {
+        const int su = gw + i * NW;
         const float sc = score16(reinterpret_cast<const float*>(st), qv);
         const int r = su * kRows + lane;
         offer16<R1>(l1, lane < kRows && r < n_cand ? make_key(sc, p.sink + r) : 0ull, p.kc);
@@ -568,87 +606,145 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
           }
         }
     }
+    if (NC > 1)
+      for (int c = tid; c < p.kc; c += W * 32) ckey[c] = 0ull;  // this CTA's slice top-kc
     named_sync(kBarStream, W * 32);  // B1
 
-    // ---- level 1: the kc best of the W lists, by rank, into chunks (rank order)
+    // ---- level 1: the kc best of the W lists, by rank, into chunks (rank order);
+    // in a cluster, each CTA's slice top-kc first, then rank 0 over the NC lists
     for (int c = tid; c < W * p.kc; c += W * 32) {
       const uint64_t key = s_union[c];
       if (key == 0ull) continue;
       const int rank = rank_among(s_union, W * p.kc, key);
-      if (rank < ns) {
+      if (NC > 1) {
+        if (rank < p.kc) ckey[rank] = key;
+      } else if (rank < ns) {
         chunks[rank] = key_id(key);
         ckey[rank] = key;
       }
     }
+    if (NC > 1) {
+      named_sync(kBarStream, W * 32);
+      const uint32_t dst = ptx::map_to_rank(ptx::smem_u32(&s_l1all[crank][0]), 0);
+      for (int c = tid; c < p.kc; c += W * 32) ptx::st_cluster_u64(dst + 8u * c, ckey[c]);
+      ptx::fence_cluster();
+      named_sync(kBarStream, W * 32);
+      if (tid == 0) ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(&s_l1bar), 0));
+      if (crank == 0) {
+        if (!ptx::mbar_wait_cluster(&s_l1bar, item_no & 1, kWaitLimit, limit_ns)) timed_out = true;
+        for (int c = tid; c < NC * p.kc; c += W * 32) {
+          const uint64_t key = s_l1all[c / p.kc][c % p.kc];
+          if (key == 0ull) continue;
+          int rank = 0;
+          for (int r = 0; r < NC; ++r) rank += rank_among(s_l1all[r], p.kc, key);
+          if (rank < ns) {
+            chunks[rank] = key_id(key);
+            ckey[rank] = key;
+          }
+        }
+      }
+    }
     named_sync(kBarStream, W * 32);  // B2
 
-    // ---- level 2: this warp's chosen chunks' group rows (then its window units
-    // queue behind them and land while the selection runs)
-    issue_upto(e_rt);
-    consume(e_l2, e_fw, e_rt, [&](int i, uint8_t* st) {
-      const float sc = score16(reinterpret_cast<const float*>(st), qv);
-      const int k0 = (i - e_l2) * cpu;
-      const int rows = (min(n_mine, k0 + cpu) - k0) * p.Ng;
-      if (lane < rows) {
-        const int e = warp + (k0 + lane / p.Ng) * W;  // chosen chunk (rank order)
-        const int g = lane % p.Ng;
-        gkey[e * p.Ng + g] = make_key(sc, chunks[e] * p.Ng + g);
-      }
-    });
-    named_sync(kBarStream, W * 32);  // B3
-    // the kg best group keys, by rank, into glist (rank order)
-    for (int j = tid; j < n_l2; j += W * 32) {
-      const uint64_t key = gkey[j];
-      const int rank = rank_among(gkey, n_l2, key);
-      if (rank < ng) {
-        glist[rank] = key_id(key);
-        gsc[rank] = key_score(key);
-      }
-    }
-    named_sync(kBarStream, W * 32);  // B4
-
-    // ---- window and routed units
     WarpState ws;
-    ws.init();
     int attended = 0;
-    issue_upto(e_all);
-    if (warp == 0) {  // outputs, ascending ids, while the units load
-      int32_t* cidx = a.chunk_idx + static_cast<size_t>(item) * p.kc;
-      float* cscore = a.chunk_score ? a.chunk_score + static_cast<size_t>(item) * p.kc : nullptr;
-      for (int e = lane; e < p.kc; e += 32) {
-        if (e < ns) {
-          const int id = chunks[e];
-          int at = 0;
-          for (int f = 0; f < ns; ++f) at += chunks[f] < id;
-          cidx[at] = id;
-          if (cscore) cscore[at] = key_score(ckey[e]);
-        } else {
-          cidx[e] = -1;
-          if (cscore) cscore[e] = CUDART_NAN_F;
-        }
-      }
-      int32_t* gidx = a.group_idx + static_cast<size_t>(item) * p.kg;
-      float* gscore = a.group_score ? a.group_score + static_cast<size_t>(item) * p.kg : nullptr;
-      for (int e = lane; e < p.kg; e += 32) {
-        if (e < ng) {
-          const int id = glist[e];
-          int at = 0;
-          for (int f = 0; f < ng; ++f) at += glist[f] < id;
-          gidx[at] = id;
-          if (gscore) gscore[at] = gsc[e];
-        } else {
-          gidx[e] = -1;
-          if (gscore) gscore[e] = CUDART_NAN_F;
-        }
-      }
-    }
-    consume(e_fw, e_all, e_all, [&](int i, uint8_t* st) {
+    // attends one landed K/V unit of stream position i (window units may end at the query)
+    auto attend_fn = [&](int i, uint8_t* st) {
       const uint32_t kt = ptx::smem_u32(st);
       int valid = kUnit;
-      if (i < e_rt && warp + (i - e_fw) * W == n_forced - 1) valid = static_cast<int>(pb % kUnit) + 1;
+      if (i < e_rt && gw + (i - e_fw) * NW == n_forced - 1) valid = static_cast<int>(pb % kUnit) + 1;
       attend_unit(kt, kt + kTileBytes, valid, qa, scale, ws);
       ++attended;
-    });
+    };
+    if (NC == 1 || crank == 0) {
+      // ---- level 2: this warp's chosen chunks' group rows (then its window units
+      // queue behind them and land while the selection runs)
+      issue_upto(e_rt);
+      consume(e_l2, e_fw, e_rt, [&](int i, uint8_t* st) {
+        const float sc = score16(reinterpret_cast<const float*>(st), qv);
+        const int k0 = (i - e_l2) * cpu;
+        const int rows = (min(n_mine, k0 + cpu) - k0) * p.Ng;
+        if (lane < rows) {
+          const int e = warp + (k0 + lane / p.Ng) * W;  // chosen chunk (rank order)
+          const int g = lane % p.Ng;
+          gkey[e * p.Ng + g] = make_key(sc, chunks[e] * p.Ng + g);
+        }
+      });
+      named_sync(kBarStream, W * 32);  // B3
+      // the kg best group keys, by rank, into glist (rank order)
+      for (int j = tid; j < n_l2; j += W * 32) {
+        const uint64_t key = gkey[j];
+        const int rank = rank_among(gkey, n_l2, key);
+        if (rank < ng) {
+          glist[rank] = key_id(key);
+          gsc[rank] = key_score(key);
+        }
+      }
+      if (NC > 1 && timed_out) s_bad[item_no & 1] = 1;  // read after B4 by warp 0
+      named_sync(kBarStream, W * 32);  // B4
+
+      if (NC > 1 && warp == 0) {  // the routed list to the other CTAs of the cluster
+        const bool bad = s_bad[item_no & 1] != 0;
+        for (int r = 1; r < NC; ++r) {
+          const uint32_t dst = ptx::map_to_rank(ptx::smem_u32(glist), r);
+          for (int i = lane; i < ng; i += 32) ptx::st_cluster(dst + 4u * i, static_cast<uint32_t>(glist[i]));
+          if (lane == 0)
+            ptx::st_cluster(ptx::map_to_rank(ptx::smem_u32(&s_ng_in), r), static_cast<uint32_t>(bad ? 0 : ng));
+        }
+        ptx::fence_cluster();
+        __syncwarp();
+        if (lane == 0)
+          for (int r = 1; r < NC; ++r) ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(&s_hand), r));
+      }
+      // ---- window and routed units
+      ws.init();
+      issue_upto(e_all);
+      if (warp == 0) {  // outputs, ascending ids, while the units load
+        int32_t* cidx = a.chunk_idx + static_cast<size_t>(item) * p.kc;
+        float* cscore = a.chunk_score ? a.chunk_score + static_cast<size_t>(item) * p.kc : nullptr;
+        for (int e = lane; e < p.kc; e += 32) {
+          if (e < ns) {
+            const int id = chunks[e];
+            int at = 0;
+            for (int f = 0; f < ns; ++f) at += chunks[f] < id;
+            cidx[at] = id;
+            if (cscore) cscore[at] = key_score(ckey[e]);
+          } else {
+            cidx[e] = -1;
+            if (cscore) cscore[e] = CUDART_NAN_F;
+          }
+        }
+        int32_t* gidx = a.group_idx + static_cast<size_t>(item) * p.kg;
+        float* gscore = a.group_score ? a.group_score + static_cast<size_t>(item) * p.kg : nullptr;
+        for (int e = lane; e < p.kg; e += 32) {
+          if (e < ng) {
+            const int id = glist[e];
+            int at = 0;
+            for (int f = 0; f < ng; ++f) at += glist[f] < id;
+            gidx[at] = id;
+            if (gscore) gscore[at] = gsc[e];
+          } else {
+            gidx[e] = -1;
+            if (gscore) gscore[e] = CUDART_NAN_F;
+          }
+        }
+      }
+      consume(e_fw, e_all, e_all, attend_fn);
+    } else {
+      // ---- the cluster's other CTAs: their window units now, their routed units on arrival
+      ws.init();
+      issue_upto(e_rt);
+      consume(e_fw, e_rt, e_rt, attend_fn);
+      int ng_in = 0;
+      if (ptx::mbar_wait_cluster(&s_hand, item_no & 1, kWaitLimit, limit_ns)) {
+        ng_in = min(s_ng_in, p.kg);
+      } else {
+        timed_out = true;
+      }
+      e_all = e_rt + count(ng_in);
+      issue_upto(e_all);
+      consume(e_rt, e_all, e_all, attend_fn);
+    }
     bool drained = true;
     if (timed_out) {
       // A wait gave up: the partial is dropped (the output is wrong and flagged),
@@ -656,7 +752,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
       // barrier below is still reached.  Later items of this CTA are skipped.
       if (lane == 0) {
         flag_error(a.err, kErrTimeout);
-        s_abort = 1;
+        if (NC == 1) s_abort = 1;
       }
       for (; done < issued; ++done) drained &= wait_stage(done);
       ws.m0 = ws.m1 = -CUDART_INF_F;
@@ -691,6 +787,11 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
       s_ml[warp][g + 8][1] = ws.l1;
     }
     named_sync(kBarStream, W * 32);
+    if (NC > 1 && crank == 0 &&
+        !ptx::mbar_wait_cluster(&s_peerbar, item_no & 1, kWaitLimit, limit_ns) && lane == 0)
+      flag_error(a.err, kErrTimeout);  // a partial did not come: flagged
+    // peer layout: o [NC][G][kD], then (m, l) [NC][G]
+    const uint32_t peer0 = NC > 1 && crank > 0 ? ptx::map_to_rank(ptx::smem_u32(peer), 0) : 0u;
     for (int idx = tid; idx < p.G * kD; idx += W * 32) {
       const int hh = idx / kD, d = idx % kD;
       float mm = -CUDART_INF_F;
@@ -708,16 +809,45 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k,
                     [hh * kD + (d ^ ((hh & 7) << 3))] * f;
         }
       }
+      if (NC > 1 && crank > 0) {  // this CTA's partial, to rank 0
+        ptx::st_cluster(peer0 + 4u * ((crank * p.G + hh) * kD + d), __float_as_uint(oo));
+        if (d == 0) {
+          const uint32_t ml = peer0 + 4u * (NC * p.G * kD + 2 * (crank * p.G + hh));
+          ptx::st_cluster(ml, __float_as_uint(mm));
+          ptx::st_cluster(ml + 4u, __float_as_uint(ll));
+        }
+        continue;
+      }
+      for (int r = 1; r < NC; ++r) {  // rank 0: the other CTAs' partials, by log-sum-exp
+        const float pm = peer[NC * p.G * kD + 2 * (r * p.G + hh)];
+        const float pl = peer[NC * p.G * kD + 2 * (r * p.G + hh) + 1];
+        const float po = peer[(r * p.G + hh) * kD + d];
+        const float mx = fmaxf(mm, pm);
+        if (mx != -CUDART_INF_F) {
+          const float f0 = mm == -CUDART_INF_F ? 0.f : exp2f(mm - mx);
+          const float f1 = pm == -CUDART_INF_F ? 0.f : exp2f(pm - mx);
+          ll = ll * f0 + pl * f1;
+          oo = oo * f0 + po * f1;
+          mm = mx;
+        }
+      }
       const size_t row = static_cast<size_t>(b) * p.Hq + h * p.G + hh;
       store_out(a.out + row * kD + d, ll > 0.f ? oo / ll : 0.f);
       if (a.lse && d == 0) a.lse[row] = ll > 0.f ? (mm + log2f(ll)) * kLn2 : -CUDART_INF_F;
     }
+    if (NC > 1 && crank > 0) {  // the partial is in rank 0's shared memory: say so
+      ptx::fence_cluster();
+      named_sync(kBarStream, W * 32);
+      if (tid == 0) ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(&s_peerbar), 0));
+    }
+    if (NC > 1 && tid == 0) s_bad[(item_no + 1) & 1] = 0;  // the next item's flag, before its writes
     // the rings and the lists are reused by the next item (its copies are
     // ordered after this item's shared-memory writes)
     ptx::fence_proxy_async();
     named_sync(kBarStream, W * 32);
   }
   cta_sync();
+  if (NC > 1) ptx::cluster_barrier();  // no CTA leaves while another may still write to it
   pdl_trigger();
 }
 
@@ -727,41 +857,65 @@ struct StepShape {
   int W;           // streaming warps per CTA (7: one CTA per SM; 3: two per SM), plus one append warp
   int R1;          // key registers per lane of the level-1 lists (top-kc <= 32 R1)
   int grid;
+  int nc;          // CTAs per item (a cluster): small batches spread each item over nc SMs
 };
 
-StepShape step_shape(const LayerParams& p) {
+size_t step_smem_bytes(const LayerParams& p, int W, int n_pt, int nc) {
+  return StepSmem{W, summ::table_entries(p, kD), n_pt, nc > 1 ? nc * p.G * (kD + 2) : 0}.bytes();
+}
+
+// More items than SMs: three-warp CTAs, two per SM.  Up to one item per SM: one
+// seven-warp CTA per SM, and when at most half the SMs would be busy, each item
+// on a cluster of nc CTAs (the largest of 8, 4, 2 that keeps one CTA per SM and
+// fits the shared memory of n_pt staged block-table entries).
+StepShape step_shape(const LayerParams& p, int n_pt) {
   const int64_t items = static_cast<int64_t>(p.B) * p.Hkv;
   const int sms = device_sm_count();
   StepShape s;
   s.W = items <= sms ? 7 : 3;
   s.R1 = p.kc <= 32 ? 1 : 2;
+  s.nc = 1;
+  if (s.W == 7)
+    for (int nc = 8; nc >= 2; nc /= 2)
+      if (items * nc <= sms && step_smem_bytes(p, 7, n_pt, nc) <= 225 * 1024) {
+        s.nc = nc;
+        break;
+      }
   const int64_t slots = static_cast<int64_t>(sms) * (s.W == 7 ? 1 : 2);
-  s.grid = static_cast<int>(items < slots ? items : slots);
+  s.grid = s.nc > 1 ? static_cast<int>(items * s.nc)
+                    : static_cast<int>(items < slots ? items : slots);
   return s;
 }
 
-size_t step_smem_bytes(const LayerParams& p, int W, int n_pt) {
-  return StepSmem{W, summ::table_entries(p, kD), n_pt}.bytes();
+template <int W, int R1, typename TO, bool PAGED, int NC>
+cudaError_t launch_t(const LayerParams& p, int grid, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const StepArgs<TO>& a, cudaStream_t s) {
+  const size_t smem = step_smem_bytes(p, W, PAGED ? a.kv.max_pages : 0, NC);
+  cudaError_t e = ensure_smem<decode_step_kernel<W, R1, TO, PAGED, NC>>(smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_step_kernel<W, R1, TO, PAGED, NC>, dim3(grid), dim3((W + 1) * 32), smem,
+                    s, NC, tk, tv, a, p);
 }
 
 template <int W, int R1, typename TO, bool PAGED>
-cudaError_t launch_t(const LayerParams& p, int grid, const CUtensorMap& tk, const CUtensorMap& tv,
-                     const StepArgs<TO>& a, cudaStream_t s) {
-  const size_t smem = step_smem_bytes(p, W, PAGED ? a.kv.max_pages : 0);
-  cudaError_t e = ensure_smem<decode_step_kernel<W, R1, TO, PAGED>>(smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(decode_step_kernel<W, R1, TO, PAGED>, dim3(grid), dim3((W + 1) * 32), smem, s,
-                    1, tk, tv, a, p);
+cudaError_t launch_nc(const LayerParams& p, const StepShape& sh, const CUtensorMap& tk,
+                      const CUtensorMap& tv, const StepArgs<TO>& a, cudaStream_t s) {
+  switch (sh.nc) {
+    case 8: return launch_t<W, R1, TO, PAGED, 8>(p, sh.grid, tk, tv, a, s);
+    case 4: return launch_t<W, R1, TO, PAGED, 4>(p, sh.grid, tk, tv, a, s);
+    case 2: return launch_t<W, R1, TO, PAGED, 2>(p, sh.grid, tk, tv, a, s);
+    default: return launch_t<W, R1, TO, PAGED, 1>(p, sh.grid, tk, tv, a, s);
+  }
 }
 
 template <typename TO, bool PAGED>
 cudaError_t dispatch(const LayerParams& p, const StepShape& sh, const CUtensorMap& tk,
                      const CUtensorMap& tv, const StepArgs<TO>& a, cudaStream_t s) {
   if (sh.W == 7)
-    return sh.R1 == 1 ? launch_t<7, 1, TO, PAGED>(p, sh.grid, tk, tv, a, s)
-                      : launch_t<7, 2, TO, PAGED>(p, sh.grid, tk, tv, a, s);
-  return sh.R1 == 1 ? launch_t<3, 1, TO, PAGED>(p, sh.grid, tk, tv, a, s)
-                    : launch_t<3, 2, TO, PAGED>(p, sh.grid, tk, tv, a, s);
+    return sh.R1 == 1 ? launch_nc<7, 1, TO, PAGED>(p, sh, tk, tv, a, s)
+                      : launch_nc<7, 2, TO, PAGED>(p, sh, tk, tv, a, s);
+  return sh.R1 == 1 ? launch_t<3, 1, TO, PAGED, 1>(p, sh.grid, tk, tv, a, s)
+                    : launch_t<3, 2, TO, PAGED, 1>(p, sh.grid, tk, tv, a, s);
 }
 
 template <typename TO>
@@ -774,11 +928,11 @@ cudaError_t dispatch_kv(const LayerParams& p, const StepShape& sh, const CUtenso
 }  // namespace
 
 bool decode_item_path(const LayerParams& p, int n_pt) {
-  const StepShape sh = step_shape(p);
+  const StepShape sh = step_shape(p, n_pt);
   // dynamic shared memory: one CTA per SM may take 225 KB, two per SM 112 KB each
   const size_t limit = sh.W == 7 ? 225 * 1024 : 112 * 1024;
   return p.kc <= kKcMax && p.kg <= kKgMax && p.Ng <= 8 &&
-         kRows % p.Ng == 0 && step_smem_bytes(p, sh.W, n_pt) <= limit;
+         kRows % p.Ng == 0 && step_smem_bytes(p, sh.W, n_pt, sh.nc) <= limit;
 }
 
 bool decode_step_path(const LayerParams& p, int dtype) {
@@ -811,7 +965,7 @@ cudaError_t launch_decode_step(const LayerParams& p, int out_dtype, const void* 
   cudaError_t e = make_bf16_map(&tk, k, all_rows, kUnit);
   if (e == cudaSuccess) e = make_bf16_map(&tv, v, all_rows, kUnit);
   if (e != cudaSuccess) return e;
-  const StepShape sh = step_shape(p);
+  const StepShape sh = step_shape(p, paged ? kv.max_pages : 0);
   const int n_items = p.B * p.Hkv;
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);

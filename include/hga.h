@@ -383,7 +383,10 @@ hga_status hga_attend(const hga_config* cfg, const void* q, int32_t q_len, const
  *
  * With topk_chunks <= 64 and topk_groups <= 128 the step is one launch: each
  * CTA works through (sequence, KV head) items, one at a time (one CTA per SM up
- * to one item per SM, two per SM above); its warps stream the candidate chunk
+ * to one item per SM, two per SM above; when at most half the SMs would be
+ * busy, each item is spread over a cluster of 2, 4 or 8 CTAs that scan slices
+ * of the candidates, gather their selections in the first CTA and merge their
+ * partials there); its warps stream the candidate chunk
  * summaries and the K/V of the always-visible chunks through shared-memory
  * rings, select the chunks and then the groups between barriers, attend the
  * routed groups and merge their partials, while another warp does the summary

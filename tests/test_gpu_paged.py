@@ -126,12 +126,14 @@ def _closed_rows_equal(batch, upto):
 RAGGED = [8191, 5000, 40 * 64 + 17, 1023, 7777, 4095, 64 * 3 - 1, 2 * 64 * 16 - 1]
 
 
-@pytest.mark.parametrize("page,many", [(16, False), (64, False), (256, False), (32, True)])
+@pytest.mark.parametrize("page,many", [(16, 0), (64, 0), (256, 0), (32, 20), (64, 16)])
 def test_paged_step_is_bitwise_the_dense_step(page, many):
-    """many: 20 sequences x 8 KV heads, more items than SMs (two CTAs per SM)."""
+    """many = 20: 20 sequences x 8 KV heads, more items than SMs (two CTAs per SM);
+    many = 16: 128 items, one CTA each; else 8 sequences (each item on a cluster of
+    CTAs)."""
     if many:
-        pos = np.random.default_rng(4).integers(100, 4096, 20)
-        wl = S.workload("llama3_8b_decode_32k", batch=20, context=4096)
+        pos = np.random.default_rng(4).integers(100, 4096, many)
+        wl = S.workload("llama3_8b_decode_32k", batch=many, context=4096)
     else:
         pos = RAGGED
         wl = S.workload("llama3_8b_decode_32k", batch=len(RAGGED), context=8192)

@@ -864,6 +864,13 @@ size_t step_smem_bytes(const LayerParams& p, int W, int n_pt, int nc) {
   return StepSmem{W, summ::table_entries(p, kD), n_pt, nc > 1 ? nc * p.G * (kD + 2) : 0}.bytes();
 }
 
+// Dynamic shared memory a CTA may take: 225 KB with one CTA per SM, 112 KB with
+// two, less the static slice lists that a cluster of nc CTAs adds (the CTA's
+// whole shared memory stays within the 227 KB a block may have).
+size_t step_smem_limit(int W, int nc) {
+  return (W == 7 ? 225 * 1024 : 112 * 1024) - static_cast<size_t>(nc - 1) * kKcMax * 8;
+}
+
 // More items than SMs: three-warp CTAs, two per SM.  Up to one item per SM: one
 // seven-warp CTA per SM, and when at most half the SMs would be busy, each item
 // on a cluster of nc CTAs (the largest of 8, 4, 2 that keeps one CTA per SM and
@@ -877,7 +884,7 @@ StepShape step_shape(const LayerParams& p, int n_pt) {
   s.nc = 1;
   if (s.W == 7)
     for (int nc = 8; nc >= 2; nc /= 2)
-      if (items * nc <= sms && step_smem_bytes(p, 7, n_pt, nc) <= 225 * 1024) {
+      if (items * nc <= sms && step_smem_bytes(p, 7, n_pt, nc) <= step_smem_limit(7, nc)) {
         s.nc = nc;
         break;
       }
@@ -929,10 +936,8 @@ cudaError_t dispatch_kv(const LayerParams& p, const StepShape& sh, const CUtenso
 
 bool decode_item_path(const LayerParams& p, int n_pt) {
   const StepShape sh = step_shape(p, n_pt);
-  // dynamic shared memory: one CTA per SM may take 225 KB, two per SM 112 KB each
-  const size_t limit = sh.W == 7 ? 225 * 1024 : 112 * 1024;
-  return p.kc <= kKcMax && p.kg <= kKgMax && p.Ng <= 8 &&
-         kRows % p.Ng == 0 && step_smem_bytes(p, sh.W, n_pt, sh.nc) <= limit;
+  return p.kc <= kKcMax && p.kg <= kKgMax && p.Ng <= 8 && kRows % p.Ng == 0 &&
+         step_smem_bytes(p, sh.W, n_pt, sh.nc) <= step_smem_limit(sh.W, sh.nc);
 }
 
 bool decode_step_path(const LayerParams& p, int dtype) {

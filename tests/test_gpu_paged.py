@@ -172,6 +172,35 @@ def test_paged_step_matches_the_oracle():
         compare_head(wl, xp, res, b, (3 * b) % wl.heads_kv)
 
 
+def test_paged_small_batch_long_block_table():
+    """One sequence at 80K tokens in 16-token pages: 5120 block-table entries staged
+    in shared memory beside a cluster's partial buffers.  The step takes a cluster
+    size whose whole shared memory (dynamic and static) a block may have, and
+    matches the dense step: the same routing and scores, bit for bit, and the
+    output up to the merge order of a different cluster size."""
+    wl = S.workload("llama3_8b_decode_32k", batch=1, context=81920)
+    x = S.make_inputs(wl, 75)
+    bt = Batch(wl, x, [81919], 16, seed=11)
+    bt.summaries()
+    bt.step("dense")
+    bt.step("paged")
+    torch.cuda.synchronize()
+    assert B.hga_device_status() == 0
+    d, p = bt.bufs["dense"], bt.bufs["paged"]
+    for name in ("ci", "gi"):
+        assert torch.equal(d[name], p[name]), name
+    for name in ("csc", "gsc"):
+        assert _same_bits(d[name], p[name]), name
+    # another cluster size deals the units to other warps, whose P is rounded to bf16
+    # against another running maximum: differences of a few 1e-5 in the output
+    torch.testing.assert_close(p["out"], d["out"], atol=1e-3, rtol=0)
+    torch.testing.assert_close(p["lse"], d["lse"], atol=1e-4, rtol=0)
+    res = dict(chunk_idx=p["ci"].cpu().numpy().reshape(wl.batch, wl.heads_kv, 1, -1),
+               group_idx=p["gi"].cpu().numpy().reshape(wl.batch, wl.heads_kv, 1, -1),
+               out=p["out"].cpu().numpy(), lse=p["lse"].cpu().numpy())
+    compare_head(wl, dict(x, pos=bt.pos), res, 0, 5)
+
+
 def test_paged_decode_loop_keeps_matching_the_dense_loop():
     """Consecutive steps with appends across group and chunk boundaries: the
     paged tables and outputs stay bitwise equal to the dense ones."""

@@ -520,10 +520,14 @@ hga_status hga_build_summaries_paged(const hga_config* cfg, const void* k_pages,
                                      float* chunk_sum, float* group_sum, void* stream);
 
 /*
- * hga_decode_step over a paged pool: the same outputs, bit for bit, as
- * hga_decode_step on a dense cache holding the same rows (per-sequence
+ * hga_decode_step over a paged pool: the same routing and scores, bit for bit,
+ * as hga_decode_step on a dense cache holding the same rows (per-sequence
  * positions pos[b] < n_alloc = kv->max_pages * kv->page_size; the summary
- * append reads the closed group's rows through the block table).  One launch
+ * append reads the closed group's rows through the block table), and the same
+ * output bits when both split the work alike.  (For a batch of at most half as
+ * many items as SMs, a long block-table row can leave room for fewer CTAs per
+ * item than the dense step takes; the output then differs by the bf16
+ * rounding of the attention weights, a few 1e-5.)  One launch
  * of the decode-step kernel, which stages each sequence's block-table row in
  * shared memory; shapes it cannot take (hga_decode_step_launches would say 2,
  * or the block-table row does not fit beside the kernel's buffers) return

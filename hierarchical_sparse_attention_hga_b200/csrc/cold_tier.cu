@@ -16,6 +16,7 @@
 #include <atomic>
 #include <cerrno>
 #include <cstring>
+#include <system_error>
 #include <thread>
 #include <vector>
 
@@ -40,7 +41,9 @@ std::string full_io(int fd, void* buf, int64_t bytes, int64_t off, bool write) {
   return "";
 }
 
-// Runs fn(u) for u in [0, units) on up to `threads` threads; the first error wins.
+// Runs fn(u) for u in [0, units) on up to `threads` threads (the calling one
+// included; if the system refuses a thread, the ones started share the units);
+// the first error wins.
 template <typename Fn>
 std::string parallel_units(int64_t units, int threads, Fn fn) {
   const int nt = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(threads, units)));
@@ -56,13 +59,13 @@ std::string parallel_units(int64_t units, int threads, Fn fn) {
       }
     }
   };
-  if (nt == 1) {
-    work(0);
-  } else {
-    std::vector<std::thread> pool;
-    for (int w = 0; w < nt; ++w) pool.emplace_back(work, w);
-    for (auto& t : pool) t.join();
+  std::vector<std::thread> pool;
+  try {
+    for (int w = 1; w < nt; ++w) pool.emplace_back(work, w);
+  } catch (const std::system_error&) {
   }
+  work(0);
+  for (auto& t : pool) t.join();
   for (auto& e : errs)
     if (!e.empty()) return e;
   return "";
@@ -72,7 +75,7 @@ std::string parallel_units(int64_t units, int threads, Fn fn) {
 
 std::string cold_open(const char* path, int64_t units, int64_t n_alloc, int64_t row_bytes,
                       bool create, ColdStore* out) {
-  const int fd = ::open(path, create ? (O_RDWR | O_CREAT) : O_RDWR, 0644);
+  const int fd = ::open(path, O_RDWR | O_CLOEXEC | (create ? O_CREAT : 0), 0644);
   if (fd < 0) return std::string("open ") + path + ": " + std::strerror(errno);
   const int64_t need = 2 * units * n_alloc * row_bytes;
   struct stat st;
